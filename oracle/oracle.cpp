@@ -1,0 +1,307 @@
+// CPU oracle for the routed int4 expert layer -- TEST INFRASTRUCTURE ONLY.
+//
+// A plain, slow, single-threaded restatement of what the layer computes, used
+// to check the CUDA library.  Only the tests, the smoke check and the
+// benchmark's CPU-baseline leg may load it; the library itself never does.
+// It shares no code with the CUDA path (its own format reader, its own fp16
+// decoder, its own routing), and nothing here is blocked, fused or reordered
+// beyond what the definition states.
+//
+// What it computes, and the passages it follows:
+//  * Routing: "route each token to its top-k experts" with an fp32 router
+//    GEMV, softmax, top-k with lowest-index tie-break and renormalisation
+//    (the layer statement this library implements; the fused router dispatch
+//    of Strata "docs/MAC.md", section "Switches", two opt-ins paragraph).
+//    Reading taken where the pages are silent: products x*W are exact in
+//    double and are summed in double in ascending h order, the bias is added
+//    in double, the sum is rounded once to an fp32 logit; top-k compares the
+//    fp32 logits; softmax is fp32 with max subtraction over all experts; the
+//    selected probabilities are divided by their sum.
+//  * Expert lookup through a slot table ("routed experts ... leased into VRAM
+//    per decode step through an LRU cache", ro99/strata README, "Residency").
+//  * Expert FFN on W4A16 weights ("INT4 ... W4A16 execution", ro99/strata
+//    README, model table): w = float(fp16 scale) * q, exact in fp32; gate and
+//    up dot products in fp32 in ascending K; h = silu(g) * u with
+//    silu(z) = z / (1 + exp(-z)) in fp32; down projection in fp32 ascending K.
+//  * Combine: out[t] = sum_j w[t][j] * y[t][j] (j = 0..k-1, descending logit)
+//    followed by + y_shared[t][s] (s = 0..S-1), fp32, in that fixed order
+//    (a fixed order is what the bit-exact fidelity tier of
+//    strata.amperor.ai "/methods/", "Fidelity (paged vs resident output)",
+//    requires).
+//
+// Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -shared -fPIC.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <utility>
+#include <vector>
+
+namespace {
+
+enum {
+  ORC_OK = 0,
+  ORC_BAD_ARG = 1,
+  ORC_NOT_BOUND = 2,
+  ORC_SLOT_CONFLICT = 3,
+};
+
+size_t round_up_256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Section offsets of one expert blob, in bytes from its start.
+struct Layout {
+  size_t gq, uq, dq, gs, us, ds, total;
+};
+
+Layout layout_of(int H, int I) {
+  Layout L;
+  size_t off = 0;
+  L.gq = off; off = round_up_256(off + (size_t)I * H / 2);
+  L.uq = off; off = round_up_256(off + (size_t)I * H / 2);
+  L.dq = off; off = round_up_256(off + (size_t)H * I / 2);
+  L.gs = off; off = round_up_256(off + (size_t)I * (H / 32) * 2);
+  L.us = off; off = round_up_256(off + (size_t)I * (H / 32) * 2);
+  L.ds = off; off = round_up_256(off + (size_t)H * (I / 32) * 2);
+  L.total = off;
+  return L;
+}
+
+// bfloat16 bits -> float: the top 16 bits of an IEEE binary32.
+float bf16_value(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+// IEEE binary16 bits -> float, from the definition of the format:
+// sign, 5-bit exponent (bias 15), 10-bit fraction; subnormals have exponent
+// field 0 and value 2^-14 * fraction / 1024.
+float f16_value(uint16_t bits) {
+  int sign = (bits >> 15) & 1;
+  int expo = (bits >> 10) & 0x1F;
+  int frac = bits & 0x3FF;
+  double v;
+  if (expo == 0) {
+    v = std::ldexp((double)frac, -24);
+  } else if (expo == 31) {
+    v = frac ? NAN : INFINITY;
+  } else {
+    v = std::ldexp(1.0 + frac / 1024.0, expo - 15);
+  }
+  return (float)(sign ? -v : v);
+}
+
+// Element `col` of a packed int4 row: byte col/2, low nibble for even col,
+// high nibble for odd col, two's complement.
+int int4_at(const uint8_t *row, int col) {
+  uint8_t byte = row[col / 2];
+  int n = (col % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+  return n >= 8 ? n - 16 : n;
+}
+
+// One dequantised row of a [rows][K] int4 matrix with [rows][K/32] scales.
+void dequant_row(const uint8_t *q, const uint16_t *s, int K, int row, float *out) {
+  const uint8_t *qr = q + (size_t)row * (K / 2);
+  const uint16_t *sr = s + (size_t)row * (K / 32);
+  for (int c = 0; c < K; ++c) out[c] = f16_value(sr[c / 32]) * (float)int4_at(qr, c);
+}
+
+float silu(float z) { return z / (1.0f + std::exp(-z)); }
+
+// y[n][H] = FFN(x[n][H]) for n tokens through one expert blob.
+// Optional g, u, h outputs are [n][I].
+void expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
+                float *g_out, float *u_out, float *h_out, float *y) {
+  Layout L = layout_of(H, I);
+  const uint8_t *gq = blob + L.gq, *uq = blob + L.uq, *dq = blob + L.dq;
+  const uint16_t *gs = (const uint16_t *)(blob + L.gs);
+  const uint16_t *us = (const uint16_t *)(blob + L.us);
+  const uint16_t *ds = (const uint16_t *)(blob + L.ds);
+  std::vector<float> wg(H), wu(H), wd(I), h((size_t)n * I);
+  for (int i = 0; i < I; ++i) {
+    dequant_row(gq, gs, H, i, wg.data());
+    dequant_row(uq, us, H, i, wu.data());
+    for (int t = 0; t < n; ++t) {
+      const float *xt = x + (size_t)t * H;
+      float g = 0.0f, u = 0.0f;
+      for (int c = 0; c < H; ++c) {
+        g = g + wg[c] * xt[c];
+        u = u + wu[c] * xt[c];
+      }
+      float hv = silu(g) * u;
+      h[(size_t)t * I + i] = hv;
+      if (g_out) g_out[(size_t)t * I + i] = g;
+      if (u_out) u_out[(size_t)t * I + i] = u;
+      if (h_out) h_out[(size_t)t * I + i] = hv;
+    }
+  }
+  for (int r = 0; r < H; ++r) {
+    dequant_row(dq, ds, I, r, wd.data());
+    for (int t = 0; t < n; ++t) {
+      const float *ht = h.data() + (size_t)t * I;
+      float acc = 0.0f;
+      for (int c = 0; c < I; ++c) acc = acc + wd[c] * ht[c];
+      y[(size_t)t * H + r] = acc;
+    }
+  }
+}
+
+// Blob bound to expert e in the slot table, or nullptr.
+const uint8_t *lookup(const int32_t *slot_expert, const uint8_t *const *slot_blob,
+                      int n_slots, int e) {
+  for (int s = 0; s < n_slots; ++s)
+    if (slot_expert[s] == e && slot_blob[s]) return slot_blob[s];
+  return nullptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t oracle_expert_bytes(int H, int I) { return layout_of(H, I).total; }
+
+// Router for T tokens.  x: bf16 bits [T][H]; Wr: fp32 [E][H]; bias: fp32 [E]
+// or null.  Outputs: logits fp32 [T][E] (may be null), idx [T][k], w [T][k].
+int oracle_route(const uint16_t *x, int T, int H, const float *Wr, const float *bias,
+                 int E, int k, float *logits, int32_t *idx, float *w) {
+  if (T < 0 || H <= 0 || E <= 0 || k <= 0 || k > E) return ORC_BAD_ARG;
+  std::vector<float> l(E), p(E);
+  std::vector<char> taken(E);
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += (double)bf16_value(x[(size_t)t * H + h]) * (double)Wr[(size_t)e * H + h];
+      if (bias) acc += (double)bias[e];
+      l[e] = (float)acc;
+      if (logits) logits[(size_t)t * E + e] = l[e];
+    }
+    // top-k: repeatedly take the largest remaining logit; a strict comparison
+    // keeps the lowest index among equal logits.
+    std::fill(taken.begin(), taken.end(), 0);
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e)
+        if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+      taken[best] = 1;
+      idx[(size_t)t * k + j] = best;
+    }
+    // softmax over all experts (fp32, max subtracted), then renormalise the
+    // selected probabilities.
+    float m = l[0];
+    for (int e = 1; e < E; ++e) m = l[e] > m ? l[e] : m;
+    float Z = 0.0f;
+    for (int e = 0; e < E; ++e) {
+      p[e] = std::exp(l[e] - m);
+      Z = Z + p[e];
+    }
+    for (int e = 0; e < E; ++e) p[e] = p[e] / Z;
+    float sel = 0.0f;
+    for (int j = 0; j < k; ++j) sel = sel + p[idx[(size_t)t * k + j]];
+    for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = p[idx[(size_t)t * k + j]] / sel;
+  }
+  return ORC_OK;
+}
+
+// One expert on n tokens given as fp32 activations.  Any of g, u, h may be
+// null; y is [n][H].
+int oracle_expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
+                      float *g, float *u, float *h, float *y) {
+  if (!blob || H <= 0 || I <= 0 || H % 32 || I % 32 || n < 0) return ORC_BAD_ARG;
+  expert_ffn(blob, H, I, x, n, g, u, h, y);
+  return ORC_OK;
+}
+
+// Layer output for T tokens with routing given.  Experts are found through
+// the slot table (slot s holds expert slot_expert[s] at slot_blob[s]; -1 or a
+// null blob = empty).  out: fp32 [T][H].  A token whose routed expert is not
+// bound gets a zero output row and the call returns ORC_NOT_BOUND.
+int oracle_forward_routed(const uint16_t *x, int T, int H, int I, int E, int k, int S,
+                          const int32_t *slot_expert, const uint8_t *const *slot_blob,
+                          int n_slots, const uint8_t *const *shared_blob,
+                          const int32_t *idx, const float *w, float *out) {
+  if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || S < 0 || n_slots < 0)
+    return ORC_BAD_ARG;
+  if (H % 32 || I % 32) return ORC_BAD_ARG;
+  // the same expert in two slots is a conflict
+  for (int a = 0; a < n_slots; ++a)
+    for (int b = a + 1; b < n_slots; ++b)
+      if (slot_expert[a] >= 0 && slot_expert[a] == slot_expert[b]) return ORC_SLOT_CONFLICT;
+  int status = ORC_OK;
+  std::vector<float> xf((size_t)T * H);
+  for (size_t i = 0; i < xf.size(); ++i) xf[i] = bf16_value(x[i]);
+  // y[t][j] for j < k + S, computed expert by expert (each expert's weights
+  // are decoded once and applied to every token routed to it).
+  std::vector<float> y((size_t)T * (k + S) * H, 0.0f);
+  std::vector<char> token_ok(T, 1);
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) return ORC_BAD_ARG;
+      if (!lookup(slot_expert, slot_blob, n_slots, e)) token_ok[t] = 0;
+    }
+  std::vector<float> xin, yout;
+  for (int e = 0; e < E + S; ++e) {
+    std::vector<std::pair<int, int>> uses;  // (t, j)
+    for (int t = 0; t < T; ++t) {
+      if (!token_ok[t]) continue;
+      if (e < E) {
+        for (int j = 0; j < k; ++j)
+          if (idx[(size_t)t * k + j] == e) uses.push_back({t, j});
+      } else {
+        uses.push_back({t, k + (e - E)});
+      }
+    }
+    if (uses.empty()) continue;
+    const uint8_t *blob = e < E ? lookup(slot_expert, slot_blob, n_slots, e) : shared_blob[e - E];
+    if (!blob) return ORC_BAD_ARG;  // a shared expert must be given
+    int n = (int)uses.size();
+    xin.assign((size_t)n * H, 0.0f);
+    yout.assign((size_t)n * H, 0.0f);
+    for (int a = 0; a < n; ++a)
+      std::memcpy(&xin[(size_t)a * H], &xf[(size_t)uses[a].first * H], sizeof(float) * H);
+    expert_ffn(blob, H, I, xin.data(), n, nullptr, nullptr, nullptr, yout.data());
+    for (int a = 0; a < n; ++a)
+      std::memcpy(&y[((size_t)uses[a].first * (k + S) + uses[a].second) * H],
+                  &yout[(size_t)a * H], sizeof(float) * H);
+  }
+  for (int t = 0; t < T; ++t) {
+    float *o = out + (size_t)t * H;
+    for (int r = 0; r < H; ++r) o[r] = 0.0f;
+    if (!token_ok[t]) {
+      status = ORC_NOT_BOUND;
+      continue;
+    }
+    for (int j = 0; j < k; ++j) {
+      float wj = w[(size_t)t * k + j];
+      const float *yj = &y[((size_t)t * (k + S) + j) * H];
+      for (int r = 0; r < H; ++r) o[r] = o[r] + wj * yj[r];
+    }
+    for (int s = 0; s < S; ++s) {
+      const float *ys = &y[((size_t)t * (k + S) + k + s) * H];
+      for (int r = 0; r < H; ++r) o[r] = o[r] + ys[r];
+    }
+  }
+  return status;
+}
+
+// Router followed by the routed layer.  idx/w/logits outputs may be null.
+int oracle_forward(const uint16_t *x, int T, int H, int I, int E, int k, int S,
+                   const float *Wr, const float *bias, const int32_t *slot_expert,
+                   const uint8_t *const *slot_blob, int n_slots,
+                   const uint8_t *const *shared_blob, float *logits, int32_t *idx_out,
+                   float *w_out, float *out) {
+  if (T < 0 || k <= 0 || k > E) return ORC_BAD_ARG;
+  std::vector<int32_t> idx((size_t)T * k);
+  std::vector<float> w((size_t)T * k);
+  int st = oracle_route(x, T, H, Wr, bias, E, k, logits, idx.data(), w.data());
+  if (st != ORC_OK) return st;
+  if (idx_out) std::memcpy(idx_out, idx.data(), sizeof(int32_t) * idx.size());
+  if (w_out) std::memcpy(w_out, w.data(), sizeof(float) * w.size());
+  return oracle_forward_routed(x, T, H, I, E, k, S, slot_expert, slot_blob, n_slots,
+                               shared_blob, idx.data(), w.data(), out);
+}
+
+}  // extern "C"

@@ -1,0 +1,237 @@
+"""Seeded synthetic inputs for the routed int4 expert layer.
+
+This module draws inputs and packs them into the expert-blob format; it holds
+none of the layer's arithmetic (no routing, no dequantisation, no matmul).  It
+is the one module that both the CPU oracle's tests and the CUDA path's tests
+and benchmarks use, so that both sides see byte-identical inputs.
+
+Workloads (shapes, distributions) follow the five layer configurations of the
+problem statement: a tiny layer, a DeepSeek-V2-Lite-shaped decode layer, a
+Mixtral-shaped decode layer, a 256-expert "wide" decode layer with a 64-slot
+arena, and a 256-expert prefill layer.  The pages (Strata "docs/MAC.md",
+"Strata on a Mac"; ro99/strata README, "Residency" and "Kernels") describe the
+same problem on real checkpoints; nothing here reads a checkpoint.
+
+Expert blob format (one contiguous blob per expert, after Strata "docs/MAC.md",
+which keeps "each expert's three matrices together"):
+
+    section   shape            type
+    Wg_q      [I][H/2]         u8   gate weights, 2 int4 per byte
+    Wu_q      [I][H/2]         u8   up weights
+    Wd_q      [H][I/2]         u8   down weights
+    Wg_s      [I][H/32]        f16  one scale per 32 consecutive K elements
+    Wu_s      [I][H/32]        f16
+    Wd_s      [H][I/32]        f16
+
+Each section starts at a multiple of 256 bytes from the blob start and the
+blob size is rounded up to 256 bytes.  Byte j of a row holds element 2j in its
+low nibble and element 2j+1 in its high nibble; a nibble is a two's-complement
+int4 in [-8, 7].  The dequantised weight is float(scale) * q.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+QBLOCK = 32  # K elements per fp16 scale
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerConfig:
+    name: str
+    hidden: int
+    inter: int
+    n_experts: int
+    top_k: int
+    n_shared: int
+    n_slots: int
+    tokens: tuple
+    bias: str = "none"          # "none" | "normal" | "zipf"
+    bias_var: float = 0.0       # variance of the normal bias
+    zipf_s: float = 0.0         # Zipf exponent of the bias
+    zipf_beta: float = 1.0      # multiplier on the Zipf log-pmf
+    description: str = ""
+
+
+# beta for the wide layer: the value at which ~80% of the routed hits of the
+# seed-0 tokens land in the 64 highest-ranked experts (checked by
+# tests/test_oracle_pins.py::test_wide_zipf_share; derived by
+# tests/golden/calibrate_zipf_beta.py, which calls only the oracle).
+WIDE_ZIPF_BETA = 0.5390625
+
+CONFIGS = {
+    "tiny": LayerConfig(
+        "tiny", 256, 512, 8, 2, 0, 8, (4,),
+        description="hidden 256, inter 512, 8 experts top-2, 8 slots bound in "
+                    "shuffled order, 4 tokens"),
+    "dsv2lite": LayerConfig(
+        "dsv2lite", 2048, 1408, 64, 6, 2, 64, (1, 8), bias="normal", bias_var=0.5,
+        description="DeepSeek-V2-Lite-shaped decode: hidden 2048, inter 1408, 64 "
+                    "experts top-6 + 2 shared, per-expert router bias ~N(0,0.5)"),
+    "mixtral": LayerConfig(
+        "mixtral", 4096, 14336, 8, 2, 0, 8, (1, 4, 16),
+        description="Mixtral-shaped decode: hidden 4096, inter 14336, 8 experts "
+                    "top-2"),
+    "wide": LayerConfig(
+        "wide", 4096, 1024, 256, 10, 0, 64, (1, 4), bias="zipf", zipf_s=1.1,
+        zipf_beta=WIDE_ZIPF_BETA,
+        description="wide-expert decode: hidden 4096, inter 1024, 256 experts "
+                    "top-10, 64-slot arena, Zipf(1.1) router bias"),
+    "prefill": LayerConfig(
+        "prefill", 4096, 2048, 256, 8, 1, 256, (8192,), bias="zipf", zipf_s=0.8,
+        zipf_beta=1.0,
+        description="prefill: hidden 4096, inter 2048, 256 experts top-8 + 1 "
+                    "shared, 8192 tokens, Zipf(0.8) router bias"),
+}
+
+
+def custom_config(name, hidden, inter, n_experts, top_k, n_shared=0, n_slots=None,
+                  tokens=(4,), bias="none", bias_var=0.0, zipf_s=0.0, zipf_beta=1.0):
+    """A config with the same distributions at other sizes (tests, edge cases)."""
+    return LayerConfig(name, hidden, inter, n_experts, top_k, n_shared,
+                       n_experts if n_slots is None else n_slots, tuple(tokens),
+                       bias, bias_var, zipf_s, zipf_beta)
+
+
+# ----------------------------------------------------------------------------
+# format helpers (layout only; no arithmetic of the layer)
+
+def _align256(v: int) -> int:
+    return (v + 255) // 256 * 256
+
+
+def blob_layout(hidden: int, inter: int) -> dict:
+    """Byte offsets of the six sections and the blob size."""
+    H, I = hidden, inter
+    sizes = [("gq", I * H // 2), ("uq", I * H // 2), ("dq", H * I // 2),
+             ("gs", I * (H // QBLOCK) * 2), ("us", I * (H // QBLOCK) * 2),
+             ("ds", H * (I // QBLOCK) * 2)]
+    off, out = 0, {}
+    for name, size in sizes:
+        out[name] = off
+        off = _align256(off + size)
+    out["total"] = off
+    return out
+
+
+def expert_bytes(hidden: int, inter: int) -> int:
+    return blob_layout(hidden, inter)["total"]
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """int array [rows][K] with values in [-8, 7] -> u8 [rows][K/2]."""
+    q = np.asarray(q)
+    if q.min(initial=0) < -8 or q.max(initial=0) > 7:
+        raise ValueError("int4 values must lie in [-8, 7]")
+    n = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    return (n[..., 0::2] | (n[..., 1::2] << 4)).astype(np.uint8)
+
+
+def build_blob(hidden, inter, gq, uq, dq, gs, us, ds) -> np.ndarray:
+    """Assemble one expert blob from explicit int4 values and fp16 scales.
+
+    gq, uq: int [I][H]; dq: int [H][I]; gs, us: float16 [I][H/32];
+    ds: float16 [H][I/32].
+    """
+    H, I = hidden, inter
+    lay = blob_layout(H, I)
+    blob = np.zeros(lay["total"], np.uint8)
+
+    def put(name, arr):
+        raw = np.ascontiguousarray(arr).view(np.uint8).reshape(-1)
+        blob[lay[name]:lay[name] + raw.size] = raw
+
+    put("gq", pack_int4(np.asarray(gq).reshape(I, H)))
+    put("uq", pack_int4(np.asarray(uq).reshape(I, H)))
+    put("dq", pack_int4(np.asarray(dq).reshape(H, I)))
+    put("gs", np.asarray(gs, np.float16).reshape(I, H // QBLOCK))
+    put("us", np.asarray(us, np.float16).reshape(I, H // QBLOCK))
+    put("ds", np.asarray(ds, np.float16).reshape(H, I // QBLOCK))
+    return blob
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (round to nearest even); returns u16 bits."""
+    b = np.ascontiguousarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    rounded = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# seeded draws; every stream is keyed by (seed, purpose, index)
+
+_STREAM_X, _STREAM_ROUTER, _STREAM_BIAS, _STREAM_EXPERT, _STREAM_SLOTS, _STREAM_RANK = range(6)
+
+
+def _rng(seed: int, stream: int, index: int = 0) -> np.random.Generator:
+    return np.random.default_rng(np.random.SeedSequence([int(seed), stream, int(index)]))
+
+
+def make_x(cfg: LayerConfig, n_tokens: int, seed: int = 0, step: int = 0) -> np.ndarray:
+    """Token activations: bf16 (round to nearest even) of N(0,1); u16 bits [T][H]."""
+    r = _rng(seed, _STREAM_X, step)
+    return f32_to_bf16_bits(r.standard_normal((n_tokens, cfg.hidden), dtype=np.float32))
+
+
+def zipf_ranks(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
+    """Rank (1 = most popular) of every expert under the Zipf bias."""
+    r = _rng(seed, _STREAM_RANK)
+    return r.permutation(cfg.n_experts).astype(np.int64) + 1
+
+
+def make_router(cfg: LayerConfig, seed: int = 0):
+    """Router weights fp32 [E][H] ~ N(0, 1/H) and bias fp32 [E] (or None)."""
+    r = _rng(seed, _STREAM_ROUTER)
+    W = (r.standard_normal((cfg.n_experts, cfg.hidden), dtype=np.float64)
+         / math.sqrt(cfg.hidden)).astype(np.float32)
+    if cfg.bias == "none":
+        b = None
+    elif cfg.bias == "normal":
+        rb = _rng(seed, _STREAM_BIAS)
+        b = (rb.standard_normal(cfg.n_experts) * math.sqrt(cfg.bias_var)).astype(np.float32)
+    elif cfg.bias == "zipf":
+        ranks = zipf_ranks(cfg, seed)
+        b = (-cfg.zipf_beta * cfg.zipf_s * np.log(ranks.astype(np.float64))).astype(np.float32)
+    else:
+        raise ValueError(cfg.bias)
+    return W, b
+
+
+def make_expert_blob(cfg: LayerConfig, expert: int, seed: int = 0) -> np.ndarray:
+    """One expert blob; expert in [0, E) routed, [E, E+S) shared.
+
+    int4 values are uniform in [-8, 7] (a uniform random byte is two independent
+    uniform nibbles); scales are fp16 (round to nearest even) of U[0.005, 0.02].
+    """
+    H, I = cfg.hidden, cfg.inter
+    lay = blob_layout(H, I)
+    r = _rng(seed, _STREAM_EXPERT, expert)
+    blob = np.zeros(lay["total"], np.uint8)
+    nq = I * H // 2
+    for name in ("gq", "uq", "dq"):
+        blob[lay[name]:lay[name] + nq] = np.frombuffer(r.bytes(nq), np.uint8)
+    for name, rows, cols in (("gs", I, H // QBLOCK), ("us", I, H // QBLOCK), ("ds", H, I // QBLOCK)):
+        s = r.uniform(0.005, 0.02, size=rows * cols).astype(np.float32).astype(np.float16)
+        raw = s.view(np.uint8)
+        blob[lay[name]:lay[name] + raw.size] = raw
+    return blob
+
+
+def make_all_blobs(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
+    """All E + S blobs as one u8 array [E+S][expert_bytes]."""
+    nb = expert_bytes(cfg.hidden, cfg.inter)
+    out = np.empty((cfg.n_experts + cfg.n_shared, nb), np.uint8)
+    for e in range(cfg.n_experts + cfg.n_shared):
+        out[e] = make_expert_blob(cfg, e, seed)
+    return out
+
+
+def make_slot_permutation(cfg: LayerConfig, seed: int = 0, index: int = 0) -> np.ndarray:
+    """Seeded permutation: slot s holds expert perm[s] (all experts bound)."""
+    return _rng(seed, _STREAM_SLOTS, index).permutation(cfg.n_experts).astype(np.int32)

@@ -1,0 +1,107 @@
+"""A deliberately naive fp64 restatement of the layer, used only to pin the oracle.
+
+It shares no code with the oracle: its own int4 unpacking (vectorised numpy),
+dense dequantisation of every expert, every expert evaluated for every token,
+exact router sums (fractions), top-k found by enumerating all expert subsets,
+and fp64 softmax / combine.  It is far too slow for anything but tiny shapes.
+"""
+from __future__ import annotations
+
+import itertools
+from fractions import Fraction
+
+import numpy as np
+
+from quantized_routed_expert_04_b200 import synth
+
+
+def unpack_int4(packed: np.ndarray, rows: int, K: int) -> np.ndarray:
+    b = np.asarray(packed, np.uint8).reshape(rows, K // 2)
+    lo = (b & 0xF).astype(np.int16)
+    hi = (b >> 4).astype(np.int16)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    q = np.empty((rows, K), np.int16)
+    q[:, 0::2] = lo
+    q[:, 1::2] = hi
+    return q
+
+
+def dense_expert(blob: np.ndarray, H: int, I: int):
+    """(Wg [I][H], Wu [I][H], Wd [H][I]) dequantised to float64."""
+    lay = synth.blob_layout(H, I)
+
+    def mat(qn, sn, rows, K):
+        q = unpack_int4(blob[lay[qn]:lay[qn] + rows * K // 2], rows, K)
+        s = blob[lay[sn]:lay[sn] + rows * (K // 32) * 2].view(np.float16)
+        s = s.reshape(rows, K // 32).astype(np.float64)
+        return q.astype(np.float64) * np.repeat(s, 32, axis=1)
+
+    return mat("gq", "gs", I, H), mat("uq", "us", I, H), mat("dq", "ds", H, I)
+
+
+def ffn64(dense, x: np.ndarray) -> np.ndarray:
+    Wg, Wu, Wd = dense
+    g = Wg @ x
+    u = Wu @ x
+    h = g / (1.0 + np.exp(-g)) * u
+    return Wd @ h
+
+
+def exact_logits(x_bf16: np.ndarray, W: np.ndarray, bias) -> np.ndarray:
+    """fp32 logits from the exact real-number sum (fractions), rounded once.
+
+    Rounding Fraction -> float64 -> float32 can double-round; the chance is
+    about 2^-29 per logit, negligible for the tiny sizes used here.
+    """
+    x = synth.bf16_bits_to_f32(x_bf16).astype(np.float64)
+    T, H = x.shape
+    E = W.shape[0]
+    out = np.zeros((T, E), np.float32)
+    for t in range(T):
+        for e in range(E):
+            acc = Fraction(0)
+            for h in range(H):
+                acc += Fraction(float(x[t, h])) * Fraction(float(W[e, h]))
+            if bias is not None:
+                acc += Fraction(float(bias[e]))
+            out[t, e] = np.float32(float(acc))
+    return out
+
+
+def topk_by_subsets(l: np.ndarray, k: int):
+    """Top-k set = the subset with the largest exact logit sum; among equal sums
+    the lexicographically smallest sorted index tuple (lower indices first).
+    Returned in descending logit order, ties by ascending index."""
+    best, best_sum = None, None
+    for sub in itertools.combinations(range(len(l)), k):
+        s = sum(Fraction(float(l[e])) for e in sub)
+        if best is None or s > best_sum:
+            best, best_sum = sub, s
+    return sorted(best, key=lambda e: (-float(l[e]), e))
+
+
+def layer64(x_bf16, blobs, shared, W, bias, k, H, I):
+    """Naive layer: returns (out fp64 [T][H], idx [T][k], w fp64 [T][k])."""
+    E = W.shape[0]
+    logits = exact_logits(x_bf16, W, bias)
+    x = synth.bf16_bits_to_f32(x_bf16).astype(np.float64)
+    dense = [dense_expert(b, H, I) for b in blobs]
+    dense_sh = [dense_expert(b, H, I) for b in shared]
+    T = x.shape[0]
+    out = np.zeros((T, H))
+    idx = np.zeros((T, k), np.int64)
+    wts = np.zeros((T, k))
+    for t in range(T):
+        ys = [ffn64(d, x[t]) for d in dense]          # every expert, every token
+        l64 = logits[t].astype(np.float64)
+        p = np.exp(l64 - l64.max())
+        p /= p.sum()
+        sel = topk_by_subsets(logits[t], k)
+        w = p[sel] / p[sel].sum()
+        idx[t] = sel
+        wts[t] = w
+        out[t] = sum(w[j] * ys[sel[j]] for j in range(k))
+        for d in dense_sh:
+            out[t] += ffn64(d, x[t])
+    return out, idx, wts
