@@ -1,0 +1,170 @@
+/*
+ * strata_moe.h -- C interface of the routed int4 expert (mixture-of-experts)
+ * layer for one NVIDIA B200 (sm_100a).
+ *
+ * The layer, for each of n_tokens tokens x[t] (bf16, length hidden):
+ *   1. routes the token to its top_k experts: logit[e] = x[t] . Wr[e] + b[e]
+ *      (fp32 router weights), softmax over the n_experts logits, the top_k
+ *      largest logits (ties: lower expert id first), and the selected
+ *      probabilities divided by their sum -> weights w[t][j];
+ *   2. finds each selected expert's weights through an expert-id -> slot
+ *      table over a fixed-size arena of expert blobs (ro99/strata README,
+ *      "Residency": routed experts leased into VRAM through an LRU cache;
+ *      "Strata on a Mac", "What you need": an arena of the most-used experts
+ *      with the rest read as tokens need them);
+ *   3. runs the expert FFN on 4-bit block-quantised weights ("INT4 ...
+ *      W4A16 execution", ro99/strata README, model table):
+ *      h = silu(Wg x) * (Wu x), y = Wd h, silu(z) = z / (1 + exp(-z));
+ *   4. writes out[t] = sum_j w[t][j] * y[t][j] + sum_s y_shared[t][s].
+ * The output does not depend on which slot holds which expert, nor on
+ * whether experts that are not routed are bound at all (the bit-exact tier of
+ * "How these numbers are measured", "Fidelity (paged vs resident output)").
+ *
+ * Expert blob format (the contract behind every device_ptr; one contiguous
+ * blob per expert, as "Strata on a Mac", "What you need", keeps each
+ * expert's three matrices together):
+ *     section  shape          type  offset
+ *     Wg_q     [I][H/2]       u8    0
+ *     Wu_q     [I][H/2]       u8    each section starts at the next
+ *     Wd_q     [H][I/2]       u8    multiple of 256 bytes after the
+ *     Wg_s     [I][H/32]      f16   previous one; the blob size is
+ *     Wu_s     [I][H/32]      f16   rounded up to 256 bytes
+ *     Wd_s     [H][I/32]      f16   (strata_moe_expert_bytes)
+ * with H = hidden, I = inter.  Byte j of a row holds element 2j in its low
+ * nibble and element 2j+1 in its high nibble; a nibble is a two's-complement
+ * int4 in [-8, 7]; one fp16 scale covers 32 consecutive elements of a row;
+ * the weight is scale * q.
+ *
+ * Ownership: the caller owns every buffer it passes (activations, outputs,
+ * routing arrays, router weights, expert blobs); they must stay valid until
+ * the stream work that uses them has completed.  The library owns its handle
+ * and a device workspace, and never frees caller memory.
+ *
+ * Ordering: bind and set calls are host-only and synchronous; each forward or
+ * route call takes a snapshot of the slot table when it is enqueued, so a
+ * later bind affects only later calls.  Rebinding a slot whose blob is still
+ * read by enqueued work is the caller's hazard, as for any stream-ordered
+ * buffer.
+ *
+ * Errors: a call that finds a problem on the host returns a status and
+ * enqueues nothing.  Problems only the device can see (a routed expert with
+ * no slot, an out-of-range expert id given to forward_routed, a kernel wait
+ * that timed out) are recorded in a device status word: the affected
+ * tokens' outputs are written as zeros, and strata_moe_get_status reports
+ * the word.  Nothing traps, and nothing falls back to another computation.
+ * n_tokens == 0 returns STRATA_OK and enqueues nothing.
+ */
+#ifndef STRATA_MOE_H
+#define STRATA_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *strata_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef struct strata_moe strata_moe; /* opaque */
+
+typedef enum {
+  STRATA_OK = 0,
+  STRATA_ERR_INVALID_ARG = 1,      /* bad dimension, index, pointer or alignment */
+  STRATA_ERR_UNSUPPORTED = 2,      /* a shape the kernels do not handle */
+  STRATA_ERR_NOT_BOUND = 3,        /* a routed expert had no slot (device-detected) */
+  STRATA_ERR_SLOT_CONFLICT = 4,    /* the expert is already bound to another slot */
+  STRATA_ERR_TOO_MANY_EXPERTS = 5, /* more distinct experts than slots were asked for */
+  STRATA_ERR_OOM = 6,              /* workspace allocation failed */
+  STRATA_ERR_CUDA = 7,             /* a CUDA runtime call failed */
+  STRATA_ERR_DEVICE_STATUS = 8     /* another device-side error (bad routing, timeout) */
+} strata_status;
+
+/* Create a layer on the current CUDA device.
+ * hidden, inter: H and I, multiples of 64.  n_experts: 1..256.
+ * top_k: 1..min(32, n_experts).  n_shared: 0..4 always-on experts of the same
+ * shape.  n_slots: arena slots, top_k..n_experts.  On success *out owns a
+ * handle (free with strata_moe_destroy).  Errors: INVALID_ARG, OOM, CUDA. */
+strata_status strata_moe_create(int hidden, int inter, int n_experts, int top_k, int n_shared,
+                                int n_slots, strata_moe **out);
+
+/* Free the handle and its workspace (synchronises the device first). */
+void strata_moe_destroy(strata_moe *h);
+
+/* Size in bytes of one expert blob (the format above) for hidden x inter. */
+size_t strata_moe_expert_bytes(int hidden, int inter);
+
+/* Router weights: W_dev fp32 [n_experts][hidden] row-major (device), bias_dev
+ * fp32 [n_experts] (device) or NULL for none.  Pointers must be 16-byte
+ * aligned.  Errors: INVALID_ARG. */
+strata_status strata_moe_set_router(strata_moe *h, const float *W_dev, const float *bias_dev);
+
+/* Bind shared expert i (0 <= i < n_shared) to the blob at device_ptr
+ * (256-byte aligned, strata_moe_expert_bytes long).  Errors: INVALID_ARG. */
+strata_status strata_moe_bind_shared(strata_moe *h, int i, const void *device_ptr);
+
+/* Put expert_id's blob at device_ptr into slot `slot` (0 <= slot < n_slots);
+ * expert_id == -1 empties the slot (device_ptr ignored).  device_ptr must be
+ * 256-byte aligned.  Errors: INVALID_ARG (range, alignment, NULL),
+ * SLOT_CONFLICT (expert_id already sits in another slot). */
+strata_status strata_moe_bind_slot(strata_moe *h, int slot, int expert_id, const void *device_ptr);
+
+/* Expert id held by `slot`, or -1 (empty) or -2 (slot out of range). */
+int strata_moe_slot_expert(const strata_moe *h, int slot);
+
+/* Grow the device workspace to hold max_tokens tokens now (synchronous), so
+ * that later forward/route calls with n_tokens <= max_tokens allocate nothing
+ * (for example before capturing them in a CUDA graph).  Errors: OOM, CUDA. */
+strata_status strata_moe_reserve(strata_moe *h, int max_tokens);
+
+/* Routing only.  x_bf16: device bf16 [n_tokens][hidden].  logits_out: device
+ * fp32 [n_tokens][n_experts] or NULL.  idx_out: device int32
+ * [n_tokens][top_k], experts in descending logit order (ties: lower id
+ * first).  w_out: device fp32 [n_tokens][top_k], the renormalised softmax
+ * weights.  Asynchronous on `stream`.  Errors: INVALID_ARG, OOM, CUDA. */
+strata_status strata_moe_route(strata_moe *h, const void *x_bf16, int n_tokens, float *logits_out,
+                               int32_t *idx_out, float *w_out, strata_stream_t stream);
+
+/* The whole layer.  x_bf16: device bf16 [n_tokens][hidden]; out_bf16: device
+ * bf16 [n_tokens][hidden] (round to nearest even of the fp32 combine).
+ * Asynchronous on `stream`.  Host errors: INVALID_ARG (including no router
+ * set or a shared expert not bound), OOM, CUDA.  Device errors (see
+ * strata_moe_get_status): NOT_BOUND. */
+strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens, void *out_bf16,
+                                 strata_stream_t stream);
+
+/* The layer with routing given: idx (device int32 [n_tokens][top_k], each in
+ * [0, n_experts), distinct within a token) and w (device fp32
+ * [n_tokens][top_k]), e.g. from strata_moe_route after the caller has bound
+ * the routed experts.  Device errors: NOT_BOUND, DEVICE_STATUS (bad id). */
+strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n_tokens,
+                                        const int32_t *idx, const float *w, void *out_bf16,
+                                        strata_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the device status word: STRATA_OK,
+ * STRATA_ERR_NOT_BOUND, STRATA_ERR_DEVICE_STATUS, or STRATA_ERR_CUDA if the
+ * stream itself failed. */
+strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream);
+
+/* Raw device status bits of the last get_status call (1 = not bound,
+ * 2 = bad routing id, 4 = wait timeout, 8 = bounds), for diagnostics. */
+int strata_moe_last_device_bits(const strata_moe *h);
+
+/* Per-kernel timing for measurement.  enable != 0 makes every later call
+ * record a CUDA event pair around each kernel on the call's stream;
+ * strata_moe_profile_read synchronises those events and returns, per phase,
+ * the number of launches and their summed milliseconds, then clears them.
+ * Phases: 0 router, 1 top-k, 2 bucketing, 3 activation pack, 4 gate/up+SwiGLU,
+ * 5 down projection, 6 combine, 7 prefill gather.  n_phases <= 8.
+ * Errors: INVALID_ARG, CUDA. */
+strata_status strata_moe_profile(strata_moe *h, int enable);
+strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches, double *ms);
+
+/* Human-readable name of a status. */
+const char *strata_status_str(strata_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STRATA_MOE_H */

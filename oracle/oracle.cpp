@@ -105,7 +105,10 @@ int int4_at(const uint8_t *row, int col) {
 void dequant_row(const uint8_t *q, const uint16_t *s, int K, int row, float *out) {
   const uint8_t *qr = q + (size_t)row * (K / 2);
   const uint16_t *sr = s + (size_t)row * (K / 32);
-  for (int c = 0; c < K; ++c) out[c] = f16_value(sr[c / 32]) * (float)int4_at(qr, c);
+  for (int b = 0; b < K / 32; ++b) {
+    const float scale = f16_value(sr[b]);
+    for (int c = 32 * b; c < 32 * b + 32; ++c) out[c] = scale * (float)int4_at(qr, c);
+  }
 }
 
 float silu(float z) { return z / (1.0f + std::exp(-z)); }

@@ -1,0 +1,63 @@
+// Internal definitions shared by the host side and the kernels of the routed
+// int4 expert layer (not part of the public C interface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace strata {
+
+constexpr int kMaxExperts = 256;   // routed experts per layer
+constexpr int kMaxShared = 4;      // always-on shared experts per layer
+constexpr int kMaxIds = kMaxExperts + kMaxShared;
+constexpr int kMaxTopK = 32;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per barrier wait
+
+// Device status word bits (OR-ed by kernels, read by strata_moe_get_status).
+enum : int {
+  STATUS_NOT_BOUND = 1,      // a routed expert had no arena slot
+  STATUS_BAD_ROUTING = 2,    // forward_routed got an expert id out of range
+  STATUS_TIMEOUT = 4,        // a bounded wait in a kernel gave up
+  STATUS_BOUNDS = 8,         // a computed offset fell outside its buffer
+};
+
+// Byte offsets of the six sections of an expert blob.
+struct BlobLayout {
+  size_t gq, uq, dq, gs, us, ds, total;
+};
+
+inline BlobLayout blob_layout(int H, int I) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  BlobLayout L;
+  size_t off = 0;
+  L.gq = off; off = up(off + (size_t)I * H / 2);
+  L.uq = off; off = up(off + (size_t)I * H / 2);
+  L.dq = off; off = up(off + (size_t)H * I / 2);
+  L.gs = off; off = up(off + (size_t)I * (H / 32) * 2);
+  L.us = off; off = up(off + (size_t)I * (H / 32) * 2);
+  L.ds = off; off = up(off + (size_t)H * (I / 32) * 2);
+  L.total = off;
+  return L;
+}
+
+// Blob address of every expert id, taken by value at launch time: routed
+// experts 0..E-1 (nullptr = not bound to a slot), then shared experts.
+struct ExpertTable {
+  const uint8_t *ptr[kMaxIds];
+};
+
+// Routing workspace (device memory), written by the bucketing kernels.
+// Pairs (t, j) -- token t's j-th routed expert (j < k) or shared expert
+// j - k -- are sorted by expert id, then by token.
+struct Routing {
+  int *cnt;        // [E+S] pairs per expert id
+  int *off;        // [E+S+1] first sorted position of each id
+  int *active;     // [E+S] ids with cnt > 0, ascending
+  int *n_active;   // [1]
+  int *pair_tok;   // [P] token of sorted pair
+  int *pair_j;     // [P] j of sorted pair
+  int *inv;        // [T][k+S] sorted position of pair (t, j)
+};
+
+}  // namespace strata

@@ -1,0 +1,344 @@
+// Routing, bucketing, activation packing and the weighted combine.
+//
+// Router ("the router GEMV and moe_route", "Strata on a Mac", "Switches",
+// two opt-ins paragraph): logit = x . Wr[e] + b[e] with x bf16 and Wr fp32;
+// every product is exact in double and the sum is kept in double, then
+// rounded once to fp32.  Top-k takes the largest fp32 logits, lower expert id
+// first among equal ones; the weights are the softmax probabilities of the
+// selected experts divided by their sum, computed directly as
+// exp(l_j - l_max) / sum_j exp(l_j - l_max).
+//
+// Bucketing sorts the (token, j) pairs by expert id, then token, with no
+// atomics in the ordering (each expert's block walks the pairs in order), so
+// the layout -- and every result downstream -- is a pure function of the
+// routing, independent of slots and of scheduling.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace strata {
+
+// ---------------------------------------------------------------- router GEMV
+// One warp per expert row, all tokens in groups of kTokGroup; each lane sums
+// its strided share of h in double, then a fixed xor-shuffle tree adds the
+// lanes.  Used for small batches (decode).
+constexpr int kTokGroup = 8;
+
+__global__ void router_gemv_kernel(const __nv_bfloat16 *__restrict__ x,
+                                   const float *__restrict__ W, const float *__restrict__ bias,
+                                   int T, int H, int E, float *__restrict__ logits) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (e >= E) return;
+  const float *wr = W + (size_t)e * H;
+  for (int t0 = 0; t0 < T; t0 += kTokGroup) {
+    const int nt = min(kTokGroup, T - t0);
+    double acc[kTokGroup];
+#pragma unroll
+    for (int i = 0; i < kTokGroup; ++i) acc[i] = 0.0;
+    for (int h = lane * 2; h < H; h += 64) {
+      const float2 wv = *reinterpret_cast<const float2 *>(wr + h);
+#pragma unroll
+      for (int i = 0; i < kTokGroup; ++i) {
+        if (i < nt) {
+          const __nv_bfloat162 xv =
+              *reinterpret_cast<const __nv_bfloat162 *>(x + (size_t)(t0 + i) * H + h);
+          const float2 xf = __bfloat1622float2(xv);
+          acc[i] = fma((double)xf.x, (double)wv.x, acc[i]);
+          acc[i] = fma((double)xf.y, (double)wv.y, acc[i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kTokGroup; ++i) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    }
+    if (lane == 0) {
+      const double b = bias ? (double)bias[e] : 0.0;
+      for (int i = 0; i < nt; ++i) logits[(size_t)(t0 + i) * E + e] = (float)(acc[i] + b);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- router GEMM
+// 64 tokens x 64 experts per block; each thread owns 4 x 4 logits and adds
+// products in ascending h, in double.  Used for large batches (prefill).
+constexpr int kRT = 64, kRE = 64, kRK = 32;
+
+__global__ void __launch_bounds__(256) router_gemm_kernel(
+    const __nv_bfloat16 *__restrict__ x, const float *__restrict__ W,
+    const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits) {
+  grid_dependency_wait();
+  __shared__ float xs[kRK][kRT + 1];
+  __shared__ float ws[kRK][kRE + 1];
+  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  for (int k0 = 0; k0 < H; k0 += kRK) {
+    for (int v = tid; v < kRT * kRK; v += 256) {
+      const int r = v / kRK, c = v % kRK;
+      const int t = t0 + r;
+      xs[c][r] = t < T ? __bfloat162float(x[(size_t)t * H + k0 + c]) : 0.0f;
+      const int e = e0 + r;
+      ws[c][r] = e < E ? W[(size_t)e * H + k0 + c] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < kRK; ++kk) {
+      double a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = ws[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e >= E) continue;
+      double v = acc[i][j];
+      if (bias) v += (double)bias[e];
+      logits[(size_t)t * E + e] = (float)v;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- top-k
+// One warp per token.  Lane l holds logits l, l+32, ...; k rounds of a warp
+// arg-max (larger logit wins, equal logits: lower id wins).
+__global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+                            int32_t *__restrict__ idx, float *__restrict__ w) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  constexpr int kPer = kMaxExperts / 32;
+  float v[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? logits[(size_t)t * E + e] : -INFINITY;
+  }
+  unsigned taken = 0;
+  float sel_l[kMaxTopK];
+  int sel_e[kMaxTopK];
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    sel_l[j] = bv;
+    sel_e[j] = be;
+  }
+  if (lane == 0) {
+    float z = 0.0f;
+    float p[kMaxTopK];
+    for (int j = 0; j < k; ++j) {
+      p[j] = expf(sel_l[j] - sel_l[0]);
+      z += p[j];
+    }
+    for (int j = 0; j < k; ++j) {
+      idx[(size_t)t * k + j] = sel_e[j];
+      w[(size_t)t * k + j] = p[j] / z;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- activation pack
+// x bf16 -> f16 with each group of 8 stored in the order 0,4,1,5,2,6,3,7 (the
+// order in which the int4 unpacking produces weight pairs, so one 16-byte
+// load gives a thread its four mma B-fragment registers).
+__global__ void pack_x_kernel(const __nv_bfloat16 *__restrict__ x, int n8,
+                              __half *__restrict__ x16) {
+  grid_dependency_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)i * 8);
+  const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+  const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
+  const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
+  // elements: 0=f0.x 1=f0.y 2=f1.x 3=f1.y 4=f2.x 5=f2.y 6=f3.x 7=f3.y
+  uint4 o;
+  __half2 h;
+  h = __floats2half2_rn(f0.x, f2.x); o.x = h2_bits(h);
+  h = __floats2half2_rn(f0.y, f2.y); o.y = h2_bits(h);
+  h = __floats2half2_rn(f1.x, f3.x); o.z = h2_bits(h);
+  h = __floats2half2_rn(f1.y, f3.y); o.w = h2_bits(h);
+  *reinterpret_cast<uint4 *>(x16 + (size_t)i * 8) = o;
+}
+
+// ---------------------------------------------------------------- bucketing
+// Pair counts per expert id.  Ids outside [0, E) are flagged and skipped.
+__global__ void bucket_count_kernel(const int32_t *__restrict__ idx, int T, int k, int E,
+                                    int *__restrict__ cnt, int *status) {
+  grid_dependency_wait();
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= T * k) return;
+  const int e = idx[p];
+  if (e < 0 || e >= E) {
+    set_status(status, STATUS_BAD_ROUTING);
+    return;
+  }
+  atomicAdd(&cnt[e], 1);
+}
+
+// One block per expert id (E routed + S shared).  Computes the id's offset
+// and active-list position from the counts, then writes its pairs in token
+// order.  cnt of shared ids is T (set here).
+__global__ void __launch_bounds__(256) bucket_fill_kernel(const int32_t *__restrict__ idx, int T,
+                                                          int k, int E, int S, Routing rt) {
+  grid_dependency_wait();
+  const int id = blockIdx.x;
+  const int nid = E + S;
+  const int tid = threadIdx.x;
+  __shared__ int s_sum[8], s_act[8];
+  __shared__ int s_base;
+  // offset = sum of counts of lower ids; active rank = number of lower ids in use
+  int part = 0, act = 0;
+  for (int i = tid; i < id; i += blockDim.x) {
+    const int c = i < E ? rt.cnt[i] : T;
+    part += c;
+    act += c > 0;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    part += __shfl_xor_sync(0xffffffffu, part, o);
+    act += __shfl_xor_sync(0xffffffffu, act, o);
+  }
+  if ((tid & 31) == 0) {
+    s_sum[tid >> 5] = part;
+    s_act[tid >> 5] = act;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int off = 0, a = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+      off += s_sum[i];
+      a += s_act[i];
+    }
+    const int mine = id < E ? rt.cnt[id] : T;
+    if (id >= E) rt.cnt[id] = T;
+    rt.off[id] = off;
+    if (mine > 0) rt.active[a] = id;
+    if (id == nid - 1) {
+      rt.off[nid] = off + mine;
+      *rt.n_active = a + (mine > 0);
+    }
+    s_base = off;
+  }
+  __syncthreads();
+  const int base = s_base;
+  const int kS = k + S;
+  if (id >= E) {
+    const int j = k + (id - E);
+    for (int t = tid; t < T; t += blockDim.x) {
+      rt.pair_tok[base + t] = t;
+      rt.pair_j[base + t] = j;
+      rt.inv[(size_t)t * kS + j] = base + t;
+    }
+    return;
+  }
+  // routed: ordered compaction of the pairs p = t*k + j with idx[p] == id
+  __shared__ int s_wcnt[8];
+  int running = 0;
+  const int n = T * k;
+  for (int p0 = 0; p0 < n; p0 += blockDim.x) {
+    const int p = p0 + tid;
+    const bool m = p < n && idx[p] == id;
+    const unsigned bal = __ballot_sync(0xffffffffu, m);
+    if ((tid & 31) == 0) s_wcnt[tid >> 5] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int wi = 0; wi < (int)(blockDim.x >> 5); ++wi) {
+      if (wi < (tid >> 5)) before += s_wcnt[wi];
+      total += s_wcnt[wi];
+    }
+    if (m) {
+      const int pos = base + running + before + __popc(bal & ((1u << (tid & 31)) - 1u));
+      const int t = p / k, j = p % k;
+      rt.pair_tok[pos] = t;
+      rt.pair_j[pos] = j;
+      rt.inv[(size_t)t * kS + j] = pos;
+    }
+    running += total;
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// out[t][r] = bf16( sum_j w[t][j] * y[inv[t][j]][r] + sum_s y[inv[t][k+s]][r] )
+// in fp32, in that order.  A token with an unbound or invalid expert gets a
+// zero row.  Each thread handles 4 consecutive r.
+__global__ void combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ idx,
+                               const float *__restrict__ w, const int *__restrict__ inv,
+                               ExpertTable table, int T, int H, int k, int S, int E,
+                               __nv_bfloat16 *__restrict__ out) {
+  grid_dependency_wait();
+  const int t = blockIdx.y;
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (t >= T || r >= H) return;
+  const int kS = k + S;
+  bool ok = true;
+  for (int j = 0; j < k; ++j) {
+    const int e = idx[(size_t)t * k + j];
+    if (e < 0 || e >= E || !table.ptr[e] || inv[(size_t)t * kS + j] < 0) ok = false;
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (ok) {
+    for (int j = 0; j < kS; ++j) {
+      const float wj = j < k ? w[(size_t)t * k + j] : 1.0f;
+      const float4 v = *reinterpret_cast<const float4 *>(y + (size_t)inv[(size_t)t * kS + j] * H + r);
+      if (j < k) {
+        acc.x = __fadd_rn(acc.x, __fmul_rn(wj, v.x));
+        acc.y = __fadd_rn(acc.y, __fmul_rn(wj, v.y));
+        acc.z = __fadd_rn(acc.z, __fmul_rn(wj, v.z));
+        acc.w = __fadd_rn(acc.w, __fmul_rn(wj, v.w));
+      } else {
+        acc.x = __fadd_rn(acc.x, v.x);
+        acc.y = __fadd_rn(acc.y, v.y);
+        acc.z = __fadd_rn(acc.z, v.z);
+        acc.w = __fadd_rn(acc.w, v.w);
+      }
+    }
+  }
+  __nv_bfloat162 o0 = __floats2bfloat162_rn(acc.x, acc.y);
+  __nv_bfloat162 o1 = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t *>(&o0);
+  packed.y = *reinterpret_cast<uint32_t *>(&o1);
+  *reinterpret_cast<uint2 *>(out + (size_t)t * H + r) = packed;
+}
+
+}  // namespace strata

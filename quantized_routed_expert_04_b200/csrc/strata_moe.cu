@@ -1,0 +1,496 @@
+// Host side of the C interface in include/strata_moe.h: the handle, argument
+// checks, the expert-id -> slot table, the device workspace, the kernel
+// sequence of a forward call, the device status word and optional per-kernel
+// timing.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "kernels.h"
+#include "strata_moe.h"
+
+using namespace strata;
+
+namespace {
+
+constexpr int kPhases = 8;
+enum Phase { PH_ROUTER = 0, PH_TOPK, PH_BUCKET, PH_PACK, PH_GATEUP, PH_DOWN, PH_COMBINE, PH_GATHER };
+
+struct EventPair {
+  int phase;
+  cudaEvent_t a, b;
+};
+
+}  // namespace
+
+struct strata_moe {
+  int H, I, E, k, S, n_slots;
+  int device = 0, num_sms = 0;
+  BlobLayout layout{};
+
+  std::vector<int> slot_expert;            // per slot: expert id or -1
+  std::vector<const void *> slot_ptr;      // per slot: blob
+  std::vector<int> expert_slot;            // per expert: slot or -1
+  std::vector<const void *> shared_ptr;    // per shared expert
+  const float *router_W = nullptr;
+  const float *router_b = nullptr;
+
+  // workspace
+  int cap_tokens = 0;
+  void *ws = nullptr;
+  size_t ws_bytes = 0;
+  float *logits = nullptr;
+  int32_t *idx = nullptr;
+  float *w = nullptr;
+  int *meta = nullptr;      // cnt | off | active | n_active
+  Routing rt{};
+  __half *x16 = nullptr;
+  __half *h16 = nullptr;
+  float *y = nullptr;
+  int *status = nullptr;    // device status word (own allocation)
+  int last_bits = 0;
+
+  // per-kernel timing
+  bool profiling = false;
+  std::vector<EventPair> events;
+  std::vector<cudaEvent_t> event_pool;
+  int prof_launches[kPhases] = {};
+  double prof_ms[kPhases] = {};
+};
+
+namespace {
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+strata_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return STRATA_OK;
+  if (e == cudaErrorMemoryAllocation) return STRATA_ERR_OOM;
+  return STRATA_ERR_CUDA;
+}
+
+cudaEvent_t take_event(strata_moe *h) {
+  if (!h->event_pool.empty()) {
+    cudaEvent_t e = h->event_pool.back();
+    h->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launch `kern` on `stream`; pdl lets it start while the previous kernel in
+// the stream drains (every kernel here begins with griddepcontrol.wait
+// before it reads anything the previous kernels wrote).
+template <typename... Exp, typename... Act>
+cudaError_t launch(strata_moe *h, int phase, void (*kern)(Exp...), dim3 grid, dim3 block,
+                   size_t smem, cudaStream_t stream, bool pdl, Act &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (pdl && !h->profiling) ? 1 : 0;
+  EventPair ev{phase, nullptr, nullptr};
+  if (h->profiling) {
+    ev.a = take_event(h);
+    ev.b = take_event(h);
+    cudaEventRecord(ev.a, stream);
+  }
+  cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+  if (h->profiling) {
+    cudaEventRecord(ev.b, stream);
+    h->events.push_back(ev);
+  }
+  return err;
+}
+
+strata_status grow_workspace(strata_moe *h, int T) {
+  if (T <= h->cap_tokens) return STRATA_OK;
+  const int cap = std::max(T, 2 * h->cap_tokens);
+  const int kS = h->k + h->S;
+  const size_t P = (size_t)cap * kS;
+  const int nid = h->E + h->S;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_logits = take(sizeof(float) * cap * h->E);
+  const size_t o_idx = take(sizeof(int32_t) * cap * h->k);
+  const size_t o_w = take(sizeof(float) * cap * h->k);
+  const size_t o_meta = take(sizeof(int) * (3 * nid + 2));
+  const size_t o_ptok = take(sizeof(int) * P);
+  const size_t o_pj = take(sizeof(int) * P);
+  const size_t o_inv = take(sizeof(int) * P);
+  const size_t o_x16 = take(sizeof(__half) * cap * h->H);
+  const size_t o_h16 = take(sizeof(__half) * P * h->I);
+  const size_t o_y = take(sizeof(float) * P * h->H);
+  void *mem = nullptr;
+  cudaError_t e = cudaMalloc(&mem, off);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  if (h->ws) cudaFree(h->ws);
+  h->ws = mem;
+  h->ws_bytes = off;
+  h->cap_tokens = cap;
+  char *b = static_cast<char *>(mem);
+  h->logits = reinterpret_cast<float *>(b + o_logits);
+  h->idx = reinterpret_cast<int32_t *>(b + o_idx);
+  h->w = reinterpret_cast<float *>(b + o_w);
+  h->meta = reinterpret_cast<int *>(b + o_meta);
+  h->rt.cnt = h->meta;
+  h->rt.off = h->meta + nid;
+  h->rt.active = h->meta + 2 * nid + 1;
+  h->rt.n_active = h->meta + 3 * nid + 1;
+  h->rt.pair_tok = reinterpret_cast<int *>(b + o_ptok);
+  h->rt.pair_j = reinterpret_cast<int *>(b + o_pj);
+  h->rt.inv = reinterpret_cast<int *>(b + o_inv);
+  h->x16 = reinterpret_cast<__half *>(b + o_x16);
+  h->h16 = reinterpret_cast<__half *>(b + o_h16);
+  h->y = reinterpret_cast<float *>(b + o_y);
+  return STRATA_OK;
+}
+
+ExpertTable make_table(const strata_moe *h) {
+  ExpertTable t;
+  std::memset(&t, 0, sizeof t);
+  for (int s = 0; s < h->n_slots; ++s)
+    if (h->slot_expert[s] >= 0) t.ptr[h->slot_expert[s]] = static_cast<const uint8_t *>(h->slot_ptr[s]);
+  for (int i = 0; i < h->S; ++i) t.ptr[h->E + i] = static_cast<const uint8_t *>(h->shared_ptr[i]);
+  return t;
+}
+
+// Largest multiple of 64 that divides K and is at most 1024.
+int pick_kc(int K) {
+  int best = 64;
+  for (int kc = 64; kc <= 1024 && kc <= K; kc += 64)
+    if (K % kc == 0) best = kc;
+  return best;
+}
+
+MmParams mm_params(const strata_moe *h, bool gate_up, const ExpertTable &table) {
+  MmParams p;
+  std::memset(&p, 0, sizeof p);
+  p.table = table;
+  p.rt = h->rt;
+  p.E = h->E;
+  p.K = gate_up ? h->H : h->I;
+  p.kc = pick_kc(p.K);
+  if (gate_up) {
+    p.tiles = h->I / 16;
+    p.q_off[0] = h->layout.gq;
+    p.q_off[1] = h->layout.uq;
+    p.s_off[0] = h->layout.gs;
+    p.s_off[1] = h->layout.us;
+    p.row_base_mul = 16;
+    p.row_half[0] = 0;
+    p.row_half[1] = 0;
+    p.b_src = h->x16;
+    p.out_ld = h->I;
+  } else {
+    p.tiles = h->H / 32;
+    p.q_off[0] = p.q_off[1] = h->layout.dq;
+    p.s_off[0] = p.s_off[1] = h->layout.ds;
+    p.row_base_mul = 32;
+    p.row_half[0] = 0;
+    p.row_half[1] = 16;
+    p.b_src = h->h16;
+    p.out_ld = h->H;
+  }
+  p.h_out = h->h16;
+  p.y_out = h->y;
+  p.status = h->status;
+  p.wstride = p.kc / 2 + 16;
+  const int sbytes = p.kc / 16;
+  p.sstride = ((sbytes / 4) % 2 == 0) ? sbytes + 4 : sbytes;
+  p.bstride = 2 * p.kc + 64;
+  p.w_bytes = 32 * p.wstride;
+  p.s_bytes = (int)align_up(32 * p.sstride, 16);
+  p.stage_bytes = (int)align_up(p.w_bytes + p.s_bytes + kMmGroup * p.bstride, 128);
+  return p;
+}
+
+strata_status check_common(strata_moe *h, const void *x, int T, cudaStream_t) {
+  if (!h || T < 0) return STRATA_ERR_INVALID_ARG;
+  if (T > 0 && (!x || (reinterpret_cast<uintptr_t>(x) & 15))) return STRATA_ERR_INVALID_ARG;
+  return STRATA_OK;
+}
+
+// Bucketing + the expert passes + combine, given idx/w in device memory.
+strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *idx, const float *w,
+                          void *out, cudaStream_t stream) {
+  const ExpertTable table = make_table(h);
+  const int kS = h->k + h->S;
+  const int nid = h->E + h->S;
+  cudaError_t e;
+  e = cudaMemsetAsync(h->rt.cnt, 0, sizeof(int) * nid, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->rt.inv, 0xFF, sizeof(int) * (size_t)T * kS, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  const int n8 = T * h->H / 8;
+  e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb, n8,
+             h->x16);
+  if (e == cudaSuccess)
+    e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
+               stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
+  if (e == cudaSuccess)
+    e = launch(h, PH_BUCKET, bucket_fill_kernel, dim3(nid), dim3(256), 0, stream, true, idx, T,
+               h->k, h->E, h->S, h->rt);
+  if (e != cudaSuccess) return cuda_status(e);
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool gu = pass == 0;
+    MmParams p = mm_params(h, gu, table);
+    const size_t smem = mm_smem_bytes(p);
+    auto kern = gu ? expert_mma_kernel<true> : expert_mma_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(kMmThreads), smem,
+                 stream, true, p);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  dim3 cgrid((h->H / 4 + 127) / 128, T);
+  e = launch(h, PH_COMBINE, combine_kernel, cgrid, dim3(128), 0, stream, true, h->y, idx, w,
+             h->rt.inv, table, T, h->H, h->k, h->S, h->E, static_cast<__nv_bfloat16 *>(out));
+  return cuda_status(e);
+}
+
+strata_status run_router(strata_moe *h, const void *x, int T, float *logits, int32_t *idx,
+                         float *w, cudaStream_t stream) {
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  cudaError_t e;
+  if (T <= 64) {
+    const int warps = 8;
+    e = launch(h, PH_ROUTER, router_gemv_kernel, dim3((h->E + warps - 1) / warps),
+               dim3(32 * warps), 0, stream, false, xb, h->router_W, h->router_b, T, h->H, h->E,
+               logits);
+  } else {
+    e = launch(h, PH_ROUTER, router_gemm_kernel, dim3((T + 63) / 64, (h->E + 63) / 64), dim3(256),
+               0, stream, false, xb, h->router_W, h->router_b, T, h->H, h->E, logits);
+  }
+  if (e == cudaSuccess)
+    e = launch(h, PH_TOPK, topk_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, true, logits, T,
+               h->E, h->k, idx, w);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *strata_status_str(strata_status s) {
+  switch (s) {
+    case STRATA_OK: return "ok";
+    case STRATA_ERR_INVALID_ARG: return "invalid argument";
+    case STRATA_ERR_UNSUPPORTED: return "unsupported shape";
+    case STRATA_ERR_NOT_BOUND: return "routed expert not bound to a slot";
+    case STRATA_ERR_SLOT_CONFLICT: return "expert already bound to another slot";
+    case STRATA_ERR_TOO_MANY_EXPERTS: return "more distinct experts than slots";
+    case STRATA_ERR_OOM: return "out of device memory";
+    case STRATA_ERR_CUDA: return "CUDA error";
+    case STRATA_ERR_DEVICE_STATUS: return "device-side error";
+  }
+  return "unknown status";
+}
+
+size_t strata_moe_expert_bytes(int hidden, int inter) {
+  if (hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return 0;
+  return blob_layout(hidden, inter).total;
+}
+
+strata_status strata_moe_create(int hidden, int inter, int n_experts, int top_k, int n_shared,
+                                int n_slots, strata_moe **out) {
+  if (!out) return STRATA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (hidden <= 0 || inter <= 0 || hidden % 64 || inter % 64) return STRATA_ERR_INVALID_ARG;
+  if (n_experts < 1 || n_experts > kMaxExperts) return STRATA_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > n_experts || top_k > kMaxTopK) return STRATA_ERR_INVALID_ARG;
+  if (n_shared < 0 || n_shared > kMaxShared) return STRATA_ERR_INVALID_ARG;
+  if (n_slots < top_k || n_slots > n_experts) return STRATA_ERR_INVALID_ARG;
+  strata_moe *h = new (std::nothrow) strata_moe();
+  if (!h) return STRATA_ERR_OOM;
+  h->H = hidden;
+  h->I = inter;
+  h->E = n_experts;
+  h->k = top_k;
+  h->S = n_shared;
+  h->n_slots = n_slots;
+  h->layout = blob_layout(hidden, inter);
+  h->slot_expert.assign(n_slots, -1);
+  h->slot_ptr.assign(n_slots, nullptr);
+  h->expert_slot.assign(n_experts, -1);
+  h->shared_ptr.assign(n_shared, nullptr);
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  if (e == cudaSuccess) e = cudaMalloc(&h->status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    if (h->status) cudaFree(h->status);
+    delete h;
+    return cuda_status(e);
+  }
+  *out = h;
+  return STRATA_OK;
+}
+
+void strata_moe_destroy(strata_moe *h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  for (auto &ev : h->events) {
+    cudaEventDestroy(ev.a);
+    cudaEventDestroy(ev.b);
+  }
+  for (auto e : h->event_pool) cudaEventDestroy(e);
+  if (h->ws) cudaFree(h->ws);
+  if (h->status) cudaFree(h->status);
+  delete h;
+}
+
+strata_status strata_moe_set_router(strata_moe *h, const float *W_dev, const float *bias_dev) {
+  if (!h || !W_dev) return STRATA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(W_dev) & 15) || (reinterpret_cast<uintptr_t>(bias_dev) & 3))
+    return STRATA_ERR_INVALID_ARG;
+  h->router_W = W_dev;
+  h->router_b = bias_dev;
+  return STRATA_OK;
+}
+
+strata_status strata_moe_bind_shared(strata_moe *h, int i, const void *device_ptr) {
+  if (!h || i < 0 || i >= h->S || !device_ptr) return STRATA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(device_ptr) & 255) return STRATA_ERR_INVALID_ARG;
+  h->shared_ptr[i] = device_ptr;
+  return STRATA_OK;
+}
+
+strata_status strata_moe_bind_slot(strata_moe *h, int slot, int expert_id, const void *device_ptr) {
+  if (!h || slot < 0 || slot >= h->n_slots) return STRATA_ERR_INVALID_ARG;
+  if (expert_id < -1 || expert_id >= h->E) return STRATA_ERR_INVALID_ARG;
+  if (expert_id == -1) {
+    const int old = h->slot_expert[slot];
+    if (old >= 0) h->expert_slot[old] = -1;
+    h->slot_expert[slot] = -1;
+    h->slot_ptr[slot] = nullptr;
+    return STRATA_OK;
+  }
+  if (!device_ptr || (reinterpret_cast<uintptr_t>(device_ptr) & 255)) return STRATA_ERR_INVALID_ARG;
+  const int cur = h->expert_slot[expert_id];
+  if (cur >= 0 && cur != slot) return STRATA_ERR_SLOT_CONFLICT;
+  const int old = h->slot_expert[slot];
+  if (old >= 0) h->expert_slot[old] = -1;
+  h->slot_expert[slot] = expert_id;
+  h->slot_ptr[slot] = device_ptr;
+  h->expert_slot[expert_id] = slot;
+  return STRATA_OK;
+}
+
+int strata_moe_slot_expert(const strata_moe *h, int slot) {
+  if (!h || slot < 0 || slot >= h->n_slots) return -2;
+  return h->slot_expert[slot];
+}
+
+strata_status strata_moe_reserve(strata_moe *h, int max_tokens) {
+  if (!h || max_tokens < 0) return STRATA_ERR_INVALID_ARG;
+  return grow_workspace(h, max_tokens);
+}
+
+strata_status strata_moe_route(strata_moe *h, const void *x_bf16, int n_tokens, float *logits_out,
+                               int32_t *idx_out, float *w_out, strata_stream_t stream) {
+  strata_status st = check_common(h, x_bf16, n_tokens, stream);
+  if (st != STRATA_OK) return st;
+  if (!h->router_W) return STRATA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return STRATA_OK;
+  if (!idx_out || !w_out) return STRATA_ERR_INVALID_ARG;
+  st = grow_workspace(h, n_tokens);
+  if (st != STRATA_OK) return st;
+  return run_router(h, x_bf16, n_tokens, logits_out ? logits_out : h->logits, idx_out, w_out,
+                    stream);
+}
+
+strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens, void *out_bf16,
+                                 strata_stream_t stream) {
+  strata_status st = check_common(h, x_bf16, n_tokens, stream);
+  if (st != STRATA_OK) return st;
+  if (!h->router_W) return STRATA_ERR_INVALID_ARG;
+  for (int i = 0; i < h->S; ++i)
+    if (!h->shared_ptr[i]) return STRATA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return STRATA_OK;
+  if (!out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 15)) return STRATA_ERR_INVALID_ARG;
+  st = grow_workspace(h, n_tokens);
+  if (st != STRATA_OK) return st;
+  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream);
+  if (st != STRATA_OK) return st;
+  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream);
+}
+
+strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n_tokens,
+                                        const int32_t *idx, const float *w, void *out_bf16,
+                                        strata_stream_t stream) {
+  strata_status st = check_common(h, x_bf16, n_tokens, stream);
+  if (st != STRATA_OK) return st;
+  for (int i = 0; i < h->S; ++i)
+    if (!h->shared_ptr[i]) return STRATA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return STRATA_OK;
+  if (!idx || !w || !out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 15))
+    return STRATA_ERR_INVALID_ARG;
+  st = grow_workspace(h, n_tokens);
+  if (st != STRATA_OK) return st;
+  return run_experts(h, x_bf16, n_tokens, idx, w, out_bf16, stream);
+}
+
+strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream) {
+  if (!h) return STRATA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return STRATA_ERR_CUDA;
+  int bits = 0;
+  if (cudaMemcpy(&bits, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return STRATA_ERR_CUDA;
+  if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return STRATA_ERR_CUDA;
+  h->last_bits = bits;
+  if (bits & (STATUS_BAD_ROUTING | STATUS_TIMEOUT | STATUS_BOUNDS)) return STRATA_ERR_DEVICE_STATUS;
+  if (bits & STATUS_NOT_BOUND) return STRATA_ERR_NOT_BOUND;
+  return STRATA_OK;
+}
+
+int strata_moe_last_device_bits(const strata_moe *h) { return h ? h->last_bits : 0; }
+
+strata_status strata_moe_profile(strata_moe *h, int enable) {
+  if (!h) return STRATA_ERR_INVALID_ARG;
+  h->profiling = enable != 0;
+  return STRATA_OK;
+}
+
+strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches, double *ms) {
+  if (!h || n_phases < 0 || n_phases > kPhases) return STRATA_ERR_INVALID_ARG;
+  for (auto &ev : h->events) {
+    float t = 0.f;
+    if (cudaEventSynchronize(ev.b) != cudaSuccess) return STRATA_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, ev.a, ev.b) != cudaSuccess) return STRATA_ERR_CUDA;
+    h->prof_launches[ev.phase] += 1;
+    h->prof_ms[ev.phase] += t;
+    h->event_pool.push_back(ev.a);
+    h->event_pool.push_back(ev.b);
+  }
+  h->events.clear();
+  for (int i = 0; i < n_phases; ++i) {
+    if (launches) launches[i] = h->prof_launches[i];
+    if (ms) ms[i] = h->prof_ms[i];
+  }
+  for (int i = 0; i < kPhases; ++i) {
+    h->prof_launches[i] = 0;
+    h->prof_ms[i] = 0.0;
+  }
+  return STRATA_OK;
+}
+
+}  // extern "C"
