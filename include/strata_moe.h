@@ -22,18 +22,25 @@
  *
  * Expert blob format (the contract behind every device_ptr; one contiguous
  * blob per expert, as "Strata on a Mac", "What you need", keeps each
- * expert's three matrices together):
- *     section  shape          type  offset
- *     Wg_q     [I][H/2]       u8    0
- *     Wu_q     [I][H/2]       u8    each section starts at the next
- *     Wd_q     [H][I/2]       u8    multiple of 256 bytes after the
- *     Wg_s     [I][H/32]      f16   previous one; the blob size is
- *     Wu_s     [I][H/32]      f16   rounded up to 256 bytes
- *     Wd_s     [H][I/32]      f16   (strata_moe_expert_bytes)
- * with H = hidden, I = inter.  Byte j of a row holds element 2j in its low
- * nibble and element 2j+1 in its high nibble; a nibble is a two's-complement
- * int4 in [-8, 7]; one fp16 scale covers 32 consecutive elements of a row;
- * the weight is scale * q.
+ * expert's matrices together so that one request reads an expert).  With
+ * H = hidden and I = inter (both multiples of 128):
+ *     section  content                                 bytes
+ *     GU_q     gate and up int4 weights, I/8 tiles     I*H
+ *     D_q      down int4 weights, H/16 tiles           H*I/2
+ *     GU_s     gate and up fp16 scales, I/8 tiles      I*H/8
+ *     D_s      down fp16 scales, H/16 tiles            H*I/16
+ * each starting at the next multiple of 256 bytes; the blob size is rounded
+ * up to 256 bytes (strata_moe_expert_bytes).  A tile has 16 rows: gate/up
+ * tile t holds rows 8t..8t+7 of Wg as tile rows 0..7 and the same rows of Wu
+ * as tile rows 8..15; down tile t holds rows 16t..16t+15 of Wd.  A tile is
+ * stored K-group by K-group (128 consecutive K elements): 16 rows x 64 bytes
+ * of weights, or 16 rows x 4 fp16 scales (one per block of 32 elements; block
+ * b = elements 32b..32b+31 of the group).  In the 64 bytes of one row and
+ * group, byte 16w + 4b + m/2 (w, b in 0..3, m in 0..7) holds element
+ * 32b + 8w + m, in the low nibble for even m; a nibble is a two's-complement
+ * int4 in [-8, 7].  The weight is scale * q.  (Any K range of a tile is one
+ * contiguous run of bytes, and the 16 bytes at 16w hold word w of all four
+ * blocks of a group.)
  *
  * Ownership: the caller owns every buffer it passes (activations, outputs,
  * routing arrays, router weights, expert blobs); they must stay valid until
@@ -81,7 +88,7 @@ typedef enum {
 } strata_status;
 
 /* Create a layer on the current CUDA device.
- * hidden, inter: H and I, multiples of 64.  n_experts: 1..256.
+ * hidden, inter: H and I, multiples of 128.  n_experts: 1..256.
  * top_k: 1..min(32, n_experts).  n_shared: 0..4 always-on experts of the same
  * shape.  n_slots: arena slots, top_k..n_experts.  On success *out owns a
  * handle (free with strata_moe_destroy).  Errors: INVALID_ARG, OOM, CUDA. */

@@ -20,7 +20,8 @@
 //  * Expert lookup through a slot table ("routed experts ... leased into VRAM
 //    per decode step through an LRU cache", ro99/strata README, "Residency").
 //  * Expert FFN on W4A16 weights ("INT4 ... W4A16 execution", ro99/strata
-//    README, model table): w = float(fp16 scale) * q, exact in fp32; gate and
+//    README, model table), read from the tiled blob format described at
+//    place_of(): w = float(fp16 scale) * q, exact in fp32; gate and
 //    up dot products in fp32 in ascending K; h = silu(g) * u with
 //    silu(z) = z / (1 + exp(-z)) in fp32; down projection in fp32 ascending K.
 //  * Combine: out[t] = sum_j w[t][j] * y[t][j] (j = 0..k-1, descending logit)
@@ -49,20 +50,19 @@ enum {
 
 size_t round_up_256(size_t v) { return (v + 255) / 256 * 256; }
 
-// Section offsets of one expert blob, in bytes from its start.
+// Section offsets of one expert blob, in bytes from its start:
+// gate+up weights, down weights, gate+up scales, down scales.
 struct Layout {
-  size_t gq, uq, dq, gs, us, ds, total;
+  size_t guq, dq, gus, ds, total;
 };
 
 Layout layout_of(int H, int I) {
   Layout L;
   size_t off = 0;
-  L.gq = off; off = round_up_256(off + (size_t)I * H / 2);
-  L.uq = off; off = round_up_256(off + (size_t)I * H / 2);
-  L.dq = off; off = round_up_256(off + (size_t)H * I / 2);
-  L.gs = off; off = round_up_256(off + (size_t)I * (H / 32) * 2);
-  L.us = off; off = round_up_256(off + (size_t)I * (H / 32) * 2);
-  L.ds = off; off = round_up_256(off + (size_t)H * (I / 32) * 2);
+  L.guq = off; off = round_up_256(off + (size_t)I * H);
+  L.dq = off;  off = round_up_256(off + (size_t)H * I / 2);
+  L.gus = off; off = round_up_256(off + (size_t)I * H / 8);
+  L.ds = off;  off = round_up_256(off + (size_t)H * I / 16);
   L.total = off;
   return L;
 }
@@ -93,21 +93,60 @@ float f16_value(uint16_t bits) {
   return (float)(sign ? -v : v);
 }
 
-// Element `col` of a packed int4 row: byte col/2, low nibble for even col,
-// high nibble for odd col, two's complement.
-int int4_at(const uint8_t *row, int col) {
-  uint8_t byte = row[col / 2];
-  int n = (col % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+// The three matrices of an expert and where their rows live.  A section is
+// split into tiles of 16 rows; gate row i is row i % 8 of tile i / 8 and up
+// row i is row 8 + i % 8 of the same tile; down row r is row r % 16 of tile
+// r / 16.  A tile is stored group by group (128 K elements), each group as
+// 16 rows of 64 bytes; element k of a row sits in group k / 128, block
+// b = (k % 128) / 32, word w = (k % 32) / 8, nibble m = k % 8, at byte
+// 16 w + 4 b + m / 2 of the row's 64 bytes (low nibble for even m).  Scales:
+// per tile, group, row: four fp16 values, one per block.
+enum Matrix { GATE, UP, DOWN };
+
+struct RowPlace {
+  const uint8_t *q;      // section start
+  const uint16_t *s;     // scale section start
+  int K, tile, trow;
+};
+
+RowPlace place_of(const uint8_t *blob, int H, int I, Matrix mat, int row) {
+  Layout L = layout_of(H, I);
+  RowPlace p;
+  if (mat == DOWN) {
+    p.q = blob + L.dq;
+    p.s = (const uint16_t *)(blob + L.ds);
+    p.K = I;
+    p.tile = row / 16;
+    p.trow = row % 16;
+  } else {
+    p.q = blob + L.guq;
+    p.s = (const uint16_t *)(blob + L.gus);
+    p.K = H;
+    p.tile = row / 8;
+    p.trow = (mat == GATE ? 0 : 8) + row % 8;
+  }
+  return p;
+}
+
+int int4_at(const RowPlace &p, int k) {
+  const int j = k / 128, b = (k % 128) / 32, w = (k % 32) / 8, m = k % 8;
+  const size_t row_base = (((size_t)p.tile * (p.K / 128) + j) * 16 + p.trow) * 64;
+  const uint8_t byte = p.q[row_base + 16 * w + 4 * b + m / 2];
+  const int n = (m % 2 == 0) ? (byte & 0xF) : (byte >> 4);
   return n >= 8 ? n - 16 : n;
 }
 
-// One dequantised row of a [rows][K] int4 matrix with [rows][K/32] scales.
-void dequant_row(const uint8_t *q, const uint16_t *s, int K, int row, float *out) {
-  const uint8_t *qr = q + (size_t)row * (K / 2);
-  const uint16_t *sr = s + (size_t)row * (K / 32);
-  for (int b = 0; b < K / 32; ++b) {
-    const float scale = f16_value(sr[b]);
-    for (int c = 32 * b; c < 32 * b + 32; ++c) out[c] = scale * (float)int4_at(qr, c);
+float scale_at(const RowPlace &p, int k) {
+  const int j = k / 128, b = (k % 128) / 32;
+  return f16_value(p.s[(((size_t)p.tile * (p.K / 128) + j) * 16 + p.trow) * 4 + b]);
+}
+
+// One dequantised row of an expert matrix (K = H for gate/up, I for down).
+void dequant_row(const uint8_t *blob, int H, int I, Matrix mat, int row, float *out) {
+  const RowPlace p = place_of(blob, H, I, mat, row);
+  for (int b0 = 0; b0 < p.K; b0 += 32) {
+    const float scale = scale_at(p, b0);
+    for (int k = b0; k < b0 + 32; ++k) out[k] = scale * (float)int4_at(p, k);
   }
 }
 
@@ -117,15 +156,10 @@ float silu(float z) { return z / (1.0f + std::exp(-z)); }
 // Optional g, u, h outputs are [n][I].
 void expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
                 float *g_out, float *u_out, float *h_out, float *y) {
-  Layout L = layout_of(H, I);
-  const uint8_t *gq = blob + L.gq, *uq = blob + L.uq, *dq = blob + L.dq;
-  const uint16_t *gs = (const uint16_t *)(blob + L.gs);
-  const uint16_t *us = (const uint16_t *)(blob + L.us);
-  const uint16_t *ds = (const uint16_t *)(blob + L.ds);
   std::vector<float> wg(H), wu(H), wd(I), h((size_t)n * I);
   for (int i = 0; i < I; ++i) {
-    dequant_row(gq, gs, H, i, wg.data());
-    dequant_row(uq, us, H, i, wu.data());
+    dequant_row(blob, H, I, GATE, i, wg.data());
+    dequant_row(blob, H, I, UP, i, wu.data());
     for (int t = 0; t < n; ++t) {
       const float *xt = x + (size_t)t * H;
       float g = 0.0f, u = 0.0f;
@@ -141,7 +175,7 @@ void expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
     }
   }
   for (int r = 0; r < H; ++r) {
-    dequant_row(dq, ds, I, r, wd.data());
+    dequant_row(blob, H, I, DOWN, r, wd.data());
     for (int t = 0; t < n; ++t) {
       const float *ht = h.data() + (size_t)t * I;
       float acc = 0.0f;
@@ -212,7 +246,7 @@ int oracle_route(const uint16_t *x, int T, int H, const float *Wr, const float *
 // null; y is [n][H].
 int oracle_expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
                       float *g, float *u, float *h, float *y) {
-  if (!blob || H <= 0 || I <= 0 || H % 32 || I % 32 || n < 0) return ORC_BAD_ARG;
+  if (!blob || H <= 0 || I <= 0 || H % 128 || I % 128 || n < 0) return ORC_BAD_ARG;
   expert_ffn(blob, H, I, x, n, g, u, h, y);
   return ORC_OK;
 }
@@ -227,7 +261,7 @@ int oracle_forward_routed(const uint16_t *x, int T, int H, int I, int E, int k, 
                           const int32_t *idx, const float *w, float *out) {
   if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || S < 0 || n_slots < 0)
     return ORC_BAD_ARG;
-  if (H % 32 || I % 32) return ORC_BAD_ARG;
+  if (H % 128 || I % 128) return ORC_BAD_ARG;
   // the same expert in two slots is a conflict
   for (int a = 0; a < n_slots; ++a)
     for (int b = a + 1; b < n_slots; ++b)

@@ -54,13 +54,44 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Wait for the barrier phase, backing off with nanosleep between polls (for
+// waits off the critical path, e.g. a producer waiting for a free stage).
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, int *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = global_timer_ns();
+  unsigned ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (ns < 256) ns <<= 1;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about 1 ms passes, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the barrier phase with a time limit.  On timeout the status word
 // gets STATUS_TIMEOUT and the caller must stop waiting and wind down.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       set_status(status, STATUS_TIMEOUT);
       return false;
@@ -104,9 +135,11 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], uint32_t addr) {
 }
 
 // D = A * B + C, A 16x16 f16 (row), B 16x8 f16 (col), C/D 16x8 f32.
+// (Not volatile: it has no side effects, so the compiler may interleave
+// independent MMAs.)
 __device__ __forceinline__ void mma_16816(float d[4], const uint32_t a[4], uint32_t b0,
                                           uint32_t b1, const float c[4]) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])

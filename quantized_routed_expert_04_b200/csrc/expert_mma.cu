@@ -8,26 +8,29 @@
 // with one fp16 scale per 32 consecutive k.
 //
 // How:
-//  * A persistent grid; CTA b takes a contiguous range of work items
-//    (expert, group of <= 16 pairs, 32-row weight tile), so equal numbers of
-//    weight bytes land on every SM.
-//  * Warp 0 streams each item's K range in chunks of kc through a 4-stage
-//    shared-memory ring: 32 packed weight rows as bulk async copies (one per
-//    row, rows padded by 16 bytes so the ldmatrix reads below are free of
-//    bank conflicts), their fp16 scales as 4-byte async copies, and the
-//    activation rows of the item's pairs as bulk copies.  Completion is
-//    counted on an mbarrier per stage.
-//  * Warps 1-4 split each chunk into 64-element steps.  ldmatrix hands every
-//    thread exactly the 32-bit word of nibbles its mma A fragment needs (row
-//    g and g+8, word c of a 16-byte quant block); int4x8_to_f16 turns it into
-//    exact f16 integers; two m16n8k16 MMAs per quant block give the block's
-//    integer-weight dot products in fp32, which are scaled by the block's
-//    fp16 scale into fp32 accumulators (so the only rounding of a weight is
-//    none at all -- q and the scale are applied exactly, the activation is
-//    rounded to f16).
-//  * The four warps' partial sums are added in a fixed order; SwiGLU needs
-//    no exchange because a thread holds the gate and the up value of the same
-//    (row, pair) position.
+//  * Work item = (active expert, group of <= 16 of its pairs, one 16-row
+//    weight tile): for gate/up, 8 rows of Wg and the same 8 rows of Wu (so a
+//    thread holds gate and up of one (row, pair) and SwiGLU is local); for
+//    down, 16 rows of Wd.  A persistent grid gives each CTA a contiguous range
+//    of items (equal weight bytes per CTA); inside a CTA, item q goes to warp
+//    q mod (warps per CTA), which computes it over the whole K range -- no
+//    cross-warp reduction, no rendezvous.
+//  * The blob stores a tile K-group by K-group, so any K chunk of a tile is
+//    one contiguous run of bytes.  Each warp streams its own items' chunks
+//    through a private ring of shared-memory stages: its lane 0 issues one
+//    bulk async copy of packed weights and one of scales per stage, a few
+//    stages ahead, completion counted in transaction bytes on the stage's
+//    mbarrier.  (Many independent rings per SM keep HBM busy; one ring fed by
+//    one thread could not.)
+//  * For a K group, one 16-byte shared-memory load per row hands thread
+//    (g, c) word c of all four quant blocks of rows g and g+8 -- exactly its
+//    mma.m16n8k16 A-fragment words -- and int4x8_to_f16 turns each word into
+//    exact f16 integers.  Two MMAs per quant block give the block's
+//    integer-weight dot products in fp32, scaled by the block's fp16 scale
+//    into fp32 accumulators: the weights are applied exactly; the activations
+//    are f16.
+//  * Activation fragments (x16 or h16 rows of the item's pairs) are read from
+//    L2 one group ahead, across item boundaries.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -35,84 +38,112 @@ namespace strata {
 
 namespace {
 
-__device__ __forceinline__ void cp_async_4(void *dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-// lane 0 waits, the result is shared with the warp
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *status) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-constexpr int kRedFloats = 4 * 2 * 2 * 32 * 4;  // [warp][m][n-tile][lane][4]
+__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Orders this thread's earlier shared-memory reads before later async-proxy
+// (bulk copy) writes to the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 struct Item {
   const uint8_t *blob;
-  int id, tau, pi0, ntok;
+  int tau, pi0, ntok;
 };
 
-__device__ __forceinline__ Item decode_item(const MmParams &p, const int *item_base, int &a,
-                                            int i) {
+// Per active expert, staged in shared memory at kernel start.
+struct ActiveTable {
+  const uint8_t **blob;
+  int *off, *cnt;
+};
+
+__device__ __forceinline__ Item decode_item(const MmParams &p, const ActiveTable &at,
+                                            const int *item_base, int &a, int i) {
   while (item_base[a + 1] <= i) ++a;
   Item it;
-  it.id = p.rt.active[a];
   const int rem = i - item_base[a];
   const int g = rem / p.tiles;
   it.tau = rem - g * p.tiles;
-  const int c = p.rt.cnt[it.id];
-  it.pi0 = p.rt.off[it.id] + g * kMmGroup;
-  it.ntok = min(kMmGroup, c - g * kMmGroup);
-  it.blob = p.table.ptr[it.id];
+  it.pi0 = at.off[a] + g * p.group;
+  it.ntok = min(p.group, at.cnt[a] - g * p.group);
+  it.blob = at.blob[a];
   return it;
+}
+
+// Activation fragments of one K group for a token row: v[b] = 8 f16 at
+// k0 + 32 b + 8 c (stored in the 0,4,1,5,2,6,3,7 order).  For a padding
+// column (no token, row == nullptr) the registers keep whatever they hold:
+// that column of the MMA result is never read.
+__device__ __forceinline__ void load_b(uint4 v[4], const __half *row, int k0, int cq) {
+  if (row) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v[b] = ld_nc_v4(row + k0 + 32 * b + 8 * cq);
+  }
 }
 
 }  // namespace
 
-size_t mm_smem_bytes(const MmParams &p) {
-  return (size_t)kMmStages * p.stage_bytes + (2 * kMmStages + 2) * sizeof(uint64_t) +
-         kRedFloats * sizeof(float) + (kMaxIds + 1) * sizeof(int);
+size_t mm_fixed_smem_bytes() {
+  return (size_t)kMmWarps * kMmMaxStages * sizeof(uint64_t) + kMaxIds * sizeof(void *) +
+         (3 * kMaxIds + 1) * sizeof(int) + kMmMaxPairs * sizeof(int);
 }
 
-template <bool kGateUp>
+size_t mm_smem_bytes(const MmParams &p) {
+  return (size_t)kMmWarps * p.stages * p.stage_bytes + mm_fixed_smem_bytes();
+}
+
+template <bool kGateUp, int NT>
 __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t *stages = smem;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kMmStages * p.stage_bytes);
-  uint64_t *empty = full + kMmStages;
-  uint64_t *red_full = empty + kMmStages;  // partial sums of all 4 consumer warps written
-  uint64_t *red_free = red_full + 1;       // consumer warp 0 has read them
-  float *red = reinterpret_cast<float *>(red_free + 1);
-  int *item_base = reinterpret_cast<int *>(red + kRedFloats);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kMmStages; ++s) {
-      mbar_init(&full[s], 1 + 32);  // producer's expect_tx arrive + 32 cp.async arrivals
-      mbar_init(&empty[s], 4);      // one arrive per consumer warp
-    }
-    mbar_init(red_full, 4);
-    mbar_init(red_free, 1);
-    fence_mbar_init();
-  }
+  uint8_t *ring = smem + (size_t)warp * p.stages * p.stage_bytes;   // this warp's stages
+  uint64_t *full_all =
+      reinterpret_cast<uint64_t *>(smem + (size_t)kMmWarps * p.stages * p.stage_bytes);
+  uint64_t *full = full_all + warp * kMmMaxStages;
+  ActiveTable at;
+  at.blob = reinterpret_cast<const uint8_t **>(full_all + kMmWarps * kMmMaxStages);
+  int *item_base = reinterpret_cast<int *>(at.blob + kMaxIds);
+  at.off = item_base + kMaxIds + 1;
+  at.cnt = at.off + kMaxIds;
+  int *s_ptok = at.cnt + kMaxIds;   // token of each sorted pair (gate/up)
+
+  if (lane == 0)
+    for (int s = 0; s < p.stages; ++s) mbar_init(&full[s], 1);
+  if (threadIdx.x == 0) fence_mbar_init();
   grid_dependency_wait();
 
-  // items per active expert -> exclusive prefix (warp 0, 32 ids at a time)
+  // active experts: table in shared memory, then items per expert ->
+  // exclusive prefix (warp 0, 32 experts at a time)
   const int n_active = *p.rt.n_active;
+  const int n_pairs = p.rt.off[p.n_ids];
+  for (int a = threadIdx.x; a < n_active; a += blockDim.x) {
+    const int id = p.rt.active[a];
+    at.blob[a] = p.table.ptr[id];
+    at.off[a] = p.rt.off[id];
+    at.cnt[a] = p.rt.cnt[id];
+  }
+  if (kGateUp)
+    for (int q = threadIdx.x; q < n_pairs && q < kMmMaxPairs; q += blockDim.x)
+      s_ptok[q] = p.rt.pair_tok[q];
+  __syncthreads();
   if (warp == 0) {
     int carry = 0;
     for (int a0 = 0; a0 < n_active; a0 += 32) {
       const int a = a0 + lane;
       int v = 0;
-      if (a < n_active) {
-        const int c = p.rt.cnt[p.rt.active[a]];
-        v = ((c + kMmGroup - 1) / kMmGroup) * p.tiles;
-      }
+      if (a < n_active) v = ((at.cnt[a] + p.group - 1) / p.group) * p.tiles;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -130,187 +161,209 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
   const int n_items = item_base[n_active];
   const int i_begin = (int)((long long)n_items * blockIdx.x / gridDim.x);
   const int i_end = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
-  const int n_chunks = p.K / p.kc;
-  const int steps = p.kc / 64;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    uint32_t chunk = 0;
-    int a = 0;
-    bool alive = true;
-    for (int i = i_begin; i < i_end && alive; ++i) {
-      const Item it = decode_item(p, item_base, a, i);
-      if (!it.blob) {
-        if (lane == 0) set_status(p.status, STATUS_NOT_BOUND);
-        continue;
-      }
-      int brow = 0;
-      if (lane < it.ntok) brow = kGateUp ? p.rt.pair_tok[it.pi0 + lane] : it.pi0 + lane;
-      const int m = lane >> 4;
-      const int row = it.tau * p.row_base_mul + p.row_half[m] + (lane & 15);
-      const uint8_t *wrow = it.blob + p.q_off[m] + (size_t)row * (p.K / 2);
-      const uint8_t *srow = it.blob + p.s_off[m] + (size_t)row * (p.K / 32) * 2;
-      const __half *brow_src = p.b_src + (size_t)brow * p.K;
-      for (int c = 0; c < n_chunks; ++c, ++chunk) {
-        const int s = chunk % kMmStages;
-        const uint32_t ph = (chunk / kMmStages) & 1u;
-        if (!warp_wait(&empty[s], ph ^ 1u, p.status)) {
-          alive = false;
-          break;
-        }
-        uint8_t *st = stages + s * p.stage_bytes;
-        const uint8_t *ssrc = srow + (size_t)c * (p.kc / 32) * 2;
-        uint8_t *sdst = st + p.w_bytes + lane * p.sstride;
-        for (int u = 0; u < steps; ++u) cp_async_4(sdst + 4 * u, ssrc + 4 * u);
-        cp_async_mbar_arrive_noinc(&full[s]);
-        __syncwarp();
-        if (lane == 0)
-          mbar_arrive_expect_tx(&full[s], 32u * (p.kc / 2) + (uint32_t)it.ntok * p.kc * 2u);
-        __syncwarp();
-        bulk_g2s(st + lane * p.wstride, wrow + (size_t)c * (p.kc / 2), p.kc / 2, &full[s]);
-        if (lane < it.ntok)
-          bulk_g2s(st + p.w_bytes + p.s_bytes + lane * p.bstride, brow_src + (size_t)c * p.kc,
-                   p.kc * 2, &full[s]);
-      }
-    }
-    if (!alive) {
-      // wind down: let every stage's copies land before the CTA exits
-      for (int s = 0; s < kMmStages && s < (int)chunk; ++s) {
-        const uint32_t last = chunk - 1 - ((chunk - 1 - s) % kMmStages);
-        (void)warp_wait(&full[last % kMmStages], (last / kMmStages) & 1u, p.status);
-      }
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  const int cw = warp - 1;
+  const int gpc = p.kc / 128;                    // K groups per (full) chunk
+  const int groups = p.K / 128;                  // K groups per tile row
+  const int n_chunks = (groups + gpc - 1) / gpc; // the last chunk may be shorter
+  const uint32_t q_stage = (uint32_t)p.kc * 8;   // scale offset inside a stage
   const int g = lane >> 2, cq = lane & 3;
-  uint32_t chunk = 0, done = 0;
-  int a = 0;
-  for (int i = i_begin; i < i_end; ++i) {
-    const Item it = decode_item(p, item_base, a, i);
-    if (!it.blob) continue;
-    const int ntn = (it.ntok + 7) >> 3;
-    float acc[2][2][4];
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-      for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[m][n][v] = 0.0f;
 
-    for (int c = 0; c < n_chunks; ++c, ++chunk) {
-      const int s = chunk % kMmStages;
-      const uint32_t ph = (chunk / kMmStages) & 1u;
-      if (!warp_wait(&full[s], ph, p.status)) return;
-      const uint8_t *st = stages + s * p.stage_bytes;
-      const uint32_t w_addr = smem_u32(st);
-      const uint8_t *sreg = st + p.w_bytes;
-      const uint8_t *breg = st + p.w_bytes + p.s_bytes;
-      for (int step = cw; step < steps; step += 4) {
-        float sc[2][2][2];
+  // This warp's items: i_begin + warp, + kMmWarps, ...  Items of unbound
+  // experts are skipped and flagged.
+  auto next_item = [&](int i, int &a_hint) -> int {
+    for (; i < i_end; i += kMmWarps) {
+      while (item_base[a_hint + 1] <= i) ++a_hint;
+      if (at.blob[a_hint]) return i;
+      if (lane == 0) set_status(p.status, STATUS_NOT_BOUND);
+    }
+    return i_end;
+  };
+
+  // ---- copy issue; sequence number = (own item ordinal) * n_chunks + chunk
+  int a_issue = 0;
+  int i_issue = next_item(i_begin + warp, a_issue);
+  int c_issue = 0;
+  uint32_t s_issue = 0;
+  auto issue_next = [&]() {
+    if (i_issue >= i_end) return;
+    const Item it = decode_item(p, at, item_base, a_issue, i_issue);
+    const int slot = (int)(s_issue % p.stages);
+    uint8_t *dst = ring + slot * p.stage_bytes;
+    if (lane == 0) {
+      const size_t g0 = (size_t)it.tau * groups + (size_t)c_issue * gpc;
+      const uint32_t ng = (uint32_t)min(gpc, groups - c_issue * gpc);
+      mbar_arrive_expect_tx(&full[slot], ng * (1024u + 128u));
+      bulk_g2s(dst, it.blob + p.q_off + g0 * 1024, ng * 1024u, &full[slot]);
+      bulk_g2s(dst + q_stage, it.blob + p.s_off + g0 * 128, ng * 128u, &full[slot]);
+    }
+    ++s_issue;
+    if (++c_issue == n_chunks) {
+      c_issue = 0;
+      i_issue = next_item(i_issue + kMmWarps, a_issue);
+    }
+  };
+  for (int s = 0; s < p.stages; ++s) issue_next();
+
+  // ---- compute
+  auto act_row = [&](const Item &it, int nt) -> const __half * {
+    const int n = nt * 8 + g;
+    if (n >= it.ntok) return nullptr;
+    int src;
+    if (kGateUp) {
+      const int q = it.pi0 + n;
+      src = q < kMmMaxPairs ? s_ptok[q] : p.rt.pair_tok[q];
+    } else {
+      src = it.pi0 + n;
+    }
+    return p.b_src + (size_t)src * p.K;
+  };
+  uint4 bb0[NT][4], bb1[NT][4];
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            const uint32_t v =
-                *reinterpret_cast<const uint32_t *>(sreg + (m * 16 + g + 8 * hr) * p.sstride + step * 4);
-            const float2 f = __half22float2(bits_h2(v));
-            sc[m][hr][0] = f.x;
-            sc[m][hr][1] = f.y;
-          }
-        uint32_t f16w[2][4][4];
+    for (int b = 0; b < 4; ++b) bb0[nt][b] = bb1[nt][b] = make_uint4(0u, 0u, 0u, 0u);
+  int pb = 0;  // buffer holding the current group's fragments
+  int a = 0;
+  int i = next_item(i_begin + warp, a);
+  if (i < i_end) {
+    int a_tmp = a;
+    const Item it0 = decode_item(p, at, item_base, a_tmp, i);
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          uint32_t q[4];
-          const int r = m * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-          ldmatrix_x4(q, w_addr + r * p.wstride + step * 32 + (lane >> 4) * 16);
+    for (int nt = 0; nt < NT; ++nt) load_b(bb0[nt], act_row(it0, nt), 0, cq);
+  }
+  uint32_t s_use = 0;
+  while (i < i_end) {
+    const Item it = decode_item(p, at, item_base, a, i);
+    const int ntn = (it.ntok + 7) >> 3;
+    int a_nx = a;
+    const int i_nx = next_item(i + kMmWarps, a_nx);
+    const __half *row_cur[NT], *row_nx[NT];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) int4x8_to_f16(q[j], f16w[m][j]);
-        }
+    for (int nt = 0; nt < NT; ++nt) {
+      row_cur[nt] = act_row(it, nt);
+      row_nx[nt] = nullptr;
+    }
+    if (i_nx < i_end) {
+      int a_tmp = a_nx;
+      const Item it_nx = decode_item(p, at, item_base, a_tmp, i_nx);
 #pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
+      for (int nt = 0; nt < NT; ++nt) row_nx[nt] = act_row(it_nx, nt);
+    }
+    float acc[NT][4];
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            if (nt < ntn) {
-              const uint4 bv = *reinterpret_cast<const uint4 *>(
-                  breg + (nt * 8 + g) * p.bstride + (step * 64 + bb * 32 + cq * 8) * 2);
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-              for (int m = 0; m < 2; ++m) {
-                const uint32_t a0[4] = {f16w[m][2 * bb][0], f16w[m][2 * bb + 1][0],
-                                        f16w[m][2 * bb][1], f16w[m][2 * bb + 1][1]};
-                const uint32_t a1[4] = {f16w[m][2 * bb][2], f16w[m][2 * bb + 1][2],
-                                        f16w[m][2 * bb][3], f16w[m][2 * bb + 1][3]};
-                const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-                float d[4];
-                mma_16816(d, a0, bv.x, bv.y, zero);
-                mma_16816(d, a1, bv.z, bv.w, d);
-                acc[m][nt][0] = fmaf(sc[m][0][bb], d[0], acc[m][nt][0]);
-                acc[m][nt][1] = fmaf(sc[m][0][bb], d[1], acc[m][nt][1]);
-                acc[m][nt][2] = fmaf(sc[m][1][bb], d[2], acc[m][nt][2]);
-                acc[m][nt][3] = fmaf(sc[m][1][bb], d[3], acc[m][nt][3]);
-              }
+      for (int v = 0; v < 4; ++v) acc[n][v] = 0.0f;
+
+    for (int c = 0; c < n_chunks; ++c, ++s_use) {
+      const int slot = (int)(s_use % p.stages);
+      if (!warp_wait(&full[slot], (s_use / p.stages) & 1u, p.status)) return;
+      const uint8_t *stq = ring + slot * p.stage_bytes;
+      const uint8_t *sts = stq + q_stage;
+      const int ng = min(gpc, groups - c * gpc);
+#pragma unroll 4
+      for (int j = 0; j < ng; ++j) {
+        // fragments of the next group: this item, else the next item
+        {
+          const int G_next = c * gpc + j + 1;
+          const bool same = G_next < groups;
+          if (same || i_nx < i_end) {
+            const int k0 = same ? G_next * 128 : 0;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const __half *r = same ? row_cur[nt] : row_nx[nt];
+              if (pb == 0) load_b(bb1[nt], r, k0, cq);
+              else load_b(bb0[nt], r, k0, cq);
             }
           }
         }
+        // weights and scales of rows g and g + 8
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(stq + j * 1024 + g * 64 + cq * 16);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(stq + j * 1024 + (g + 8) * 64 + cq * 16);
+        const uint2 s0 = *reinterpret_cast<const uint2 *>(sts + j * 128 + g * 8);
+        const uint2 s1 = *reinterpret_cast<const uint2 *>(sts + j * 128 + (g + 8) * 8);
+        const uint32_t wr0[4] = {w0.x, w0.y, w0.z, w0.w};  // word c of blocks 0..3, row g
+        const uint32_t wr1[4] = {w1.x, w1.y, w1.z, w1.w};  // row g + 8
+        uint32_t f0[4][4], f1[4][4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          int4x8_to_f16(wr0[b], f0[b]);
+          int4x8_to_f16(wr1[b], f1[b]);
+        }
+        float sc0[4], sc1[4];
+        {
+          float2 f;
+          f = __half22float2(bits_h2(s0.x)); sc0[0] = f.x; sc0[1] = f.y;
+          f = __half22float2(bits_h2(s0.y)); sc0[2] = f.x; sc0[3] = f.y;
+          f = __half22float2(bits_h2(s1.x)); sc1[0] = f.x; sc1[1] = f.y;
+          f = __half22float2(bits_h2(s1.y)); sc1[2] = f.x; sc1[3] = f.y;
+        }
+        auto mma_group = [&](const uint4 (&bv)[NT][4]) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            if (NT == 1 || nt < ntn) {
+              float d[4][4];
+              const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const uint32_t a0[4] = {f0[b][0], f1[b][0], f0[b][1], f1[b][1]};
+                mma_16816(d[b], a0, bv[nt][b].x, bv[nt][b].y, zero);
+              }
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const uint32_t a1[4] = {f0[b][2], f1[b][2], f0[b][3], f1[b][3]};
+                mma_16816(d[b], a1, bv[nt][b].z, bv[nt][b].w, d[b]);
+              }
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                acc[nt][0] = fmaf(sc0[b], d[b][0], acc[nt][0]);
+                acc[nt][1] = fmaf(sc0[b], d[b][1], acc[nt][1]);
+                acc[nt][2] = fmaf(sc1[b], d[b][2], acc[nt][2]);
+                acc[nt][3] = fmaf(sc1[b], d[b][3], acc[nt][3]);
+              }
+            }
+          }
+        };
+        if (pb == 0) mma_group(bb0); else mma_group(bb1);
+        pb ^= 1;
       }
+      // the stage's bytes are in registers now: refill it
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      issue_next();
     }
 
-    // ------------------------------------------------------------ epilogue
-    // the previous item's partial sums must have been read
-    if (!warp_wait(red_free, (done & 1u) ^ 1u, p.status)) return;
-    float *mine = red + cw * (2 * 2 * 32 * 4);
+    // ---- epilogue: this warp holds the complete sums of the item
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int nt = 0; nt < NT; ++nt) {
+      if (nt >= ntn) continue;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) mine[((m * 2 + nt) * 32 + lane) * 4 + v] = acc[m][nt][v];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(red_full);
-    if (cw == 0) {
-      if (!warp_wait(red_full, done & 1u, p.status)) return;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        if (nt >= ntn) continue;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int rr = g + 8 * (v >> 1);
-          const int n = nt * 8 + 2 * cq + (v & 1);
-          if (n >= it.ntok) continue;
-          float fin[2];
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int o = ((m * 2 + nt) * 32 + lane) * 4 + v;
-            fin[m] = ((red[o] + red[o + 2 * 2 * 32 * 4]) + red[o + 2 * 2 * 2 * 32 * 4]) +
-                     red[o + 3 * 2 * 2 * 32 * 4];
-          }
-          const size_t prow = (size_t)(it.pi0 + n) * p.out_ld;
-          if (kGateUp) {
-            const float gv = fin[0], uv = fin[1];
-            const float h = gv / (1.0f + expf(-gv)) * uv;
-            const int ii = it.tau * 16 + rr;
-            // stored like the packed activations: group of 8 in order 0,4,1,5,2,6,3,7
-            const int pos = (ii & ~7) | (((ii & 3) << 1) | ((ii >> 2) & 1));
-            p.h_out[prow + pos] = __float2half_rn(h);
-          } else {
-            const int r0 = it.tau * 32 + rr;
-            p.y_out[prow + r0] = fin[0];
-            p.y_out[prow + r0 + 16] = fin[1];
-          }
+      for (int v = 0; v < 2; ++v) {
+        const int n = nt * 8 + 2 * cq + v;
+        if (n >= it.ntok) continue;
+        const size_t prow = (size_t)(it.pi0 + n) * p.out_ld;
+        if (kGateUp) {
+          // acc[v]: gate row i, acc[v + 2]: up row i, i = 8 tau + g
+          const float gv = acc[nt][v], uv = acc[nt][v + 2];
+          const float h = gv / (1.0f + expf(-gv)) * uv;
+          const int ii = it.tau * 8 + g;
+          // stored like the packed activations: group of 8 in order 0,4,1,5,2,6,3,7
+          const int pos = (ii & ~7) | (((ii & 3) << 1) | ((ii >> 2) & 1));
+          p.h_out[prow + pos] = __float2half_rn(h);
+        } else {
+          const int r0 = it.tau * 16 + g;
+          p.y_out[prow + r0] = acc[nt][v];
+          p.y_out[prow + r0 + 8] = acc[nt][v + 2];
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(red_free);
     }
-    ++done;
+    i = i_nx;
+    a = a_nx;
   }
 }
 
-template __global__ void expert_mma_kernel<true>(MmParams);
-template __global__ void expert_mma_kernel<false>(MmParams);
+template __global__ void expert_mma_kernel<true, 1>(MmParams);
+template __global__ void expert_mma_kernel<false, 1>(MmParams);
+template __global__ void expert_mma_kernel<true, 2>(MmParams);
+template __global__ void expert_mma_kernel<false, 2>(MmParams);
 
 }  // namespace strata

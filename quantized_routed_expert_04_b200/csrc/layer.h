@@ -22,21 +22,20 @@ enum : int {
   STATUS_BOUNDS = 8,         // a computed offset fell outside its buffer
 };
 
-// Byte offsets of the six sections of an expert blob.
+// Byte offsets of the four sections of an expert blob: gate+up weights,
+// down weights, gate+up scales, down scales (see include/strata_moe.h).
 struct BlobLayout {
-  size_t gq, uq, dq, gs, us, ds, total;
+  size_t guq, dq, gus, ds, total;
 };
 
 inline BlobLayout blob_layout(int H, int I) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   BlobLayout L;
   size_t off = 0;
-  L.gq = off; off = up(off + (size_t)I * H / 2);
-  L.uq = off; off = up(off + (size_t)I * H / 2);
-  L.dq = off; off = up(off + (size_t)H * I / 2);
-  L.gs = off; off = up(off + (size_t)I * (H / 32) * 2);
-  L.us = off; off = up(off + (size_t)I * (H / 32) * 2);
-  L.ds = off; off = up(off + (size_t)H * (I / 32) * 2);
+  L.guq = off; off = up(off + (size_t)I * H);
+  L.dq = off;  off = up(off + (size_t)H * I / 2);
+  L.gus = off; off = up(off + (size_t)I * H / 8);
+  L.ds = off;  off = up(off + (size_t)H * I / 16);
   L.total = off;
   return L;
 }

@@ -341,4 +341,237 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
   *reinterpret_cast<uint2 *>(out + (size_t)t * H + r) = packed;
 }
 
+// ---------------------------------------------------------------- small batches
+// Routing of up to kSmallT tokens in one launch (decode).  Every block
+// computes the logits of one expert (8 warps split h; per-warp double sums
+// added in a fixed order) and packs a slice of the activations; the last
+// block to finish -- found with a device counter, each block's writes released
+// by a fence before its counter increment and acquired by the last block with
+// a fence after it -- takes the top-k of every token and, for a forward call,
+// buckets the pairs.  The last block resets the counter for the next launch.
+namespace {
+
+__device__ void topk_token_warp(const float *__restrict__ logit_row, int E, int k, int lane,
+                                int32_t *idx_out, float *w_out, int *s_idx) {
+  constexpr int kPer = kMaxExperts / 32;
+  float v[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? __ldcg(logit_row + e) : -INFINITY;
+  }
+  unsigned taken = 0;
+  float l0 = 0.0f, z = 0.0f, my_l = 0.0f;
+  int my_e = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (j == 0) l0 = bv;
+    const float pj = expf(bv - l0);
+    z += pj;
+    if (lane == j) {  // lane j keeps selection j (k <= 32)
+      my_l = bv;
+      my_e = be;
+    }
+  }
+  if (lane < k) {
+    idx_out[lane] = my_e;
+    w_out[lane] = expf(my_l - l0) / z;
+    if (s_idx) s_idx[lane] = my_e;
+  }
+}
+
+// Bucketing of T*k routed pairs (ids in s_idx, shared memory) plus S shared
+// experts by one block of 256 threads.
+__device__ void bucket_block(const int *s_idx, int T, int k, int E, int S, const Routing &rt,
+                             int *status, int *s_cnt, int *s_off) {
+  const int tid = threadIdx.x;
+  const int nid = E + S;
+  const int n = T * k;
+  const int kS = k + S;
+  for (int i = tid; i < nid; i += blockDim.x) s_cnt[i] = i < E ? 0 : T;
+  __syncthreads();
+  for (int p = tid; p < n; p += blockDim.x) {
+    const int e = s_idx[p];
+    if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid < 32) {
+    int carry = 0, acarry = 0;
+    for (int i0 = 0; i0 < nid; i0 += 32) {
+      const int i = i0 + tid;
+      const int c = i < nid ? s_cnt[i] : 0;
+      const int f = c > 0;
+      int inc = c, finc = f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, inc, o);
+        const int b = __shfl_up_sync(0xffffffffu, finc, o);
+        if (tid >= o) {
+          inc += a;
+          finc += b;
+        }
+      }
+      if (i < nid) {
+        const int off = carry + inc - c;
+        s_off[i] = off;
+        rt.off[i] = off;
+        rt.cnt[i] = c;
+        if (f) rt.active[acarry + finc - 1] = i;
+      }
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+      acarry += __shfl_sync(0xffffffffu, finc, 31);
+    }
+    if (tid == 0) {
+      rt.off[nid] = carry;
+      *rt.n_active = acarry;
+    }
+  }
+  __syncthreads();
+  for (int p = tid; p < n; p += blockDim.x) {
+    const int e = s_idx[p];
+    const int t = p / k, j = p - (p / k) * k;
+    if (e < 0 || e >= E) {
+      set_status(status, STATUS_BAD_ROUTING);
+      rt.inv[(size_t)t * kS + j] = -1;
+      continue;
+    }
+    int rank = 0;
+    for (int q = 0; q < p; ++q) rank += (s_idx[q] == e);
+    const int pos = s_off[e] + rank;
+    rt.pair_tok[pos] = t;
+    rt.pair_j[pos] = j;
+    rt.inv[(size_t)t * kS + j] = pos;
+  }
+  for (int q = tid; q < T * S; q += blockDim.x) {
+    const int s = q / T, t = q - (q / T) * T;
+    const int pos = s_off[E + s] + t;
+    rt.pair_tok[pos] = t;
+    rt.pair_j[pos] = k + s;
+    rt.inv[(size_t)t * kS + k + s] = pos;
+  }
+}
+
+__device__ void pack_x_range(const __nv_bfloat16 *__restrict__ x, __half *__restrict__ x16, int g0,
+                             int g1) {
+  for (int i = g0 + (int)threadIdx.x; i < g1; i += blockDim.x) {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)i * 8);
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
+    const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
+    uint4 o;
+    o.x = h2_bits(__floats2half2_rn(f0.x, f2.x));
+    o.y = h2_bits(__floats2half2_rn(f0.y, f2.y));
+    o.z = h2_bits(__floats2half2_rn(f1.x, f3.x));
+    o.w = h2_bits(__floats2half2_rn(f1.y, f3.y));
+    *reinterpret_cast<uint4 *>(x16 + (size_t)i * 8) = o;
+  }
+}
+
+}  // namespace
+
+template <bool kRoute, bool kBucket>
+__global__ void __launch_bounds__(256) route_small_kernel(SmallRouteParams p) {
+  grid_dependency_wait();
+  __shared__ double s_part[8][kSmallT];
+  __shared__ int s_idx[kSmallT * kMaxTopK];
+  __shared__ int s_cnt[kMaxIds], s_off[kMaxIds];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = p.T, H = p.H, E = p.E, k = p.k;
+
+  if (kBucket) {
+    const int n8 = T * H / 8;
+    pack_x_range(p.x, p.x16, (int)((long long)n8 * blockIdx.x / gridDim.x),
+                 (int)((long long)n8 * (blockIdx.x + 1) / gridDim.x));
+  }
+  if (kRoute) {
+    const int e = blockIdx.x;
+    const float *wr = p.W + (size_t)e * H;
+    const int span = H / 8;
+    const int h0 = warp * span;
+    for (int t0 = 0; t0 < T; t0 += 8) {
+      const int nt = min(8, T - t0);
+      double acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+#pragma unroll 2
+      for (int h = h0 + lane * 4; h < h0 + span; h += 128) {
+        const float4 wv = *reinterpret_cast<const float4 *>(wr + h);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (i < nt) {
+            const uint2 raw = *reinterpret_cast<const uint2 *>(p.x + (size_t)(t0 + i) * H + h);
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+            acc[i] = fma((double)a.x, (double)wv.x, acc[i]);
+            acc[i] = fma((double)a.y, (double)wv.y, acc[i]);
+            acc[i] = fma((double)b.x, (double)wv.z, acc[i]);
+            acc[i] = fma((double)b.y, (double)wv.w, acc[i]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+      }
+      if (lane == 0)
+        for (int i = 0; i < nt; ++i) s_part[warp][t0 + i] = acc[i];
+    }
+    __syncthreads();
+    for (int t = tid; t < T; t += blockDim.x) {
+      double v = s_part[0][t];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) v += s_part[w][t];
+      if (p.bias) v += (double)p.bias[e];
+      p.logits[(size_t)t * E + e] = (float)v;
+    }
+  }
+  // ---- hand over to the last block
+  if (gridDim.x > 1) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int prev = atomicAdd(p.counter, 1);
+      s_last = prev == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+  }
+  if (kRoute) {
+    for (int t = warp; t < T; t += 8)
+      topk_token_warp(p.logits + (size_t)t * E, E, k, lane, p.idx + (size_t)t * k,
+                      p.w + (size_t)t * k, kBucket ? s_idx + t * k : nullptr);
+  } else {
+    for (int q = tid; q < T * k; q += blockDim.x) s_idx[q] = p.idx[q];
+  }
+  __syncthreads();
+  if (kBucket) bucket_block(s_idx, T, k, E, p.S, p.rt, p.status, s_cnt, s_off);
+  if (tid == 0 && gridDim.x > 1) *p.counter = 0;
+}
+
+template __global__ void route_small_kernel<true, true>(SmallRouteParams);
+template __global__ void route_small_kernel<true, false>(SmallRouteParams);
+template __global__ void route_small_kernel<false, true>(SmallRouteParams);
+
 }  // namespace strata

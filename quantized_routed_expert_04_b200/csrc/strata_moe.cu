@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -52,6 +53,7 @@ struct strata_moe {
   __half *h16 = nullptr;
   float *y = nullptr;
   int *status = nullptr;    // device status word (own allocation)
+  int *counter = nullptr;   // last-block counter of the small-batch routing kernel
   int last_bits = 0;
 
   // per-kernel timing
@@ -172,53 +174,45 @@ ExpertTable make_table(const strata_moe *h) {
   return t;
 }
 
-// Largest multiple of 64 that divides K and is at most 1024.
-int pick_kc(int K) {
-  int best = 64;
-  for (int kc = 64; kc <= 1024 && kc <= K; kc += 64)
-    if (K % kc == 0) best = kc;
-  return best;
+// Stage size and count of the per-warp rings: K chunks of 512 elements (4 KB
+// of packed weights per copy; the last chunk of a row may be shorter), as
+// many stages as fit.
+void pick_chunk(int K, int *kc_out, int *stages_out) {
+  const size_t avail = 232448 - 1024 - mm_fixed_smem_bytes();
+  const size_t per_warp = avail / kMmWarps;
+  const int kc = std::min(K, 512);
+  const size_t stage = align_up((size_t)kc * 9, 128);
+  *kc_out = kc;
+  *stages_out = (int)std::max<size_t>(2, std::min<size_t>(kMmMaxStages, per_warp / stage));
 }
 
-MmParams mm_params(const strata_moe *h, bool gate_up, const ExpertTable &table) {
+MmParams mm_params(const strata_moe *h, bool gate_up, const ExpertTable &table, int T) {
   MmParams p;
   std::memset(&p, 0, sizeof p);
   p.table = table;
   p.rt = h->rt;
   p.E = h->E;
   p.K = gate_up ? h->H : h->I;
-  p.kc = pick_kc(p.K);
+  pick_chunk(p.K, &p.kc, &p.stages);
+  p.group = T <= 8 ? 8 : kMmMaxGroup;
+  p.n_ids = h->E + h->S;
   if (gate_up) {
-    p.tiles = h->I / 16;
-    p.q_off[0] = h->layout.gq;
-    p.q_off[1] = h->layout.uq;
-    p.s_off[0] = h->layout.gs;
-    p.s_off[1] = h->layout.us;
-    p.row_base_mul = 16;
-    p.row_half[0] = 0;
-    p.row_half[1] = 0;
+    p.tiles = h->I / 8;
+    p.q_off = h->layout.guq;
+    p.s_off = h->layout.gus;
     p.b_src = h->x16;
     p.out_ld = h->I;
   } else {
-    p.tiles = h->H / 32;
-    p.q_off[0] = p.q_off[1] = h->layout.dq;
-    p.s_off[0] = p.s_off[1] = h->layout.ds;
-    p.row_base_mul = 32;
-    p.row_half[0] = 0;
-    p.row_half[1] = 16;
+    p.tiles = h->H / 16;
+    p.q_off = h->layout.dq;
+    p.s_off = h->layout.ds;
     p.b_src = h->h16;
     p.out_ld = h->H;
   }
   p.h_out = h->h16;
   p.y_out = h->y;
   p.status = h->status;
-  p.wstride = p.kc / 2 + 16;
-  const int sbytes = p.kc / 16;
-  p.sstride = ((sbytes / 4) % 2 == 0) ? sbytes + 4 : sbytes;
-  p.bstride = 2 * p.kc + 64;
-  p.w_bytes = 32 * p.wstride;
-  p.s_bytes = (int)align_up(32 * p.sstride, 16);
-  p.stage_bytes = (int)align_up(p.w_bytes + p.s_bytes + kMmGroup * p.bstride, 128);
+  p.stage_bytes = (int)align_up((size_t)p.kc * 9, 128);
   return p;
 }
 
@@ -229,31 +223,36 @@ strata_status check_common(strata_moe *h, const void *x, int T, cudaStream_t) {
 }
 
 // Bucketing + the expert passes + combine, given idx/w in device memory.
+// routed_small: the small-batch routing kernel already bucketed the pairs and
+// packed the activations.
 strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *idx, const float *w,
-                          void *out, cudaStream_t stream) {
+                          void *out, cudaStream_t stream, bool routed_small) {
   const ExpertTable table = make_table(h);
   const int kS = h->k + h->S;
   const int nid = h->E + h->S;
-  cudaError_t e;
-  e = cudaMemsetAsync(h->rt.cnt, 0, sizeof(int) * nid, stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(h->rt.inv, 0xFF, sizeof(int) * (size_t)T * kS, stream);
-  if (e != cudaSuccess) return cuda_status(e);
-  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
-  const int n8 = T * h->H / 8;
-  e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb, n8,
-             h->x16);
-  if (e == cudaSuccess)
-    e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
-               stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
-  if (e == cudaSuccess)
-    e = launch(h, PH_BUCKET, bucket_fill_kernel, dim3(nid), dim3(256), 0, stream, true, idx, T,
-               h->k, h->E, h->S, h->rt);
-  if (e != cudaSuccess) return cuda_status(e);
+  cudaError_t e = cudaSuccess;
+  if (!routed_small) {
+    e = cudaMemsetAsync(h->rt.cnt, 0, sizeof(int) * nid, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->rt.inv, 0xFF, sizeof(int) * (size_t)T * kS, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+    const int n8 = T * h->H / 8;
+    e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb,
+               n8, h->x16);
+    if (e == cudaSuccess)
+      e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
+                 stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
+    if (e == cudaSuccess)
+      e = launch(h, PH_BUCKET, bucket_fill_kernel, dim3(nid), dim3(256), 0, stream, true, idx, T,
+                 h->k, h->E, h->S, h->rt);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   for (int pass = 0; pass < 2; ++pass) {
     const bool gu = pass == 0;
-    MmParams p = mm_params(h, gu, table);
+    MmParams p = mm_params(h, gu, table, T);
     const size_t smem = mm_smem_bytes(p);
-    auto kern = gu ? expert_mma_kernel<true> : expert_mma_kernel<false>;
+    auto kern = p.group <= 8 ? (gu ? expert_mma_kernel<true, 1> : expert_mma_kernel<false, 1>)
+                             : (gu ? expert_mma_kernel<true, 2> : expert_mma_kernel<false, 2>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
       e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(kMmThreads), smem,
@@ -266,19 +265,44 @@ strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *id
   return cuda_status(e);
 }
 
+SmallRouteParams small_params(strata_moe *h, const void *x, int T, float *logits, int32_t *idx,
+                              float *w) {
+  SmallRouteParams p;
+  p.x = static_cast<const __nv_bfloat16 *>(x);
+  p.W = h->router_W;
+  p.bias = h->router_b;
+  p.T = T;
+  p.H = h->H;
+  p.E = h->E;
+  p.k = h->k;
+  p.S = h->S;
+  p.logits = logits;
+  p.idx = idx;
+  p.w = w;
+  p.rt = h->rt;
+  p.x16 = h->x16;
+  p.counter = h->counter;
+  p.status = h->status;
+  return p;
+}
+
+// Router + top-k (+ bucketing and activation pack when `bucket`).
 strata_status run_router(strata_moe *h, const void *x, int T, float *logits, int32_t *idx,
-                         float *w, cudaStream_t stream) {
+                         float *w, cudaStream_t stream, bool bucket) {
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
   cudaError_t e;
-  if (T <= 64) {
-    const int warps = 8;
-    e = launch(h, PH_ROUTER, router_gemv_kernel, dim3((h->E + warps - 1) / warps),
-               dim3(32 * warps), 0, stream, false, xb, h->router_W, h->router_b, T, h->H, h->E,
-               logits);
-  } else {
-    e = launch(h, PH_ROUTER, router_gemm_kernel, dim3((T + 63) / 64, (h->E + 63) / 64), dim3(256),
-               0, stream, false, xb, h->router_W, h->router_b, T, h->H, h->E, logits);
+  if (T <= kSmallT) {
+    const SmallRouteParams p = small_params(h, x, T, logits, idx, w);
+    if (bucket)
+      e = launch(h, PH_ROUTER, route_small_kernel<true, true>, dim3(h->E), dim3(256), 0, stream,
+                 false, p);
+    else
+      e = launch(h, PH_ROUTER, route_small_kernel<true, false>, dim3(h->E), dim3(256), 0, stream,
+                 false, p);
+    return cuda_status(e);
   }
+  e = launch(h, PH_ROUTER, router_gemm_kernel, dim3((T + 63) / 64, (h->E + 63) / 64), dim3(256), 0,
+             stream, false, xb, h->router_W, h->router_b, T, h->H, h->E, logits);
   if (e == cudaSuccess)
     e = launch(h, PH_TOPK, topk_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, true, logits, T,
                h->E, h->k, idx, w);
@@ -305,7 +329,7 @@ const char *strata_status_str(strata_status s) {
 }
 
 size_t strata_moe_expert_bytes(int hidden, int inter) {
-  if (hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return 0;
+  if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128) return 0;
   return blob_layout(hidden, inter).total;
 }
 
@@ -313,7 +337,7 @@ strata_status strata_moe_create(int hidden, int inter, int n_experts, int top_k,
                                 int n_slots, strata_moe **out) {
   if (!out) return STRATA_ERR_INVALID_ARG;
   *out = nullptr;
-  if (hidden <= 0 || inter <= 0 || hidden % 64 || inter % 64) return STRATA_ERR_INVALID_ARG;
+  if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128) return STRATA_ERR_INVALID_ARG;
   if (n_experts < 1 || n_experts > kMaxExperts) return STRATA_ERR_INVALID_ARG;
   if (top_k < 1 || top_k > n_experts || top_k > kMaxTopK) return STRATA_ERR_INVALID_ARG;
   if (n_shared < 0 || n_shared > kMaxShared) return STRATA_ERR_INVALID_ARG;
@@ -333,8 +357,9 @@ strata_status strata_moe_create(int hidden, int inter, int n_experts, int top_k,
   h->shared_ptr.assign(n_shared, nullptr);
   cudaError_t e = cudaGetDevice(&h->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
-  if (e == cudaSuccess) e = cudaMalloc(&h->status, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMalloc(&h->status, 64);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, 64);
+  h->counter = h->status + 16;
   if (e != cudaSuccess) {
     cudaGetLastError();
     if (h->status) cudaFree(h->status);
@@ -415,7 +440,7 @@ strata_status strata_moe_route(strata_moe *h, const void *x_bf16, int n_tokens, 
   st = grow_workspace(h, n_tokens);
   if (st != STRATA_OK) return st;
   return run_router(h, x_bf16, n_tokens, logits_out ? logits_out : h->logits, idx_out, w_out,
-                    stream);
+                    stream, false);
 }
 
 strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens, void *out_bf16,
@@ -429,9 +454,10 @@ strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens
   if (!out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 15)) return STRATA_ERR_INVALID_ARG;
   st = grow_workspace(h, n_tokens);
   if (st != STRATA_OK) return st;
-  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream);
+  const bool small = n_tokens <= kSmallT;
+  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream, small);
   if (st != STRATA_OK) return st;
-  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream);
+  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream, small);
 }
 
 strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n_tokens,
@@ -446,7 +472,15 @@ strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n
     return STRATA_ERR_INVALID_ARG;
   st = grow_workspace(h, n_tokens);
   if (st != STRATA_OK) return st;
-  return run_experts(h, x_bf16, n_tokens, idx, w, out_bf16, stream);
+  const bool small = n_tokens <= kSmallT;
+  if (small) {
+    const SmallRouteParams p = small_params(h, x_bf16, n_tokens, nullptr, const_cast<int32_t *>(idx),
+                                            nullptr);
+    cudaError_t e = launch(h, PH_BUCKET, route_small_kernel<false, true>, dim3(1), dim3(256), 0,
+                           stream, false, p);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return run_experts(h, x_bf16, n_tokens, idx, w, out_bf16, stream, small);
 }
 
 strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream) {

@@ -13,20 +13,27 @@ arena, and a 256-expert prefill layer.  The pages (Strata "docs/MAC.md",
 same problem on real checkpoints; nothing here reads a checkpoint.
 
 Expert blob format (one contiguous blob per expert, after Strata "docs/MAC.md",
-which keeps "each expert's three matrices together"):
+"What you need", which keeps each expert's matrices together so one request
+reads an expert).  H = hidden, I = inter, both multiples of 128.
 
-    section   shape            type
-    Wg_q      [I][H/2]         u8   gate weights, 2 int4 per byte
-    Wu_q      [I][H/2]         u8   up weights
-    Wd_q      [H][I/2]         u8   down weights
-    Wg_s      [I][H/32]        f16  one scale per 32 consecutive K elements
-    Wu_s      [I][H/32]        f16
-    Wd_s      [H][I/32]        f16
+    section  content                                   bytes
+    GU_q     gate + up int4 weights, I/8 row tiles      I*H
+    D_q      down int4 weights, H/16 row tiles          H*I/2
+    GU_s     gate + up fp16 scales, same tiling         I*H/8
+    D_s      down fp16 scales, same tiling              H*I/16
 
-Each section starts at a multiple of 256 bytes from the blob start and the
-blob size is rounded up to 256 bytes.  Byte j of a row holds element 2j in its
-low nibble and element 2j+1 in its high nibble; a nibble is a two's-complement
-int4 in [-8, 7].  The dequantised weight is float(scale) * q.
+Each section starts at a multiple of 256 bytes; the blob size is rounded up
+to 256 bytes.  A row tile has 16 rows: gate/up tile t holds rows 8t..8t+7 of
+Wg as tile rows 0..7 and the same rows of Wu as tile rows 8..15; down tile t
+holds rows 16t..16t+15 of Wd.  A tile is stored K-group by K-group (128
+consecutive K elements), each group as its 16 rows of 64 bytes (q) or of four
+fp16 scales (one per block of 32 K elements, block b = elements 32b..32b+31
+of the group).  Inside the 64 bytes of one row and group, byte 16w + 4b + m/2
+(w, b in 0..3, m in 0..7) holds element 32b + 8w + m, in the low nibble for
+even m; a nibble is a two's-complement int4 in [-8, 7].  The weight is
+float(scale) * q.  (So the 16 bytes at 16w are word w of each of the four
+blocks: one 16-byte load gives the word of every block that an mma.m16n8k16
+A fragment needs.)
 """
 from __future__ import annotations
 
@@ -103,11 +110,9 @@ def _align256(v: int) -> int:
 
 
 def blob_layout(hidden: int, inter: int) -> dict:
-    """Byte offsets of the six sections and the blob size."""
+    """Byte offsets of the four sections and the blob size."""
     H, I = hidden, inter
-    sizes = [("gq", I * H // 2), ("uq", I * H // 2), ("dq", H * I // 2),
-             ("gs", I * (H // QBLOCK) * 2), ("us", I * (H // QBLOCK) * 2),
-             ("ds", H * (I // QBLOCK) * 2)]
+    sizes = [("guq", I * H), ("dq", H * I // 2), ("gus", I * H // 8), ("ds", H * I // 16)]
     off, out = 0, {}
     for name, size in sizes:
         out[name] = off
@@ -120,13 +125,49 @@ def expert_bytes(hidden: int, inter: int) -> int:
     return blob_layout(hidden, inter)["total"]
 
 
-def pack_int4(q: np.ndarray) -> np.ndarray:
-    """int array [rows][K] with values in [-8, 7] -> u8 [rows][K/2]."""
+def _check_int4(q):
     q = np.asarray(q)
     if q.min(initial=0) < -8 or q.max(initial=0) > 7:
         raise ValueError("int4 values must lie in [-8, 7]")
-    n = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    return q
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """Plain row-major packing: int [rows][K] -> u8 [rows][K/2] (element 2j in
+    the low nibble of byte j).  Used to state the nibble convention."""
+    n = (_check_int4(q).astype(np.int16) & 0xF).astype(np.uint8)
     return (n[..., 0::2] | (n[..., 1::2] << 4)).astype(np.uint8)
+
+
+def pack_tiles(q_tiles: np.ndarray) -> np.ndarray:
+    """int [tiles][16][K] -> u8 [tiles][K/128][16][64] in the group layout."""
+    q = _check_int4(q_tiles)
+    t, r, K = q.shape
+    assert r == 16 and K % 128 == 0
+    # element 32b + 8w + m of a group -> (b, w, m); stored in order (w, b, m)
+    g = q.reshape(t, 16, K // 128, 4, 4, 8).transpose(0, 2, 1, 4, 3, 5)
+    n = (g.astype(np.int16) & 0xF).astype(np.uint8)
+    packed = n[..., 0::2] | (n[..., 1::2] << 4)          # [t][G][16][w][b][4]
+    return packed.reshape(t, K // 128, 16, 64)
+
+
+def pack_tile_scales(s_tiles: np.ndarray) -> np.ndarray:
+    """f16 [tiles][16][K/32] -> f16 [tiles][K/128][16][4]."""
+    s = np.asarray(s_tiles, np.float16)
+    t, r, nb = s.shape
+    return s.reshape(t, 16, nb // 4, 4).transpose(0, 2, 1, 3).copy()
+
+
+def gate_up_tiles(wg: np.ndarray, wu: np.ndarray) -> np.ndarray:
+    """[I][K] gate and up arrays -> [I/8][16][K] tiles (8 gate rows, 8 up rows)."""
+    wg, wu = np.asarray(wg), np.asarray(wu)
+    I = wg.shape[0]
+    return np.concatenate([wg.reshape(I // 8, 8, -1), wu.reshape(I // 8, 8, -1)], axis=1)
+
+
+def down_tiles(wd: np.ndarray) -> np.ndarray:
+    wd = np.asarray(wd)
+    return wd.reshape(wd.shape[0] // 16, 16, -1)
 
 
 def build_blob(hidden, inter, gq, uq, dq, gs, us, ds) -> np.ndarray:
@@ -143,12 +184,11 @@ def build_blob(hidden, inter, gq, uq, dq, gs, us, ds) -> np.ndarray:
         raw = np.ascontiguousarray(arr).view(np.uint8).reshape(-1)
         blob[lay[name]:lay[name] + raw.size] = raw
 
-    put("gq", pack_int4(np.asarray(gq).reshape(I, H)))
-    put("uq", pack_int4(np.asarray(uq).reshape(I, H)))
-    put("dq", pack_int4(np.asarray(dq).reshape(H, I)))
-    put("gs", np.asarray(gs, np.float16).reshape(I, H // QBLOCK))
-    put("us", np.asarray(us, np.float16).reshape(I, H // QBLOCK))
-    put("ds", np.asarray(ds, np.float16).reshape(H, I // QBLOCK))
+    put("guq", pack_tiles(gate_up_tiles(np.asarray(gq).reshape(I, H), np.asarray(uq).reshape(I, H))))
+    put("dq", pack_tiles(down_tiles(np.asarray(dq).reshape(H, I))))
+    put("gus", pack_tile_scales(gate_up_tiles(np.asarray(gs, np.float16).reshape(I, H // QBLOCK),
+                                              np.asarray(us, np.float16).reshape(I, H // QBLOCK))))
+    put("ds", pack_tile_scales(down_tiles(np.asarray(ds, np.float16).reshape(H, I // QBLOCK))))
     return blob
 
 
@@ -207,17 +247,17 @@ def make_expert_blob(cfg: LayerConfig, expert: int, seed: int = 0) -> np.ndarray
     """One expert blob; expert in [0, E) routed, [E, E+S) shared.
 
     int4 values are uniform in [-8, 7] (a uniform random byte is two independent
-    uniform nibbles); scales are fp16 (round to nearest even) of U[0.005, 0.02].
+    uniform nibbles, whatever the byte's place in the layout); scales are fp16
+    (round to nearest even) of U[0.005, 0.02].
     """
     H, I = cfg.hidden, cfg.inter
     lay = blob_layout(H, I)
     r = _rng(seed, _STREAM_EXPERT, expert)
     blob = np.zeros(lay["total"], np.uint8)
-    nq = I * H // 2
-    for name in ("gq", "uq", "dq"):
-        blob[lay[name]:lay[name] + nq] = np.frombuffer(r.bytes(nq), np.uint8)
-    for name, rows, cols in (("gs", I, H // QBLOCK), ("us", I, H // QBLOCK), ("ds", H, I // QBLOCK)):
-        s = r.uniform(0.005, 0.02, size=rows * cols).astype(np.float32).astype(np.float16)
+    for name, nbytes in (("guq", I * H), ("dq", H * I // 2)):
+        blob[lay[name]:lay[name] + nbytes] = np.frombuffer(r.bytes(nbytes), np.uint8)
+    for name, count in (("gus", I * H // 16), ("ds", H * I // 32)):
+        s = r.uniform(0.005, 0.02, size=count).astype(np.float32).astype(np.float16)
         raw = s.view(np.uint8)
         blob[lay[name]:lay[name] + raw.size] = raw
     return blob

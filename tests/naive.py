@@ -15,29 +15,39 @@ import numpy as np
 from quantized_routed_expert_04_b200 import synth
 
 
-def unpack_int4(packed: np.ndarray, rows: int, K: int) -> np.ndarray:
-    b = np.asarray(packed, np.uint8).reshape(rows, K // 2)
+def unpack_tiles(raw: np.ndarray, tiles: int, K: int) -> np.ndarray:
+    """u8 bytes of a tiled section -> int [tiles][16][K].
+
+    Byte 16w + 4b + c of a row's 64-byte group holds elements 32b + 8w + 2c
+    (low nibble) and 32b + 8w + 2c + 1 (high nibble)."""
+    b = np.asarray(raw, np.uint8).reshape(tiles, K // 128, 16, 4, 4, 4)  # t, g, row, w, blk, c
+    out = np.empty((tiles, K // 128, 16, 4, 4, 8), np.int16)               # t, g, row, w, blk, m
     lo = (b & 0xF).astype(np.int16)
     hi = (b >> 4).astype(np.int16)
-    lo = np.where(lo >= 8, lo - 16, lo)
-    hi = np.where(hi >= 8, hi - 16, hi)
-    q = np.empty((rows, K), np.int16)
-    q[:, 0::2] = lo
-    q[:, 1::2] = hi
-    return q
+    out[..., 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[..., 1::2] = np.where(hi >= 8, hi - 16, hi)
+    # element index within the group = 32*blk + 8*w + m
+    return out.transpose(0, 2, 1, 4, 3, 5).reshape(tiles, 16, K)
+
+
+def tile_scales(raw: np.ndarray, tiles: int, K: int) -> np.ndarray:
+    """f16 bytes of a tiled scale section -> float64 [tiles][16][K/32]."""
+    s = np.asarray(raw, np.uint8).view(np.float16).reshape(tiles, K // 128, 16, 4)
+    return s.transpose(0, 2, 1, 3).reshape(tiles, 16, K // 32).astype(np.float64)
 
 
 def dense_expert(blob: np.ndarray, H: int, I: int):
     """(Wg [I][H], Wu [I][H], Wd [H][I]) dequantised to float64."""
     lay = synth.blob_layout(H, I)
-
-    def mat(qn, sn, rows, K):
-        q = unpack_int4(blob[lay[qn]:lay[qn] + rows * K // 2], rows, K)
-        s = blob[lay[sn]:lay[sn] + rows * (K // 32) * 2].view(np.float16)
-        s = s.reshape(rows, K // 32).astype(np.float64)
-        return q.astype(np.float64) * np.repeat(s, 32, axis=1)
-
-    return mat("gq", "gs", I, H), mat("uq", "us", I, H), mat("dq", "ds", H, I)
+    gu = unpack_tiles(blob[lay["guq"]:lay["guq"] + I * H], I // 8, H)
+    gus = tile_scales(blob[lay["gus"]:lay["gus"] + I * H // 8], I // 8, H)
+    d = unpack_tiles(blob[lay["dq"]:lay["dq"] + H * I // 2], H // 16, I)
+    ds = tile_scales(blob[lay["ds"]:lay["ds"] + H * I // 16], H // 16, I)
+    w_gu = gu * np.repeat(gus, 32, axis=2)
+    Wg = w_gu[:, :8, :].reshape(I, H)
+    Wu = w_gu[:, 8:, :].reshape(I, H)
+    Wd = (d * np.repeat(ds, 32, axis=2)).reshape(H, I)
+    return Wg, Wu, Wd
 
 
 def ffn64(dense, x: np.ndarray) -> np.ndarray:

@@ -55,7 +55,7 @@ def test_route_prefill_all_tokens():
 
 
 def test_route_ties_lowest_index():
-    cfg = synth.custom_config("ties", 128, 64, 8, 3, tokens=(2,))
+    cfg = synth.custom_config("ties", 128, 128, 8, 3, tokens=(2,))
     lay = GpuLayer(cfg)
     W = lay.W.copy()
     W[6] = W[2] = W[5] = 0.5
@@ -102,7 +102,7 @@ def test_forward_mixtral_16_tokens():
 def test_forward_ragged_token_groups(T):
     """Experts with more than 16 pairs (several token groups), ragged tails,
     shared experts, hidden/inter not multiples of 1024."""
-    cfg = synth.custom_config("ragged", 320, 192, 6, 2, n_shared=1, tokens=(T,), bias="normal",
+    cfg = synth.custom_config("ragged", 384, 256, 6, 2, n_shared=1, tokens=(T,), bias="normal",
                               bias_var=0.5)
     lay = GpuLayer(cfg)
     x = synth.make_x(cfg, T, step=5)

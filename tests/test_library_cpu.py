@@ -37,14 +37,14 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_expert_bytes_matches_format(lib):
-    for H, I in [(256, 512), (2048, 1408), (4096, 14336), (4096, 1024), (4096, 2048), (320, 192)]:
+    for H, I in [(256, 512), (2048, 1408), (4096, 14336), (4096, 1024), (4096, 2048), (384, 256)]:
         assert binding.strata_moe_expert_bytes(H, I) == synth.expert_bytes(H, I)
     assert binding.strata_moe_expert_bytes(100, 64) == 0
 
 
 @pytest.mark.parametrize("args", [
     (0, 512, 8, 2, 0, 8),        # hidden 0
-    (256, 500, 8, 2, 0, 8),      # inter not a multiple of 64
+    (256, 448, 8, 2, 0, 8),      # inter not a multiple of 128
     (256, 512, 0, 1, 0, 1),      # no experts
     (256, 512, 300, 2, 0, 300),  # too many experts
     (256, 512, 8, 9, 0, 8),      # top_k > n_experts

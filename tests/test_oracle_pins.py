@@ -36,22 +36,46 @@ def bf16(a):
 
 # --------------------------------------------------------------------- format
 
+def binding_free_layout_ok(H, I):
+    lay = synth.blob_layout(H, I)
+    return all(lay[k] % 256 == 0 for k in lay)
+
+
 def test_pack_int4_hand_bytes():
     # element 2j -> low nibble, 2j+1 -> high nibble, two's complement
     q = np.array([[-8, 7, 1, -1, 0, -2]])
     assert synth.pack_int4(q).tolist() == [[0x78, 0xF1, 0xE0]]
 
 
+def test_group_layout_hand_bytes():
+    """One gate row, one group: element 32b + 8w + m sits at byte 16w + 4b + m/2."""
+    H, I = 128, 128
+    q = np.zeros((I, H), int)
+    q[0, 0] = 1        # b0 w0 m0 -> byte 0 low
+    q[0, 9] = 2        # b0 w1 m1 -> byte 16 high
+    q[0, 32 + 7] = -1  # b1 w0 m7 -> byte 4 + 3 high
+    q[0, 96 + 24] = 3  # b3 w3 m0 -> byte 48 + 12 low
+    z = np.zeros((I, H // 32), np.float16)
+    blob = synth.build_blob(H, I, q, np.zeros_like(q), np.zeros((H, I), int), z, z,
+                            np.zeros((H, I // 32), np.float16))
+    row0 = blob[:64]
+    assert row0[0] == 0x01 and row0[16] == 0x20 and row0[7] == 0xF0 and row0[60] == 0x03
+    assert np.count_nonzero(row0) == 4
+    # up row 0 is tile row 8 of tile 0: bytes 8*64 .. 9*64
+    assert not blob[8 * 64:9 * 64].any()
+
+
 def test_blob_size_formula():
     # B_e = 3*H*I*(1/2 + 2/32) when every section is a multiple of 256 bytes
     for H, I in [(256, 512), (2048, 1408), (4096, 14336), (4096, 1024), (4096, 2048)]:
         assert oracle.expert_bytes(H, I) == synth.expert_bytes(H, I) == int(3 * H * I * 0.5625)
+        assert binding_free_layout_ok(H, I)
 
 
 def test_dequant_matches_drawn_values_one_hot():
     """x = identity makes g[t] the t-th column of Wg: oracle g must equal
     float(scale) * q for the drawn ints, exactly (one nonzero product)."""
-    H, I = 64, 96
+    H, I = 128, 256
     blob, p = rand_blob(H, I)
     # edge fp16 scales: min subnormal, a subnormal, min normal, max
     p["gs"][0, 0] = np.float16(2.0 ** -24)
@@ -69,7 +93,7 @@ def test_dequant_matches_drawn_values_one_hot():
 
 def test_down_projection_columns():
     """y = Wd h with Wd dequantised from the drawn ints (fp64 reference)."""
-    H, I = 64, 64
+    H, I = 128, 128
     blob, p = rand_blob(H, I)
     x = np.eye(H, dtype=np.float32)
     g, u, h, y = oracle.expert_ffn(blob, H, I, x)
@@ -80,7 +104,7 @@ def test_down_projection_columns():
 
 def test_swiglu_formula():
     """h = silu(g) * u with silu(z) = z / (1 + e^-z) (spec: SwiGLU)."""
-    H, I = 64, 64
+    H, I = 128, 128
     blob, _ = rand_blob(H, I)
     x = synth.bf16_bits_to_f32(bf16(RNG.standard_normal((5, H)) * 4))
     g, u, h, _ = oracle.expert_ffn(blob, H, I, x)
@@ -91,7 +115,7 @@ def test_swiglu_formula():
 
 def test_gate_all_equal_weights_closed_form():
     """All q = 1 with scale s: g_i = s * sum(x) for every row."""
-    H, I = 128, 32
+    H, I = 128, 128
     s = np.float16(0.0125)
     parts = dict(gq=np.ones((I, H), int), uq=np.ones((I, H), int), dq=np.ones((H, I), int),
                  gs=np.full((I, H // 32), s), us=np.full((I, H // 32), s),
@@ -108,10 +132,10 @@ def test_gate_all_equal_weights_closed_form():
 
 def test_negative_extreme_nibble():
     """q = -8 everywhere (nibble 0x8) must read as -8, not +8."""
-    H, I = 32, 32
+    H, I = 128, 128
     s = np.float16(1.0)
     parts = dict(gq=np.full((I, H), -8), uq=np.full((I, H), 7), dq=np.zeros((H, I), int),
-                 gs=np.full((I, 1), s), us=np.full((I, 1), s), ds=np.full((H, 1), s))
+                 gs=np.full((I, 4), s), us=np.full((I, 4), s), ds=np.full((H, 4), s))
     blob = synth.build_blob(H, I, **parts)
     x = np.ones((1, H), np.float32)
     g, u, _, _ = oracle.expert_ffn(blob, H, I, x)
@@ -184,8 +208,8 @@ def _bind_all(blobs, perm=None):
     return perm.astype(np.int32), [blobs[e] for e in perm]
 
 
-@pytest.mark.parametrize("E,k,S,T,H,I", [(4, 1, 0, 2, 64, 64), (6, 2, 1, 3, 64, 32),
-                                          (8, 3, 2, 2, 32, 64), (5, 2, 0, 1, 96, 64)])
+@pytest.mark.parametrize("E,k,S,T,H,I", [(4, 1, 0, 2, 128, 128), (6, 2, 1, 3, 128, 256),
+                                          (8, 3, 2, 2, 256, 128), (5, 2, 0, 1, 128, 128)])
 def test_layer_matches_naive_bruteforce(E, k, S, T, H, I):
     rng = np.random.default_rng(E * 100 + k * 10 + S)
     blobs = [rand_blob(H, I, rng)[0] for _ in range(E)]
@@ -205,7 +229,7 @@ def test_layer_matches_naive_bruteforce(E, k, S, T, H, I):
 
 def test_topk_all_experts_is_dense_softmax_mixture():
     """top_k = n_experts: out = sum_e softmax(l)_e FFN_e(x) (torch fp64)."""
-    E, H, I, T = 5, 64, 64, 3
+    E, H, I, T = 5, 128, 128, 3
     rng = np.random.default_rng(7)
     blobs = [rand_blob(H, I, rng)[0] for _ in range(E)]
     W = (rng.standard_normal((E, H)) / np.sqrt(H)).astype(np.float32)
@@ -227,7 +251,7 @@ def test_topk_all_experts_is_dense_softmax_mixture():
 
 def test_single_expert_weight_one_is_swiglu_ffn():
     """E = 1, k = 1: w = 1 and out = Wd (silu(Wg x) * (Wu x)) (torch fp64)."""
-    H, I, T = 96, 64, 4
+    H, I, T = 256, 128, 4
     rng = np.random.default_rng(11)
     blob = rand_blob(H, I, rng)[0]
     W = rng.standard_normal((1, H)).astype(np.float32)
@@ -244,16 +268,16 @@ def test_paged_vs_resident_bitwise():
     """strata.amperor.ai "/methods/", Fidelity: paged output is bit-identical to
     resident.  Any slot permutation, and binding only the routed experts, give
     the same fp32 bits."""
-    cfg = synth.custom_config("t", 64, 64, 8, 2, n_shared=1, n_slots=8, tokens=(3,))
+    cfg = synth.custom_config("t", 128, 128, 8, 2, n_shared=1, n_slots=8, tokens=(3,))
     blobs = [synth.make_expert_blob(cfg, e) for e in range(8)]
     shared = [synth.make_expert_blob(cfg, 8)]
     W, b = synth.make_router(cfg)
     x = synth.make_x(cfg, 3)
-    st, ref, _, idx, w = oracle.forward(x, 64, 64, W, b, 2, *_bind_all(blobs), shared)
+    st, ref, _, idx, w = oracle.forward(x, 128, 128, W, b, 2, *_bind_all(blobs), shared)
     assert st == oracle.OK
     for p in range(4):
         perm = synth.make_slot_permutation(cfg, index=p)
-        st, out, *_ = oracle.forward(x, 64, 64, W, b, 2, *_bind_all(blobs, perm), shared)
+        st, out, *_ = oracle.forward(x, 128, 128, W, b, 2, *_bind_all(blobs, perm), shared)
         assert st == oracle.OK and out.view(np.uint32).tolist() == ref.view(np.uint32).tolist()
     routed = sorted(set(idx.reshape(-1).tolist()))
     se = np.full(8, -1, np.int32)
@@ -261,21 +285,21 @@ def test_paged_vs_resident_bitwise():
     for s, e in zip(np.random.default_rng(3).permutation(8)[:len(routed)], routed):
         se[s] = e
         sb[s] = blobs[e]
-    st, out = oracle.forward_routed(x, 64, 64, 8, 2, se, sb, shared, idx, w)
+    st, out = oracle.forward_routed(x, 128, 128, 8, 2, se, sb, shared, idx, w)
     assert st == oracle.OK and out.view(np.uint32).tolist() == ref.view(np.uint32).tolist()
 
 
 def test_unbound_expert_reports_and_zeroes_token():
-    cfg = synth.custom_config("t", 64, 32, 6, 2, tokens=(4,))
+    cfg = synth.custom_config("t", 128, 128, 6, 2, tokens=(4,))
     blobs = [synth.make_expert_blob(cfg, e) for e in range(6)]
     W, b = synth.make_router(cfg)
     x = synth.make_x(cfg, 4)
-    st, ref, _, idx, w = oracle.forward(x, 64, 32, W, b, 2, *_bind_all(blobs), [])
+    st, ref, _, idx, w = oracle.forward(x, 128, 128, W, b, 2, *_bind_all(blobs), [])
     victim = int(idx[1, 0])
     se = np.arange(6, dtype=np.int32)
     se[victim] = -1
     sb = [None if e == victim else blobs[e] for e in range(6)]
-    st, out = oracle.forward_routed(x, 64, 32, 6, 2, se, sb, [], idx, w)
+    st, out = oracle.forward_routed(x, 128, 128, 6, 2, se, sb, [], idx, w)
     assert st == oracle.NOT_BOUND
     for t in range(4):
         if victim in idx[t]:
@@ -285,18 +309,18 @@ def test_unbound_expert_reports_and_zeroes_token():
 
 
 def test_slot_conflict():
-    cfg = synth.custom_config("t", 32, 32, 4, 1, tokens=(1,))
+    cfg = synth.custom_config("t", 128, 128, 4, 1, tokens=(1,))
     blobs = [synth.make_expert_blob(cfg, e) for e in range(4)]
     x = synth.make_x(cfg, 1)
     se = np.array([0, 1, 1, 3], np.int32)
-    st, _ = oracle.forward_routed(x, 32, 32, 4, 1, se, blobs, [], np.array([[0]]), np.array([[1.0]]))
+    st, _ = oracle.forward_routed(x, 128, 128, 4, 1, se, blobs, [], np.array([[0]]), np.array([[1.0]]))
     assert st == oracle.SLOT_CONFLICT
 
 
 def test_combine_order_is_weighted_then_shared():
     """out = sum_j w_j y_j + sum_s y_s: with a zero routed weight the output is
     exactly the shared expert's y, and with w = (1, 0) it is y_0 + y_shared."""
-    H, I = 32, 32
+    H, I = 128, 128
     rng = np.random.default_rng(5)
     blobs = [rand_blob(H, I, rng)[0] for _ in range(3)]
     sh = rand_blob(H, I, rng)[0]
