@@ -72,6 +72,27 @@ template <bool kGateUp, int NT>   // NT: 8-pair MMA tiles per item (1 or 2)
 __global__ void expert_mma_kernel(MmParams p);
 
 size_t mm_smem_bytes(const MmParams &p);
+
+// ---- expert matmuls for many tokens per expert (prefill_tc.cu)
+struct TcParams {
+  ExpertTable table;
+  Routing rt;
+  int K;              // H (gate/up) or I (down)
+  int row_tiles;      // 128-row weight tiles: I/64 (gate/up) or H/128 (down)
+  size_t q_off, s_off;
+  int out_ld;         // I (h16) or H (y)
+  __half *h_out;
+  float *y_out;
+  int *status;
+};
+}  // namespace strata
+#include <cuda.h>
+namespace strata {
+template <bool kGateUp>
+__global__ void expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b);
+__global__ void gather_rows_kernel(const __half *x16, const int *pair_tok, const int *n_pairs_dev,
+                                   int H, int P_cap, __half *xp);
+size_t tc_smem_bytes();
 size_t mm_fixed_smem_bytes();
 
 }  // namespace strata

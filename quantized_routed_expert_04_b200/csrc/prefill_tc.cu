@@ -1,0 +1,414 @@
+// Expert matmuls for many tokens per expert (prefill): a grouped GEMM on the
+// 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory).
+//
+// What it computes (the W4A16 expert FFN of ro99/strata README, model table
+// and "Kernels"; the prompt-time expert GEMMs of "Strata on a Mac",
+// "Switches"): for every active expert e and the pairs routed to it,
+//   gate/up pass:  h = silu(Wg x) * (Wu x)  -> h16 [P][I] (f16)
+//   down pass:     y = Wd h                -> y   [P][H] (fp32)
+//
+// Tile = (expert, chunk of <= 128 of its pairs, 128 weight rows).  For
+// gate/up the 128 rows are 8 blob tiles, i.e. 64 gate rows and the same 64 up
+// rows interleaved by 8 (TMEM lane l holds gate if l % 16 < 8, else up; its
+// partner is lane l ^ 8, in the same warp).  For down they are 128
+// consecutive rows of Wd.
+//
+// Warp roles (one CTA per SM, persistent; tiles interleaved over CTAs):
+//   warp 0      producer: per K group (128 elements) a TMA load of the
+//               activation rows (f16, 128-byte swizzle; x_perm or h16), and
+//               every 4 K groups one bulk copy per blob tile of packed
+//               weights and of scales;
+//   warp 1      MMA: allocates 256 TMEM columns (two 128-column accumulator
+//               buffers), and one thread issues 8 tcgen05.mma (M=128, N=pairs
+//               rounded up to 16, K=16) per K group, then commits to the
+//               stage barriers and, at the end of a tile, to the accumulator;
+//   warps 2-5   dequant: int4 -> exact f16 integers -> times the fp16 scale
+//               (one f16 rounding) -> the K-major 128-byte-swizzled A layout;
+//   warps 6-9   epilogue: tcgen05.ld 32 columns at a time, SwiGLU (gate/up)
+//               or plain (down), transposed through shared memory, stored.
+// Every wait is bounded; on a timeout the status word is set and the roles
+// wind down (the allocating warp still frees the tensor memory).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace strata {
+
+namespace {
+
+constexpr int kTcM = 128;          // weight rows per tile
+constexpr int kTcN = 128;          // pairs per tile (max MMA N used)
+constexpr int kPkStages = 2;       // packed-weight stages (4 K groups each)
+constexpr int kPkGroups = 4;
+constexpr int kAStages = 2;        // dequantised A stages (one K group)
+constexpr int kBStages = 2;        // activation stages (one K group)
+constexpr int kAccCols = 128;      // TMEM columns per accumulator buffer
+constexpr uint32_t kTmemCols = 256;
+
+constexpr int kAStageBytes = 2 * kTcM * 128;           // two 64-wide atoms
+constexpr int kBStageBytes = 2 * kTcN * 128;
+constexpr int kPkQBytes = 8 * kPkGroups * 1024;        // 8 blob tiles
+constexpr int kPkSBytes = 8 * kPkGroups * 128;
+constexpr int kPkStageBytes = kPkQBytes + kPkSBytes;
+constexpr int kEpiBytes = 4 * 4096;                    // per epilogue warp: 32 x 32 fp32
+
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kAStages * kAStageBytes;
+constexpr int kOffPk = kOffB + kBStages * kBStageBytes;
+constexpr int kOffEpi = kOffPk + kPkStages * kPkStageBytes;
+constexpr int kOffBar = kOffEpi + kEpiBytes;
+constexpr int kNumBars = 2 * kPkStages + 2 * kAStages + 2 * kBStages + 4;
+constexpr int kOffTab = kOffBar + kNumBars * 8 + 16;   // + TMEM address slot
+constexpr int kTabBytes = kMaxIds * 8 + (3 * kMaxIds + 1) * 4;
+constexpr int kTcSmem = kOffTab + kTabBytes + 1024;    // + alignment slack
+
+__device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *status) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+struct Unit {
+  const uint8_t *blob;
+  int pi0, n, rt;
+};
+
+}  // namespace
+
+size_t tc_smem_bytes() { return kTcSmem; }
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(320, 1)
+    expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint64_t *pk_full = bars, *pk_empty = pk_full + kPkStages;
+  uint64_t *a_full = pk_empty + kPkStages, *a_empty = a_full + kAStages;
+  uint64_t *b_full = a_empty + kAStages, *b_empty = b_full + kBStages;
+  uint64_t *acc_full = b_empty + kBStages, *acc_empty = acc_full + 2;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
+  const uint8_t **t_blob = reinterpret_cast<const uint8_t **>(smem + kOffTab);
+  int *t_off = reinterpret_cast<int *>(t_blob + kMaxIds);
+  int *t_cnt = t_off + kMaxIds;
+  int *unit_base = t_cnt + kMaxIds;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPkStages; ++s) {
+      mbar_init(&pk_full[s], 1);
+      mbar_init(&pk_empty[s], 4);
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&a_full[s], 4);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  grid_dependency_wait();
+
+  // active experts and tiles per expert (prefix), in shared memory
+  const int n_active = *p.rt.n_active;
+  for (int a = threadIdx.x; a < n_active; a += blockDim.x) {
+    const int id = p.rt.active[a];
+    t_blob[a] = p.table.ptr[id];
+    t_off[a] = p.rt.off[id];
+    t_cnt[a] = p.rt.cnt[id];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  if (warp == 0) {
+    int carry = 0;
+    for (int a0 = 0; a0 < n_active; a0 += 32) {
+      const int a = a0 + lane;
+      const int v = a < n_active ? ((t_cnt[a] + kTcN - 1) / kTcN) * p.row_tiles : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += nb;
+      }
+      if (a < n_active) unit_base[a] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) unit_base[n_active] = carry;
+  }
+  __syncthreads();
+  grid_dependency_launch();
+
+  const int n_units = unit_base[n_active];
+  const int G = p.K / 128;  // K groups
+  auto decode = [&](int u, int &a) -> Unit {
+    while (unit_base[a + 1] <= u) ++a;
+    const int rem = u - unit_base[a];
+    const int tcn = rem / p.row_tiles;
+    Unit un;
+    un.rt = rem - tcn * p.row_tiles;
+    un.pi0 = t_off[a] + tcn * kTcN;
+    un.n = min(kTcN, t_cnt[a] - tcn * kTcN);
+    un.blob = t_blob[a];
+    return un;
+  };
+  // unbound experts: skipped by every role, flagged once
+  auto next_unit = [&](int u, int &a) -> int {
+    for (; u < n_units; u += gridDim.x) {
+      while (unit_base[a + 1] <= u) ++a;
+      if (t_blob[a]) return u;
+      if (threadIdx.x == 0) set_status(p.status, STATUS_NOT_BOUND);
+    }
+    return n_units;
+  };
+
+  if (warp == 0) {
+    // -------------------------------------------------------- producer
+    uint32_t pk_cnt = 0, b_cnt = 0;
+    bool ok = true;
+    int a = 0;
+    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+      const Unit un = decode(u, a);
+      const int nb = (un.n + 31) / 32;        // 32-row boxes of activations
+      for (int g = 0; g < G && ok; ++g) {
+        if (g % kPkGroups == 0) {
+          const int s = (int)(pk_cnt % kPkStages);
+          if (!wwait(&pk_empty[s], ((pk_cnt / kPkStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
+          ++pk_cnt;
+          const int ng = min(kPkGroups, G - g);
+          uint8_t *dst = smem + kOffPk + s * kPkStageBytes;
+          if (lane == 0) mbar_arrive_expect_tx(&pk_full[s], 8u * ng * (1024u + 128u));
+          __syncwarp();
+          if (lane < 8) {
+            const int tile = un.rt * 8 + lane;
+            const size_t g0 = (size_t)tile * G + g;
+            bulk_g2s(dst + lane * (kPkGroups * 1024), un.blob + p.q_off + g0 * 1024, ng * 1024u,
+                     &pk_full[s]);
+            bulk_g2s(dst + kPkQBytes + lane * (kPkGroups * 128), un.blob + p.s_off + g0 * 128,
+                     ng * 128u, &pk_full[s]);
+          }
+        }
+        const int s = (int)(b_cnt % kBStages);
+        if (!wwait(&b_empty[s], ((b_cnt / kBStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
+        ++b_cnt;
+        uint8_t *dst = smem + kOffB + s * kBStageBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&b_full[s], 2u * nb * 4096u);
+          for (int atom = 0; atom < 2; ++atom)
+            for (int rb = 0; rb < nb; ++rb)
+              tma_load_2d(dst + atom * (kTcN * 128) + rb * 4096, &tmap_b, g * 128 + atom * 64,
+                          un.pi0 + rb * 32, &b_full[s]);
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok) {
+      // let issued copies land before the CTA exits
+      for (uint32_t m = pk_cnt > kPkStages ? pk_cnt - kPkStages : 0; m < pk_cnt; ++m)
+        (void)wwait(&pk_full[m % kPkStages], (m / kPkStages) & 1u, p.status);
+      for (uint32_t m = b_cnt > kBStages ? b_cnt - kBStages : 0; m < b_cnt; ++m)
+        (void)wwait(&b_full[m % kBStages], (m / kBStages) & 1u, p.status);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issue
+    uint32_t a_cnt = 0, b_cnt = 0, t_cnt_local = 0;
+    bool ok = true;
+    int a = 0;
+    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+      const Unit un = decode(u, a);
+      const int N = (un.n + 15) & ~15;
+      const uint32_t idesc = umma_idesc_f16(kTcM, N);
+      const int buf = (int)(t_cnt_local & 1u);
+      if (!wwait(&acc_empty[buf], ((t_cnt_local >> 1) & 1u) ^ 1u, p.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + buf * kAccCols;
+      for (int g = 0; g < G; ++g) {
+        const int sa = (int)(a_cnt % kAStages), sb = (int)(b_cnt % kBStages);
+        if (!wwait(&a_full[sa], (a_cnt / kAStages) & 1u, p.status)) { ok = false; break; }
+        if (!wwait(&b_full[sb], (b_cnt / kBStages) & 1u, p.status)) { ok = false; break; }
+        ++a_cnt;
+        ++b_cnt;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(smem + kOffA + sa * kAStageBytes);
+          const uint32_t b_addr = smem_u32(smem + kOffB + sb * kBStageBytes);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t off = (j >> 2) * (kTcM * 128) + (j & 3) * 32;
+            const uint32_t boff = (j >> 2) * (kTcN * 128) + (j & 3) * 32;
+            umma_f16(d_tmem, umma_desc_sw128(a_addr + off), umma_desc_sw128(b_addr + boff), idesc,
+                     (g > 0 || j > 0) ? 1u : 0u);
+          }
+          umma_commit(&a_empty[sa]);
+          umma_commit(&b_empty[sb]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&acc_full[buf]);
+      __syncwarp();
+      ++t_cnt_local;
+    }
+  } else if (warp < 6) {
+    // -------------------------------------------------------- dequant
+    const int dw = warp - 2;
+    const int w = lane & 3;
+    const int q = lane >> 2;
+    const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
+    uint32_t pk_cnt = 0, a_cnt = 0;
+    bool ok = true;
+    int a = 0;
+    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+      for (int g = 0; g < G && ok; ++g) {
+        const int ps = (int)(pk_cnt % kPkStages);
+        if (g % kPkGroups == 0)
+          if (!wwait(&pk_full[ps], (pk_cnt / kPkStages) & 1u, p.status)) { ok = false; break; }
+        const int sa = (int)(a_cnt % kAStages);
+        if (!wwait(&a_empty[sa], ((a_cnt / kAStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
+        ++a_cnt;
+        const uint8_t *pq = smem + kOffPk + ps * kPkStageBytes;
+        const uint8_t *psc = pq + kPkQBytes;
+        uint8_t *ad = smem + kOffA + sa * kAStageBytes;
+        const int gi = g % kPkGroups;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int r = 32 * dw + 8 * m + row_in_8;
+          const int j = r >> 4, tr = r & 15;
+          const uint4 qv = *reinterpret_cast<const uint4 *>(pq + j * (kPkGroups * 1024) + gi * 1024 +
+                                                            tr * 64 + w * 16);
+          const uint2 sv = *reinterpret_cast<const uint2 *>(psc + j * (kPkGroups * 128) + gi * 128 +
+                                                            tr * 8);
+          const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
+          const __half2 sc[4] = {__half2half2(__low2half(bits_h2(sv.x))),
+                                 __half2half2(__high2half(bits_h2(sv.x))),
+                                 __half2half2(__low2half(bits_h2(sv.y))),
+                                 __half2half2(__high2half(bits_h2(sv.y)))};
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            uint32_t f[4];
+            int4x8_to_f16(words[b], f);
+            uint4 o;
+            o.x = h2_bits(__hmul2(bits_h2(f[0]), sc[b]));
+            o.y = h2_bits(__hmul2(bits_h2(f[1]), sc[b]));
+            o.z = h2_bits(__hmul2(bits_h2(f[2]), sc[b]));
+            o.w = h2_bits(__hmul2(bits_h2(f[3]), sc[b]));
+            const int chunk = ((b & 1) * 4 + w) ^ (r & 7);
+            *reinterpret_cast<uint4 *>(ad + (b >> 1) * (kTcM * 128) + r * 128 + chunk * 16) = o;
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[sa]);
+        if (gi == kPkGroups - 1 || g == G - 1) {
+          if (lane == 0) mbar_arrive(&pk_empty[ps]);
+          ++pk_cnt;
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------------- epilogue
+    const int qd = warp & 3;  // TMEM lane quarter of this warp
+    float *stage = reinterpret_cast<float *>(smem + kOffEpi + (warp - 6) * 4096);
+    uint32_t t_cnt_local = 0;
+    bool ok = true;
+    int a = 0;
+    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+      const Unit un = decode(u, a);
+      const int buf = (int)(t_cnt_local & 1u);
+      if (!wwait(&acc_full[buf], (t_cnt_local >> 1) & 1u, p.status)) { ok = false; break; }
+      tc_fence_after();
+      for (int col0 = 0; col0 < un.n; col0 += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * qd) << 16) + buf * kAccCols + col0, v);
+        if (kGateUp) {
+          // lane L: blob tile 2 qd + L / 16, tile row L % 16 (gate if < 8)
+          __half *hs = reinterpret_cast<__half *>(stage);  // [32 pairs][16]
+          const bool gate = (lane & 15) < 8;
+          const int pos16 = 8 * (lane >> 4) + (((lane & 3) << 1) | ((lane >> 2) & 1));
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float up = __shfl_xor_sync(0xffffffffu, v[t], 8);
+            if (gate) {
+              const float gv = v[t];
+              hs[t * 16 + pos16] = __float2half_rn(gv / (1.0f + expf(-gv)) * up);
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int piece = lane + 32 * k;  // 64 pieces of 16 bytes
+            const int t = piece >> 1, half = piece & 1;
+            if (col0 + t < un.n) {
+              const uint4 val = *reinterpret_cast<const uint4 *>(hs + t * 16 + half * 8);
+              __half *dst = p.h_out + (size_t)(un.pi0 + col0 + t) * p.out_ld +
+                            64 * un.rt + 16 * qd + 8 * half;
+              *reinterpret_cast<uint4 *>(dst) = val;
+            }
+          }
+          __syncwarp();
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) stage[t * 32 + lane] = v[t];
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int piece = lane + 32 * k;  // 256 pieces of 16 bytes
+            const int t = piece >> 3, seg = piece & 7;
+            if (col0 + t < un.n) {
+              const float4 val = *reinterpret_cast<const float4 *>(stage + t * 32 + seg * 4);
+              float *dst = p.y_out + (size_t)(un.pi0 + col0 + t) * p.out_ld + 128 * un.rt +
+                           32 * qd + 4 * seg;
+              *reinterpret_cast<float4 *>(dst) = val;
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      ++t_cnt_local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template __global__ void expert_tc_kernel<true>(TcParams, const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<false>(TcParams, const __grid_constant__ CUtensorMap);
+
+// x_perm[pair] = x16[token of pair], 16 bytes per thread.
+__global__ void gather_rows_kernel(const __half *__restrict__ x16, const int *__restrict__ pair_tok,
+                                   const int *__restrict__ n_pairs_dev, int H, int P_cap,
+                                   __half *__restrict__ xp) {
+  grid_dependency_wait();
+  const int n_pairs = min(*n_pairs_dev, P_cap);
+  const int per_row = H / 8;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)n_pairs * per_row;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int pr = (int)(i / per_row), c = (int)(i - (long long)pr * per_row);
+    const uint4 v = *reinterpret_cast<const uint4 *>(x16 + (size_t)pair_tok[pr] * H + c * 8);
+    *reinterpret_cast<uint4 *>(xp + (size_t)pr * H + c * 8) = v;
+  }
+}
+
+}  // namespace strata

@@ -2,6 +2,8 @@
 // checks, the expert-id -> slot table, the device workspace, the kernel
 // sequence of a forward call, the device status word and optional per-kernel
 // timing.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -52,6 +54,7 @@ struct strata_moe {
   __half *x16 = nullptr;
   __half *h16 = nullptr;
   float *y = nullptr;
+  __half *xp = nullptr;     // activations gathered in sorted pair order (large batches)
   int *status = nullptr;    // device status word (own allocation)
   int *counter = nullptr;   // last-block counter of the small-batch routing kernel
   int last_bits = 0;
@@ -137,6 +140,7 @@ strata_status grow_workspace(strata_moe *h, int T) {
   const size_t o_x16 = take(sizeof(__half) * cap * h->H);
   const size_t o_h16 = take(sizeof(__half) * P * h->I);
   const size_t o_y = take(sizeof(float) * P * h->H);
+  const size_t o_xp = cap > kSmallT ? take(sizeof(__half) * P * h->H) : 0;
   void *mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, off);
   if (e != cudaSuccess) {
@@ -162,6 +166,7 @@ strata_status grow_workspace(strata_moe *h, int T) {
   h->x16 = reinterpret_cast<__half *>(b + o_x16);
   h->h16 = reinterpret_cast<__half *>(b + o_h16);
   h->y = reinterpret_cast<float *>(b + o_y);
+  h->xp = cap > kSmallT ? reinterpret_cast<__half *>(b + o_xp) : nullptr;
   return STRATA_OK;
 }
 
@@ -216,6 +221,70 @@ MmParams mm_params(const strata_moe *h, bool gate_up, const ExpertTable &table, 
   return p;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Rows of f16 activations [rows][K] as the B operand of the tensor-core
+// kernel: boxes of 64 K x 32 rows, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap *m, const __half *base, int K, int rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Gather + the two tensor-core passes (large batches).
+strata_status run_tc_experts(strata_moe *h, int T, const ExpertTable &table, cudaStream_t stream) {
+  const int P = T * (h->k + h->S);
+  cudaError_t e;
+  const int per_row = h->H / 8;
+  const long long work = (long long)P * per_row;
+  const int gblocks = (int)std::min<long long>((work + 255) / 256, 8LL * h->num_sms);
+  e = launch(h, PH_GATHER, gather_rows_kernel, dim3(gblocks), dim3(256), 0, stream, true, h->x16,
+             h->rt.pair_tok, h->rt.off + (h->E + h->S), h->H, P, h->xp);
+  if (e != cudaSuccess) return cuda_status(e);
+  const size_t smem = tc_smem_bytes();
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool gu = pass == 0;
+    TcParams p;
+    std::memset(&p, 0, sizeof p);
+    p.table = table;
+    p.rt = h->rt;
+    p.K = gu ? h->H : h->I;
+    p.row_tiles = gu ? h->I / 64 : h->H / 128;
+    p.q_off = gu ? h->layout.guq : h->layout.dq;
+    p.s_off = gu ? h->layout.gus : h->layout.ds;
+    p.out_ld = gu ? h->I : h->H;
+    p.h_out = h->h16;
+    p.y_out = h->y;
+    p.status = h->status;
+    CUtensorMap m;
+    if (!encode_rows_map(&m, gu ? h->xp : h->h16, p.K, P)) return STRATA_ERR_CUDA;
+    auto kern = gu ? expert_tc_kernel<true> : expert_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(320), smem, stream, true,
+                 p, m);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return STRATA_OK;
+}
+
 strata_status check_common(strata_moe *h, const void *x, int T, cudaStream_t) {
   if (!h || T < 0) return STRATA_ERR_INVALID_ARG;
   if (T > 0 && (!x || (reinterpret_cast<uintptr_t>(x) & 15))) return STRATA_ERR_INVALID_ARG;
@@ -247,7 +316,11 @@ strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *id
                  h->k, h->E, h->S, h->rt);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  for (int pass = 0; pass < 2; ++pass) {
+  if (T > kSmallT) {
+    const strata_status st = run_tc_experts(h, T, table, stream);
+    if (st != STRATA_OK) return st;
+  }
+  for (int pass = 0; pass < 2 && T <= kSmallT; ++pass) {
     const bool gu = pass == 0;
     MmParams p = mm_params(h, gu, table, T);
     const size_t smem = mm_smem_bytes(p);
