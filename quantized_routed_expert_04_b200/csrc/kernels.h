@@ -93,6 +93,7 @@ __global__ void expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap
 __global__ void gather_rows_kernel(const __half *x16, const int *pair_tok, const int *n_pairs_dev,
                                    int H, int P_cap, __half *xp);
 size_t tc_smem_bytes();
+int tc_threads();
 size_t mm_fixed_smem_bytes();
 
 }  // namespace strata

@@ -14,18 +14,20 @@
 // consecutive rows of Wd.
 //
 // Warp roles (one CTA per SM, persistent; tiles interleaved over CTAs):
-//   warp 0      producer: per K group (128 elements) a TMA load of the
-//               activation rows (f16, 128-byte swizzle; x_perm or h16), and
-//               every 4 K groups one bulk copy per blob tile of packed
-//               weights and of scales;
+//   warp 0      producer: per 64 K elements a TMA load of the activation
+//               rows (f16, 128-byte swizzle; x_perm or h16), and every 2 K
+//               groups (of 128) one bulk copy per blob tile of packed weights
+//               and of scales;
 //   warp 1      MMA: allocates 256 TMEM columns (two 128-column accumulator
 //               buffers), and one thread issues 8 tcgen05.mma (M=128, N=pairs
 //               rounded up to 16, K=16) per K group, then commits to the
 //               stage barriers and, at the end of a tile, to the accumulator;
-//   warps 2-5   dequant: int4 -> exact f16 integers -> times the fp16 scale
+//   warps 2-9   dequant: int4 -> exact f16 integers -> times the fp16 scale
 //               (one f16 rounding) -> the K-major 128-byte-swizzled A layout;
-//   warps 6-9   epilogue: tcgen05.ld 32 columns at a time, SwiGLU (gate/up)
-//               or plain (down), transposed through shared memory, stored.
+//   warps 10-13 epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
+//               transposed through shared memory, stored.
+// Activations are staged one 64-wide swizzle atom at a time, six stages
+// deep, so TMA latency hides behind the MMAs of earlier atoms.
 // Every wait is bounded; on a timeout the status word is set and the roles
 // wind down (the allocating warp still frees the tensor memory).
 #include <cuda.h>
@@ -39,19 +41,21 @@ namespace {
 
 constexpr int kTcM = 128;          // weight rows per tile
 constexpr int kTcN = 128;          // pairs per tile (max MMA N used)
-constexpr int kPkStages = 2;       // packed-weight stages (4 K groups each)
-constexpr int kPkGroups = 4;
-constexpr int kAStages = 2;        // dequantised A stages (one K group)
-constexpr int kBStages = 2;        // activation stages (one K group)
+constexpr int kPkStages = 3;       // packed-weight stages (2 K groups each)
+constexpr int kPkGroups = 2;
+constexpr int kAStages = 2;        // dequantised A stages (one K group = two atoms)
+constexpr int kBStages = 6;        // activation stages (one 64-wide atom each)
+constexpr int kDqWarps = 8;
+constexpr int kTcThreads = 32 * (2 + kDqWarps + 4);
 constexpr int kAccCols = 128;      // TMEM columns per accumulator buffer
 constexpr uint32_t kTmemCols = 256;
 
 constexpr int kAStageBytes = 2 * kTcM * 128;           // two 64-wide atoms
-constexpr int kBStageBytes = 2 * kTcN * 128;
+constexpr int kBStageBytes = kTcN * 128;
 constexpr int kPkQBytes = 8 * kPkGroups * 1024;        // 8 blob tiles
 constexpr int kPkSBytes = 8 * kPkGroups * 128;
 constexpr int kPkStageBytes = kPkQBytes + kPkSBytes;
-constexpr int kEpiBytes = 4 * 4096;                    // per epilogue warp: 32 x 32 fp32
+constexpr int kEpiBytes = 4 * 1024;                    // per epilogue warp: 1 KB
 
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kAStages * kAStageBytes;
@@ -77,9 +81,11 @@ struct Unit {
 }  // namespace
 
 size_t tc_smem_bytes() { return kTcSmem; }
+int tc_threads() { return kTcThreads; }
+static_assert(kTcSmem <= 232448, "shared memory budget");
 
 template <bool kGateUp>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -99,10 +105,10 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPkStages; ++s) {
       mbar_init(&pk_full[s], 1);
-      mbar_init(&pk_empty[s], 4);
+      mbar_init(&pk_empty[s], kDqWarps);
     }
     for (int s = 0; s < kAStages; ++s) {
-      mbar_init(&a_full[s], 4);
+      mbar_init(&a_full[s], kDqWarps);
       mbar_init(&a_empty[s], 1);
     }
     for (int s = 0; s < kBStages; ++s) {
@@ -202,18 +208,19 @@ __global__ void __launch_bounds__(320, 1)
                      ng * 128u, &pk_full[s]);
           }
         }
-        const int s = (int)(b_cnt % kBStages);
-        if (!wwait(&b_empty[s], ((b_cnt / kBStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
-        ++b_cnt;
-        uint8_t *dst = smem + kOffB + s * kBStageBytes;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&b_full[s], 2u * nb * 4096u);
-          for (int atom = 0; atom < 2; ++atom)
+        for (int atom = 0; atom < 2 && ok; ++atom) {
+          const int s = (int)(b_cnt % kBStages);
+          if (!wwait(&b_empty[s], ((b_cnt / kBStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
+          ++b_cnt;
+          uint8_t *dst = smem + kOffB + s * kBStageBytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&b_full[s], nb * 4096u);
             for (int rb = 0; rb < nb; ++rb)
-              tma_load_2d(dst + atom * (kTcN * 128) + rb * 4096, &tmap_b, g * 128 + atom * 64,
-                          un.pi0 + rb * 32, &b_full[s]);
+              tma_load_2d(dst + rb * 4096, &tmap_b, g * 128 + atom * 64, un.pi0 + rb * 32,
+                          &b_full[s]);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
     if (!ok) {
@@ -237,25 +244,29 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + buf * kAccCols;
       for (int g = 0; g < G; ++g) {
-        const int sa = (int)(a_cnt % kAStages), sb = (int)(b_cnt % kBStages);
+        const int sa = (int)(a_cnt % kAStages);
         if (!wwait(&a_full[sa], (a_cnt / kAStages) & 1u, p.status)) { ok = false; break; }
-        if (!wwait(&b_full[sb], (b_cnt / kBStages) & 1u, p.status)) { ok = false; break; }
         ++a_cnt;
-        ++b_cnt;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t a_addr = smem_u32(smem + kOffA + sa * kAStageBytes);
-          const uint32_t b_addr = smem_u32(smem + kOffB + sb * kBStageBytes);
+        const uint32_t a_addr = smem_u32(smem + kOffA + sa * kAStageBytes);
+        for (int atom = 0; atom < 2; ++atom) {
+          const int sb = (int)(b_cnt % kBStages);
+          if (!wwait(&b_full[sb], (b_cnt / kBStages) & 1u, p.status)) { ok = false; break; }
+          ++b_cnt;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t b_addr = smem_u32(smem + kOffB + sb * kBStageBytes);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t off = (j >> 2) * (kTcM * 128) + (j & 3) * 32;
-            const uint32_t boff = (j >> 2) * (kTcN * 128) + (j & 3) * 32;
-            umma_f16(d_tmem, umma_desc_sw128(a_addr + off), umma_desc_sw128(b_addr + boff), idesc,
-                     (g > 0 || j > 0) ? 1u : 0u);
+            for (int j = 0; j < 4; ++j) {
+              umma_f16(d_tmem, umma_desc_sw128(a_addr + atom * (kTcM * 128) + j * 32),
+                       umma_desc_sw128(b_addr + j * 32), idesc,
+                       (g > 0 || atom > 0 || j > 0) ? 1u : 0u);
+            }
+            umma_commit(&b_empty[sb]);
           }
-          umma_commit(&a_empty[sa]);
-          umma_commit(&b_empty[sb]);
+          __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) umma_commit(&a_empty[sa]);
         __syncwarp();
       }
       if (!ok) break;
@@ -263,7 +274,7 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       ++t_cnt_local;
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kDqWarps) {
     // -------------------------------------------------------- dequant
     const int dw = warp - 2;
     const int w = lane & 3;
@@ -285,8 +296,8 @@ __global__ void __launch_bounds__(320, 1)
         uint8_t *ad = smem + kOffA + sa * kAStageBytes;
         const int gi = g % kPkGroups;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int r = 32 * dw + 8 * m + row_in_8;
+        for (int m = 0; m < 2; ++m) {
+          const int r = 16 * dw + 8 * m + row_in_8;
           const int j = r >> 4, tr = r & 15;
           const uint4 qv = *reinterpret_cast<const uint4 *>(pq + j * (kPkGroups * 1024) + gi * 1024 +
                                                             tr * 64 + w * 16);
@@ -322,7 +333,7 @@ __global__ void __launch_bounds__(320, 1)
   } else {
     // -------------------------------------------------------- epilogue
     const int qd = warp & 3;  // TMEM lane quarter of this warp
-    float *stage = reinterpret_cast<float *>(smem + kOffEpi + (warp - 6) * 4096);
+    float *stage = reinterpret_cast<float *>(smem + kOffEpi + (warp - 2 - kDqWarps) * 1024);
     uint32_t t_cnt_local = 0;
     bool ok = true;
     int a = 0;
@@ -361,21 +372,25 @@ __global__ void __launch_bounds__(320, 1)
           }
           __syncwarp();
         } else {
+          // 8 pairs at a time through a 1 KB stage: [8 pairs][32 rows] fp32
 #pragma unroll
-          for (int t = 0; t < 32; ++t) stage[t * 32 + lane] = v[t];
-          __syncwarp();
+          for (int t8 = 0; t8 < 32; t8 += 8) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int piece = lane + 32 * k;  // 256 pieces of 16 bytes
-            const int t = piece >> 3, seg = piece & 7;
-            if (col0 + t < un.n) {
-              const float4 val = *reinterpret_cast<const float4 *>(stage + t * 32 + seg * 4);
-              float *dst = p.y_out + (size_t)(un.pi0 + col0 + t) * p.out_ld + 128 * un.rt +
-                           32 * qd + 4 * seg;
-              *reinterpret_cast<float4 *>(dst) = val;
+            for (int t = 0; t < 8; ++t) stage[t * 32 + lane] = v[t8 + t];
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int piece = lane + 32 * k;  // 64 pieces of 16 bytes
+              const int t = piece >> 3, seg = piece & 7;
+              if (col0 + t8 + t < un.n) {
+                const float4 val = *reinterpret_cast<const float4 *>(stage + t * 32 + seg * 4);
+                float *dst = p.y_out + (size_t)(un.pi0 + col0 + t8 + t) * p.out_ld + 128 * un.rt +
+                             32 * qd + 4 * seg;
+                *reinterpret_cast<float4 *>(dst) = val;
+              }
             }
+            __syncwarp();
           }
-          __syncwarp();
         }
       }
       tc_fence_before();

@@ -278,8 +278,8 @@ strata_status run_tc_experts(strata_moe *h, int T, const ExpertTable &table, cud
     auto kern = gu ? expert_tc_kernel<true> : expert_tc_kernel<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-      e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(320), smem, stream, true,
-                 p, m);
+      e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(tc_threads()), smem,
+                 stream, true, p, m);
     if (e != cudaSuccess) return cuda_status(e);
   }
   return STRATA_OK;
