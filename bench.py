@@ -76,6 +76,27 @@ def dist_env():
     return world, rank, local
 
 
+def replica_seed(seed, rank):
+    """Each replica draws its own token stream (the weights are shared)."""
+    return seed + rank
+
+
+def max_over_ranks(value, world, device):
+    """The slowest rank's time: every rank calls this in the same order."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank, world, ms_slowest):
+    """Replicas: every rank processes its own batch; all tokens / slowest time."""
+    return tokens_per_rank * world / (ms_slowest / 1000.0)
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """NVML samples of the SM clock and throttle reasons on one GPU."""
@@ -247,7 +268,7 @@ def main():
     cfg = synth.CONFIGS[args.config]
     T = args.tokens
     E, S = cfg.n_experts, cfg.n_shared
-    seed = args.seed + rank
+    seed = replica_seed(args.seed, rank)
 
     # --- the layer, every blob resident (slots bound in a seeded permutation)
     blobs = synth.make_all_blobs(cfg, args.seed)
@@ -327,12 +348,8 @@ def main():
     prof = binding.strata_moe_profile_read(layer.h)
     binding.strata_moe_profile(layer.h, False)
     step_ms = [a.elapsed_time(bb) for a, bb in ev]
-    ms = sum(step_ms) / len(step_ms)
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = T * world / (ms / 1000.0)
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world, "cuda")
+    value = whole_job_tokens_per_s(T, world, ms)
 
     # --- dominant kernel roofline (gate/up + SwiGLU)
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -372,11 +389,8 @@ def main():
         out_host.copy_(out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(bb) for a, bb in e2e_ev) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in e2e_ev) / e2e_steps, world,
+                            "cuda")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -402,7 +416,7 @@ def main():
                          "traffic": traffic, "algorithmic_bytes_per_launch": alg_gu,
                          "avg_launch_ms": avg_gu_ms},
             "phase_ms_per_launch": phase_ms,
-            "e2e": {"value": T * world / (e2e_ms / 1000.0), "unit": UNIT,
+            "e2e": {"value": whole_job_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": T * cfg.hidden * 2,
                     "d2h_bytes_per_step": T * cfg.hidden * 2, "ms_per_step": e2e_ms},
             "gpu_launches": launches,
