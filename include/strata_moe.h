@@ -84,7 +84,8 @@ typedef enum {
   STRATA_ERR_TOO_MANY_EXPERTS = 5, /* more distinct experts than slots were asked for */
   STRATA_ERR_OOM = 6,              /* workspace allocation failed */
   STRATA_ERR_CUDA = 7,             /* a CUDA runtime call failed */
-  STRATA_ERR_DEVICE_STATUS = 8     /* another device-side error (bad routing, timeout) */
+  STRATA_ERR_DEVICE_STATUS = 8,    /* another device-side error (bad routing, timeout) */
+  STRATA_ERR_SCRATCH_LIMIT = 9     /* too large for strata_moe_forward_noalloc's fixed scratch */
 } strata_status;
 
 /* Create a layer on the current CUDA device.
@@ -166,6 +167,42 @@ int strata_moe_last_device_bits(const strata_moe *h);
  * Errors: INVALID_ARG, CUDA. */
 strata_status strata_moe_profile(strata_moe *h, int enable);
 strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches, double *ms);
+
+/* Size of the fixed device scratch of strata_moe_forward_noalloc, and the
+ * most tokens one call of it takes. */
+#define STRATA_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define STRATA_NOALLOC_MAX_TOKENS 64
+
+/* strata_moe_forward, for callers that must not allocate device memory while
+ * they run: code under a memory manager that has carved the whole device into
+ * its own pools (a cudaMalloc would fail, or break up those pools), or a
+ * decode loop that cannot afford the device-wide synchronisation that
+ * cudaMalloc and cudaFree may cause.  The pages describe no such call; it has
+ * no counterpart there.
+ *
+ * Same arguments, result and errors as strata_moe_forward, with these
+ * differences.  The workspace is one fixed array of STRATA_NOALLOC_SCRATCH_BYTES
+ * bytes of device memory owned by the library (one per device), never the
+ * handle's workspace, and the call allocates nothing: no cudaMalloc, cudaFree
+ * or other allocating routine.  n_tokens may be at most
+ * STRATA_NOALLOC_MAX_TOKENS, and the workspace for n_tokens = T must fit the
+ * array: with P = T * (top_k + n_shared) and N = n_experts + n_shared, about
+ *     4*T*n_experts + 8*T*top_k + 4*(3N + 2) + 12*P + 2*T*hidden
+ *       + 2*P*inter + 4*P*hidden  bytes (each term rounded up to 256);
+ * a request beyond either limit returns STRATA_ERR_SCRATCH_LIMIT and
+ * enqueues nothing.  The current device must be the handle's device
+ * (otherwise INVALID_ARG).  The first call on a device looks up the array's
+ * address on that device (this can load the library's device code there),
+ * so make that first call before any stream capture.  Every call on a device,
+ * from any handle, uses the same array, and the array keeps what the last
+ * call left in it: the call clears what must start at zero and writes the
+ * rest before reading it, but calls whose work overlaps on the GPU (on
+ * different streams, without an ordering between them) race on the array and
+ * give wrong results.  Per-kernel timing (strata_moe_profile) is not recorded
+ * for this call.  The handle must not be used from another host thread
+ * during the call. */
+strata_status strata_moe_forward_noalloc(strata_moe *h, const void *x_bf16, int n_tokens,
+                                         void *out_bf16, strata_stream_t stream);
 
 /* Human-readable name of a status. */
 const char *strata_status_str(strata_status s);

@@ -29,6 +29,7 @@ class Status(enum.IntEnum):
     OOM = 6
     CUDA = 7
     DEVICE_STATUS = 8
+    SCRATCH_LIMIT = 9
 
 
 class StrataError(RuntimeError):
@@ -57,6 +58,7 @@ def load_library():
             "strata_moe_route": (I, [P, P, I, P, P, P, P]),
             "strata_moe_forward": (I, [P, P, I, P, P]),
             "strata_moe_forward_routed": (I, [P, P, I, P, P, P, P]),
+            "strata_moe_forward_noalloc": (I, [P, P, I, P, P]),
             "strata_moe_get_status": (I, [P, P]),
             "strata_moe_last_device_bits": (I, [P]),
             "strata_moe_profile": (I, [P, I]),
@@ -147,6 +149,15 @@ def strata_moe_forward_routed(h, x, n_tokens, idx, w, out, stream=None):
            "strata_moe_forward_routed")
 
 
+def strata_moe_forward_noalloc(h, x, n_tokens, out, stream=None):
+    _check(_load().strata_moe_forward_noalloc(h, _addr(x), n_tokens, _addr(out), _stream(stream)),
+           "strata_moe_forward_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_MAX_TOKENS = 64
+
+
 def strata_moe_get_status(h, stream=None):
     """Synchronise and return (Status, raw device bits); does not raise."""
     st = _load().strata_moe_get_status(h, _stream(stream))
@@ -212,6 +223,9 @@ class StrataMoE:
 
     def forward_routed(self, x, idx, w, out, stream=None):
         strata_moe_forward_routed(self.h, x, x.shape[0], idx, w, out, stream)
+
+    def forward_noalloc(self, x, out, stream=None):
+        strata_moe_forward_noalloc(self.h, x, x.shape[0], out, stream)
 
     def status(self, stream=None):
         return strata_moe_get_status(self.h, stream)

@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -397,6 +398,8 @@ const char *strata_status_str(strata_status s) {
     case STRATA_ERR_OOM: return "out of device memory";
     case STRATA_ERR_CUDA: return "CUDA error";
     case STRATA_ERR_DEVICE_STATUS: return "device-side error";
+    case STRATA_ERR_SCRATCH_LIMIT:
+      return "request larger than the fixed scratch of strata_moe_forward_noalloc";
   }
   return "unknown status";
 }
@@ -601,3 +604,166 @@ strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// strata_moe_forward_noalloc: the small-batch forward with its workspace in a
+// fixed device array of this file instead of the handle's growable
+// allocation.  It is for callers that may not allocate device memory at the
+// time of the call -- code running under a memory manager that owns the
+// whole device (every byte of HBM carved into pools at start-up, where a
+// cudaMalloc would fail or fragment them), or latency-bound decode loops that
+// cannot take the device-wide synchronisation cudaMalloc and cudaFree may
+// imply.  The array is shared by every handle on a device and keeps what the
+// last call left in it.
+
+static __device__ __align__(256) unsigned char noalloc_scratch[STRATA_NOALLOC_SCRATCH_BYTES];
+static_assert(STRATA_NOALLOC_MAX_TOKENS == kSmallT, "the no-allocation forward covers the small-batch path only");
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex noalloc_mutex;
+void *noalloc_base[kNoAllocMaxDevices];  // device address of the array, per device
+
+// Device address of the array on `device`, which must be the current device.
+// The first call on a device asks the runtime for it (this may load this
+// file's device code onto the device); later calls read the cached pointer.
+strata_status noalloc_scratch_on(int device, unsigned char **out) {
+  if (device < 0 || device >= kNoAllocMaxDevices) return STRATA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(noalloc_mutex);
+  if (!noalloc_base[device]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();
+      return STRATA_ERR_CUDA;
+    }
+    noalloc_base[device] = p;
+  }
+  *out = static_cast<unsigned char *>(noalloc_base[device]);
+  return STRATA_OK;
+}
+
+// Byte offsets in the array for T tokens: the routing kernel's block counter
+// (the only thing that must be zero when a call starts), then the regions of
+// the small-batch workspace.
+struct NoAllocLayout {
+  size_t counter, logits, idx, w, meta, ptok, pj, inv, x16, h16, y, total;
+};
+
+NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
+  const size_t P = (size_t)T * (h->k + h->S);
+  const int nid = h->E + h->S;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  NoAllocLayout L;
+  L.counter = take(sizeof(int));
+  L.logits = take(sizeof(float) * T * h->E);
+  L.idx = take(sizeof(int32_t) * T * h->k);
+  L.w = take(sizeof(float) * T * h->k);
+  L.meta = take(sizeof(int) * (3 * nid + 2));
+  L.ptok = take(sizeof(int) * P);
+  L.pj = take(sizeof(int) * P);
+  L.inv = take(sizeof(int) * P);
+  L.x16 = take(sizeof(__half) * T * h->H);
+  L.h16 = take(sizeof(__half) * P * h->I);
+  L.y = take(sizeof(float) * P * h->H);
+  L.total = off;
+  return L;
+}
+
+// For the lifetime of the object the handle's workspace pointers name regions
+// of the array; the handle's own come back when it goes out of scope (kernel
+// arguments are copied at launch, so enqueued work keeps the array's
+// addresses).  Per-kernel timing is off meanwhile: recording it creates
+// events and grows a host list.
+class NoAllocWorkspace {
+ public:
+  NoAllocWorkspace(strata_moe *h, unsigned char *base, const NoAllocLayout &L)
+      : h_(h), logits_(h->logits), idx_(h->idx), w_(h->w), meta_(h->meta), rt_(h->rt),
+        x16_(h->x16), h16_(h->h16), y_(h->y), xp_(h->xp), counter_(h->counter),
+        profiling_(h->profiling) {
+    const int nid = h->E + h->S;
+    h->logits = reinterpret_cast<float *>(base + L.logits);
+    h->idx = reinterpret_cast<int32_t *>(base + L.idx);
+    h->w = reinterpret_cast<float *>(base + L.w);
+    h->meta = reinterpret_cast<int *>(base + L.meta);
+    h->rt.cnt = h->meta;
+    h->rt.off = h->meta + nid;
+    h->rt.active = h->meta + 2 * nid + 1;
+    h->rt.n_active = h->meta + 3 * nid + 1;
+    h->rt.pair_tok = reinterpret_cast<int *>(base + L.ptok);
+    h->rt.pair_j = reinterpret_cast<int *>(base + L.pj);
+    h->rt.inv = reinterpret_cast<int *>(base + L.inv);
+    h->x16 = reinterpret_cast<__half *>(base + L.x16);
+    h->h16 = reinterpret_cast<__half *>(base + L.h16);
+    h->y = reinterpret_cast<float *>(base + L.y);
+    h->xp = nullptr;
+    h->counter = reinterpret_cast<int *>(base + L.counter);
+    h->profiling = false;
+  }
+  ~NoAllocWorkspace() {
+    h_->logits = logits_;
+    h_->idx = idx_;
+    h_->w = w_;
+    h_->meta = meta_;
+    h_->rt = rt_;
+    h_->x16 = x16_;
+    h_->h16 = h16_;
+    h_->y = y_;
+    h_->xp = xp_;
+    h_->counter = counter_;
+    h_->profiling = profiling_;
+  }
+  NoAllocWorkspace(const NoAllocWorkspace &) = delete;
+  NoAllocWorkspace &operator=(const NoAllocWorkspace &) = delete;
+
+ private:
+  strata_moe *h_;
+  float *logits_;
+  int32_t *idx_;
+  float *w_;
+  int *meta_;
+  Routing rt_;
+  __half *x16_, *h16_;
+  float *y_;
+  __half *xp_;
+  int *counter_;
+  bool profiling_;
+};
+
+}  // namespace
+
+extern "C" strata_status strata_moe_forward_noalloc(strata_moe *h, const void *x_bf16,
+                                                    int n_tokens, void *out_bf16,
+                                                    strata_stream_t stream) {
+  strata_status st = check_common(h, x_bf16, n_tokens, stream);
+  if (st != STRATA_OK) return st;
+  if (!h->router_W) return STRATA_ERR_INVALID_ARG;
+  for (int i = 0; i < h->S; ++i)
+    if (!h->shared_ptr[i]) return STRATA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return STRATA_OK;
+  if (!out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 15)) return STRATA_ERR_INVALID_ARG;
+  if (n_tokens > STRATA_NOALLOC_MAX_TOKENS) return STRATA_ERR_SCRATCH_LIMIT;
+  const NoAllocLayout L = noalloc_layout(h, n_tokens);
+  if (L.total > STRATA_NOALLOC_SCRATCH_BYTES) return STRATA_ERR_SCRATCH_LIMIT;
+  int device = -1;
+  if (cudaGetDevice(&device) != cudaSuccess) return STRATA_ERR_CUDA;
+  if (device != h->device) return STRATA_ERR_INVALID_ARG;
+  unsigned char *base = nullptr;
+  st = noalloc_scratch_on(device, &base);
+  if (st != STRATA_OK) return st;
+  // The routing kernel's block counter must start at zero; a call that timed
+  // out may have left it otherwise.  Everything else is written before it is
+  // read.
+  const cudaError_t e = cudaMemsetAsync(base + L.counter, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  NoAllocWorkspace ws(h, base, L);
+  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream, true);
+  if (st != STRATA_OK) return st;
+  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream, true);
+}
