@@ -7,27 +7,37 @@
 //   gate/up pass:  h = silu(Wg x) * (Wu x)  -> h16 [P][I] (f16)
 //   down pass:     y = Wd h                -> y   [P][H] (fp32)
 //
-// Tile = (expert, chunk of <= 128 of its pairs, 128 weight rows).  For
+// Tile = (expert, chunk of <= 256 of its pairs, 128 weight rows).  For
 // gate/up the 128 rows are 8 blob tiles, i.e. 64 gate rows and the same 64 up
 // rows interleaved by 8 (TMEM lane l holds gate if l % 16 < 8, else up; its
 // partner is lane l ^ 8, in the same warp).  For down they are 128
 // consecutive rows of Wd.
 //
 // Warp roles (one CTA per SM, persistent; tiles interleaved over CTAs):
-//   warp 0      producer: per 64 K elements a TMA load of the activation
-//               rows (f16, 128-byte swizzle; x_perm or h16), and every 2 K
-//               groups (of 128) one bulk copy per blob tile of packed weights
-//               and of scales;
-//   warp 1      MMA: allocates 256 TMEM columns (two 128-column accumulator
-//               buffers), and one thread issues 8 tcgen05.mma (M=128, N=pairs
-//               rounded up to 16, K=16) per K group, then commits to the
-//               stage barriers and, at the end of a tile, to the accumulator;
-//   warps 2-9   dequant: int4 -> exact f16 integers -> times the fp16 scale
+//   warp 0      activation producer: per 64 K elements (one swizzle atom)
+//               the activation rows (f16, 128-byte swizzle; x_perm or h16)
+//               in one 256-row TMA box, or in up to three 64-row boxes for
+//               shorter tiles;
+//   last warp   weight producer: per four K groups (of 128) one bulk copy per
+//               blob tile of packed weights and one of scales (its own warp,
+//               so the weight ring runs ahead of the activations).
+// The copy engine's per-operation cost, not bytes, limits this kernel when
+// the copies are small, so both producers move few, large pieces.
+//   warp 1      MMA: allocates all 512 TMEM columns (two 256-column
+//               accumulator buffers), and one thread issues 4 tcgen05.mma
+//               (M=128, N=pairs rounded up to 16, K=16) per atom, then
+//               commits to the stage barriers and, at the end of a tile, to
+//               the accumulator;
+//   warps 2-5   dequant: int4 -> exact f16 integers -> times the fp16 scale
 //               (one f16 rounding) -> the K-major 128-byte-swizzled A layout;
-//   warps 10-13 epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
+//   warps 6-9   epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
 //               transposed through shared memory, stored.
-// Activations are staged one 64-wide swizzle atom at a time, six stages
-// deep, so TMA latency hides behind the MMAs of earlier atoms.
+// Both operands are staged one 64-wide swizzle atom at a time in a ring of
+// three stages with one "full" barrier (dequant arrivals + activation bytes)
+// and one "empty" barrier (MMA commit) per stage; packed weights are six K
+// groups deep.
+// N = 256 matters: one M=128 MMA costs about the same issue time at N = 128
+// as at N = 256, so the wide tile nearly doubles tensor throughput.
 // Every wait is bounded; on a timeout the status word is set and the roles
 // wind down (the allocating warp still frees the tensor memory).
 #include <cuda.h>
@@ -40,17 +50,19 @@ namespace strata {
 namespace {
 
 constexpr int kTcM = 128;          // weight rows per tile
-constexpr int kTcN = 128;          // pairs per tile (max MMA N used)
-constexpr int kPkStages = 3;       // packed-weight stages (2 K groups each)
-constexpr int kPkGroups = 2;
-constexpr int kAStages = 2;        // dequantised A stages (one K group = two atoms)
-constexpr int kBStages = 6;        // activation stages (one 64-wide atom each)
-constexpr int kDqWarps = 8;
-constexpr int kTcThreads = 32 * (2 + kDqWarps + 4);
-constexpr int kAccCols = 128;      // TMEM columns per accumulator buffer
-constexpr uint32_t kTmemCols = 256;
+constexpr int kTcN = 256;          // pairs per tile (max MMA N used)
+constexpr int kPkStages = 2;       // packed-weight stages (four K groups each)
+constexpr int kPkGroups = 4;
+constexpr int kStages = 3;         // operand stages: one 64-wide atom of A and of B each
+constexpr int kDqWarps = 4;
+constexpr int kDqRows = kTcM / kDqWarps;    // weight rows per dequant warp
+static_assert(kDqRows % 8 == 0, "dequant warps cover whole 8-row groups");
+constexpr int kPkWarp = 2 + kDqWarps + 4;   // the last warp
+constexpr int kTcThreads = 32 * (kPkWarp + 1);
+constexpr int kAccCols = 256;      // TMEM columns per accumulator buffer
+constexpr uint32_t kTmemCols = 512;
 
-constexpr int kAStageBytes = 2 * kTcM * 128;           // two 64-wide atoms
+constexpr int kAStageBytes = kTcM * 128;               // one 64-wide atom
 constexpr int kBStageBytes = kTcN * 128;
 constexpr int kPkQBytes = 8 * kPkGroups * 1024;        // 8 blob tiles
 constexpr int kPkSBytes = 8 * kPkGroups * 128;
@@ -58,11 +70,11 @@ constexpr int kPkStageBytes = kPkQBytes + kPkSBytes;
 constexpr int kEpiBytes = 4 * 1024;                    // per epilogue warp: 1 KB
 
 constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kAStages * kAStageBytes;
-constexpr int kOffPk = kOffB + kBStages * kBStageBytes;
+constexpr int kOffB = kOffA + kStages * kAStageBytes;
+constexpr int kOffPk = kOffB + kStages * kBStageBytes;
 constexpr int kOffEpi = kOffPk + kPkStages * kPkStageBytes;
 constexpr int kOffBar = kOffEpi + kEpiBytes;
-constexpr int kNumBars = 2 * kPkStages + 2 * kAStages + 2 * kBStages + 4;
+constexpr int kNumBars = 2 * kPkStages + 2 * kStages + 4;
 constexpr int kOffTab = kOffBar + kNumBars * 8 + 16;   // + TMEM address slot
 constexpr int kTabBytes = kMaxIds * 8 + (3 * kMaxIds + 1) * 4;
 constexpr int kTcSmem = kOffTab + kTabBytes + 1024;    // + alignment slack
@@ -86,15 +98,17 @@ static_assert(kTcSmem <= 232448, "shared memory budget");
 
 template <bool kGateUp>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b) {
+    expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b64,
+                     const __grid_constant__ CUtensorMap tmap_b256) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint64_t *pk_full = bars, *pk_empty = pk_full + kPkStages;
-  uint64_t *a_full = pk_empty + kPkStages, *a_empty = a_full + kAStages;
-  uint64_t *b_full = a_empty + kAStages, *b_empty = b_full + kBStages;
-  uint64_t *acc_full = b_empty + kBStages, *acc_empty = acc_full + 2;
+  // full[s]: the 8 dequant warps' arrivals plus the activation TMA bytes;
+  // empty[s]: the MMAs that read stage s have completed
+  uint64_t *full = pk_empty + kPkStages, *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages, *acc_empty = acc_full + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
   const uint8_t **t_blob = reinterpret_cast<const uint8_t **>(smem + kOffTab);
   int *t_off = reinterpret_cast<int *>(t_blob + kMaxIds);
@@ -107,20 +121,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&pk_full[s], 1);
       mbar_init(&pk_empty[s], kDqWarps);
     }
-    for (int s = 0; s < kAStages; ++s) {
-      mbar_init(&a_full[s], kDqWarps);
-      mbar_init(&a_empty[s], 1);
-    }
-    for (int s = 0; s < kBStages; ++s) {
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], kDqWarps + 1);
+      mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], 4);
     }
     fence_mbar_init();
-    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_b64);
+    prefetch_tmap(&tmap_b256);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -183,104 +194,119 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   if (warp == 0) {
-    // -------------------------------------------------------- producer
-    uint32_t pk_cnt = 0, b_cnt = 0;
+    // -------------------------------------------------------- activation producer
+    uint32_t issued = 0, st = 0, ph = 0;
     bool ok = true;
     int a = 0;
     for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
       const Unit un = decode(u, a);
-      const int nb = (un.n + 31) / 32;        // 32-row boxes of activations
-      for (int g = 0; g < G && ok; ++g) {
-        if (g % kPkGroups == 0) {
-          const int s = (int)(pk_cnt % kPkStages);
-          if (!wwait(&pk_empty[s], ((pk_cnt / kPkStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
-          ++pk_cnt;
-          const int ng = min(kPkGroups, G - g);
-          uint8_t *dst = smem + kOffPk + s * kPkStageBytes;
-          if (lane == 0) mbar_arrive_expect_tx(&pk_full[s], 8u * ng * (1024u + 128u));
-          __syncwarp();
-          if (lane < 8) {
-            const int tile = un.rt * 8 + lane;
-            const size_t g0 = (size_t)tile * G + g;
-            bulk_g2s(dst + lane * (kPkGroups * 1024), un.blob + p.q_off + g0 * 1024, ng * 1024u,
-                     &pk_full[s]);
-            bulk_g2s(dst + kPkQBytes + lane * (kPkGroups * 128), un.blob + p.s_off + g0 * 128,
-                     ng * 128u, &pk_full[s]);
-          }
-        }
-        for (int atom = 0; atom < 2 && ok; ++atom) {
-          const int s = (int)(b_cnt % kBStages);
-          if (!wwait(&b_empty[s], ((b_cnt / kBStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
-          ++b_cnt;
-          uint8_t *dst = smem + kOffB + s * kBStageBytes;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&b_full[s], nb * 4096u);
+      const bool wide = un.n > 192;           // one 256-row box, else 64-row boxes
+      const int nb = wide ? 1 : (un.n + 63) / 64;
+      const uint32_t tx = wide ? 32768u : nb * 8192u;
+      for (int at = 0; at < 2 * G && ok; ++at) {
+        if (!wwait(&empty[st], ph ^ 1u, p.status)) { ok = false; break; }
+        uint8_t *dst = smem + kOffB + st * kBStageBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[st], tx);
+          if (wide)
+            tma_load_2d(dst, &tmap_b256, at * 64, un.pi0, &full[st]);
+          else
             for (int rb = 0; rb < nb; ++rb)
-              tma_load_2d(dst + rb * 4096, &tmap_b, g * 128 + atom * 64, un.pi0 + rb * 32,
-                          &b_full[s]);
-          }
-          __syncwarp();
+              tma_load_2d(dst + rb * 8192, &tmap_b64, at * 64, un.pi0 + rb * 64, &full[st]);
+        }
+        __syncwarp();
+        ++issued;
+        if (++st == kStages) {
+          st = 0;
+          ph ^= 1u;
         }
       }
     }
     if (!ok) {
-      // let issued copies land before the CTA exits
-      for (uint32_t m = pk_cnt > kPkStages ? pk_cnt - kPkStages : 0; m < pk_cnt; ++m)
-        (void)wwait(&pk_full[m % kPkStages], (m / kPkStages) & 1u, p.status);
-      for (uint32_t m = b_cnt > kBStages ? b_cnt - kBStages : 0; m < b_cnt; ++m)
-        (void)wwait(&b_full[m % kBStages], (m / kBStages) & 1u, p.status);
+      // let issued copies land before the CTA exits (bounded waits)
+      for (uint32_t m = issued > kStages ? issued - kStages : 0; m < issued; ++m)
+        (void)wwait(&full[m % kStages], (m / kStages) & 1u, p.status);
     }
-  } else if (warp == 1) {
-    // -------------------------------------------------------- MMA issue
-    uint32_t a_cnt = 0, b_cnt = 0, t_cnt_local = 0;
+  } else if (warp == kPkWarp) {
+    // -------------------------------------------------------- weight producer
+    uint32_t pk_cnt = 0;
     bool ok = true;
     int a = 0;
     for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
       const Unit un = decode(u, a);
-      const int N = (un.n + 15) & ~15;
-      const uint32_t idesc = umma_idesc_f16(kTcM, N);
-      const int buf = (int)(t_cnt_local & 1u);
-      if (!wwait(&acc_empty[buf], ((t_cnt_local >> 1) & 1u) ^ 1u, p.status)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + buf * kAccCols;
-      for (int g = 0; g < G; ++g) {
-        const int sa = (int)(a_cnt % kAStages);
-        if (!wwait(&a_full[sa], (a_cnt / kAStages) & 1u, p.status)) { ok = false; break; }
-        ++a_cnt;
-        const uint32_t a_addr = smem_u32(smem + kOffA + sa * kAStageBytes);
-        for (int atom = 0; atom < 2; ++atom) {
-          const int sb = (int)(b_cnt % kBStages);
-          if (!wwait(&b_full[sb], (b_cnt / kBStages) & 1u, p.status)) { ok = false; break; }
-          ++b_cnt;
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t b_addr = smem_u32(smem + kOffB + sb * kBStageBytes);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              umma_f16(d_tmem, umma_desc_sw128(a_addr + atom * (kTcM * 128) + j * 32),
-                       umma_desc_sw128(b_addr + j * 32), idesc,
-                       (g > 0 || atom > 0 || j > 0) ? 1u : 0u);
-            }
-            umma_commit(&b_empty[sb]);
-          }
-          __syncwarp();
+      for (int g = 0; g < G && ok; g += kPkGroups) {
+        const int s = (int)(pk_cnt % kPkStages);
+        if (!wwait(&pk_empty[s], ((pk_cnt / kPkStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
+        ++pk_cnt;
+        const int ng = min(kPkGroups, G - g);
+        uint8_t *dst = smem + kOffPk + s * kPkStageBytes;
+        if (lane == 0) mbar_arrive_expect_tx(&pk_full[s], 8u * ng * (1024u + 128u));
+        __syncwarp();
+        if (lane < 8) {
+          const int tile = un.rt * 8 + lane;
+          const size_t g0 = (size_t)tile * G + g;
+          bulk_g2s(dst + lane * (kPkGroups * 1024), un.blob + p.q_off + g0 * 1024, ng * 1024u,
+                   &pk_full[s]);
+          bulk_g2s(dst + kPkQBytes + lane * (kPkGroups * 128), un.blob + p.s_off + g0 * 128,
+                   ng * 128u, &pk_full[s]);
         }
-        if (!ok) break;
-        if (lane == 0) umma_commit(&a_empty[sa]);
         __syncwarp();
       }
-      if (!ok) break;
-      if (lane == 0) umma_commit(&acc_full[buf]);
-      __syncwarp();
-      ++t_cnt_local;
     }
+    if (!ok) {
+      for (uint32_t m = pk_cnt > kPkStages ? pk_cnt - kPkStages : 0; m < pk_cnt; ++m)
+        (void)wwait(&pk_full[m % kPkStages], (m / kPkStages) & 1u, p.status);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issue
+    // One thread does it all: per atom one wait, four MMAs, one commit, so
+    // the tensor pipe's queue never runs dry behind warp-level overheads.
+    if (lane == 0) {
+      uint32_t st = 0, ph = 0, t_cnt_local = 0;
+      bool ok = true;
+      int a = 0;
+      for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+        const Unit un = decode(u, a);
+        const int N = (un.n + 15) & ~15;
+        const uint32_t idesc = umma_idesc_f16(kTcM, N);
+        const int buf = (int)(t_cnt_local & 1u);
+        if (!mbar_wait(&acc_empty[buf], ((t_cnt_local >> 1) & 1u) ^ 1u, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * kAccCols;
+        for (int at = 0; at < 2 * G; ++at) {
+          if (!mbar_wait(&full[st], ph, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + kOffA + st * kAStageBytes);
+          const uint32_t b_addr = smem_u32(smem + kOffB + st * kBStageBytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            umma_f16(d_tmem, umma_desc_sw128(a_addr + j * 32), umma_desc_sw128(b_addr + j * 32),
+                     idesc, (at > 0 || j > 0) ? 1u : 0u);
+          umma_commit(&empty[st]);
+          if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+        ++t_cnt_local;
+      }
+    }
+    __syncwarp();
   } else if (warp < 2 + kDqWarps) {
     // -------------------------------------------------------- dequant
     const int dw = warp - 2;
     const int w = lane & 3;
     const int q = lane >> 2;
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
-    uint32_t pk_cnt = 0, a_cnt = 0;
+    uint32_t pk_cnt = 0, st = 0, ph = 0;
     bool ok = true;
     int a = 0;
     for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
@@ -288,49 +314,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int ps = (int)(pk_cnt % kPkStages);
         if (g % kPkGroups == 0)
           if (!wwait(&pk_full[ps], (pk_cnt / kPkStages) & 1u, p.status)) { ok = false; break; }
-        const int sa = (int)(a_cnt % kAStages);
-        if (!wwait(&a_empty[sa], ((a_cnt / kAStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
-        ++a_cnt;
         const uint8_t *pq = smem + kOffPk + ps * kPkStageBytes;
         const uint8_t *psc = pq + kPkQBytes;
-        uint8_t *ad = smem + kOffA + sa * kAStageBytes;
         const int gi = g % kPkGroups;
+        for (int atom = 0; atom < 2 && ok; ++atom) {
+          if (!wwait(&empty[st], ph ^ 1u, p.status)) { ok = false; break; }
+          uint8_t *ad = smem + kOffA + st * kAStageBytes;
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const int r = 16 * dw + 8 * m + row_in_8;
-          const int j = r >> 4, tr = r & 15;
-          const uint4 qv = *reinterpret_cast<const uint4 *>(pq + j * (kPkGroups * 1024) + gi * 1024 +
-                                                            tr * 64 + w * 16);
-          const uint2 sv = *reinterpret_cast<const uint2 *>(psc + j * (kPkGroups * 128) + gi * 128 +
-                                                            tr * 8);
-          const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
-          const __half2 sc[4] = {__half2half2(__low2half(bits_h2(sv.x))),
-                                 __half2half2(__high2half(bits_h2(sv.x))),
-                                 __half2half2(__low2half(bits_h2(sv.y))),
-                                 __half2half2(__high2half(bits_h2(sv.y)))};
+          for (int m = 0; m < kDqRows / 8; ++m) {
+            const int r = kDqRows * dw + 8 * m + row_in_8;
+            const int j = r >> 4, tr = r & 15;
+            // blocks 2 atom and 2 atom + 1 of this row: word w of each
+            const uint2 qv = *reinterpret_cast<const uint2 *>(
+                pq + j * (kPkGroups * 1024) + gi * 1024 + tr * 64 + w * 16 + atom * 8);
+            const uint32_t sv = *reinterpret_cast<const uint32_t *>(
+                psc + j * (kPkGroups * 128) + gi * 128 + tr * 8 + atom * 4);
+            const uint32_t words[2] = {qv.x, qv.y};
+            const __half2 sc[2] = {__half2half2(__low2half(bits_h2(sv))),
+                                   __half2half2(__high2half(bits_h2(sv)))};
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            uint32_t f[4];
-            int4x8_to_f16(words[b], f);
-            uint4 o;
-            o.x = h2_bits(__hmul2(bits_h2(f[0]), sc[b]));
-            o.y = h2_bits(__hmul2(bits_h2(f[1]), sc[b]));
-            o.z = h2_bits(__hmul2(bits_h2(f[2]), sc[b]));
-            o.w = h2_bits(__hmul2(bits_h2(f[3]), sc[b]));
-            const int chunk = ((b & 1) * 4 + w) ^ (r & 7);
-            *reinterpret_cast<uint4 *>(ad + (b >> 1) * (kTcM * 128) + r * 128 + chunk * 16) = o;
+            for (int b = 0; b < 2; ++b) {
+              uint32_t f[4];
+              int4x8_to_f16(words[b], f);
+              uint4 o;
+              o.x = h2_bits(__hmul2(bits_h2(f[0]), sc[b]));
+              o.y = h2_bits(__hmul2(bits_h2(f[1]), sc[b]));
+              o.z = h2_bits(__hmul2(bits_h2(f[2]), sc[b]));
+              o.w = h2_bits(__hmul2(bits_h2(f[3]), sc[b]));
+              const int chunk = (b * 4 + w) ^ (r & 7);
+              *reinterpret_cast<uint4 *>(ad + r * 128 + chunk * 16) = o;
+            }
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[st]);
+          if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
           }
         }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[sa]);
+        if (!ok) break;
         if (gi == kPkGroups - 1 || g == G - 1) {
           if (lane == 0) mbar_arrive(&pk_empty[ps]);
           ++pk_cnt;
         }
       }
     }
-  } else {
+  } else if (warp < kPkWarp) {
     // -------------------------------------------------------- epilogue
     const int qd = warp & 3;  // TMEM lane quarter of this warp
     float *stage = reinterpret_cast<float *>(smem + kOffEpi + (warp - 2 - kDqWarps) * 1024);
@@ -408,8 +438,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template __global__ void expert_tc_kernel<true>(TcParams, const __grid_constant__ CUtensorMap);
-template __global__ void expert_tc_kernel<false>(TcParams, const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<true>(TcParams, const __grid_constant__ CUtensorMap,
+                                               const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<false>(TcParams, const __grid_constant__ CUtensorMap,
+                                                const __grid_constant__ CUtensorMap);
 
 // x_perm[pair] = x16[token of pair], 16 bytes per thread.
 __global__ void gather_rows_kernel(const __half *__restrict__ x16, const int *__restrict__ pair_tok,

@@ -236,13 +236,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Rows of f16 activations [rows][K] as the B operand of the tensor-core
-// kernel: boxes of 64 K x 32 rows, 128-byte swizzle.
-bool encode_rows_map(CUtensorMap *m, const __half *base, int K, int rows) {
+// kernel: boxes of 64 K x box_rows rows, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap *m, const __half *base, int K, int rows, int box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {64, 32};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -274,13 +274,15 @@ strata_status run_tc_experts(strata_moe *h, int T, const ExpertTable &table, cud
     p.h_out = h->h16;
     p.y_out = h->y;
     p.status = h->status;
-    CUtensorMap m;
-    if (!encode_rows_map(&m, gu ? h->xp : h->h16, p.K, P)) return STRATA_ERR_CUDA;
+    CUtensorMap m64, m256;
+    if (!encode_rows_map(&m64, gu ? h->xp : h->h16, p.K, P, 64) ||
+        !encode_rows_map(&m256, gu ? h->xp : h->h16, p.K, P, 256))
+      return STRATA_ERR_CUDA;
     auto kern = gu ? expert_tc_kernel<true> : expert_tc_kernel<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
       e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(tc_threads()), smem,
-                 stream, true, p, m);
+                 stream, true, p, m64, m256);
     if (e != cudaSuccess) return cuda_status(e);
   }
   return STRATA_OK;
