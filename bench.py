@@ -42,6 +42,7 @@ import numpy as np  # noqa: E402
 from quantized_routed_expert_04_b200 import synth  # noqa: E402
 
 METRIC = "MoE-layer tokens/s"
+SMALL_T = 64  # the library's decode kernels serve up to this many tokens
 UNIT = "tokens/s"
 PHASES = ("router", "topk", "bucket", "pack", "gate_up", "down", "combine", "gather")
 
@@ -351,23 +352,42 @@ def main():
     ms = max_over_ranks(sum(step_ms) / len(step_ms), world, "cuda")
     value = whole_job_tokens_per_s(T, world, ms)
 
-    # --- dominant kernel roofline (gate/up + SwiGLU)
+    # --- dominant kernel roofline (gate/up + SwiGLU): the HBM-bound decode
+    # kernel for small batches, the tensor-core kernel for large ones
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(peaks_path):
         peaks = json.load(open(peaks_path))
-        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+        hbm_peak, tc_peak, peak_src = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"]), \
+            "measured"
     else:
-        hbm_peak, peak_src = 6650.0, "fallback"
+        hbm_peak, tc_peak, peak_src = 6650.0, 1590.0, "fallback"
     n_gu, ms_gu = prof["gate_up"]
     timed_ids = [(args.warmup + i) % n_batches for i in range(args.steps)]
-    alg_gu = sum(gateup_bytes[j] for j in timed_ids) / len(timed_ids)
     avg_gu_ms = ms_gu / max(1, n_gu)
-    achieved = alg_gu / (avg_gu_ms / 1000.0) / 1e9
-    traffic = traffic_from_profile(
-        ["quantized_routed_expert_04_b200/csrc/expert_mma.cu",
-         "quantized_routed_expert_04_b200/csrc/common.cuh"],
-        "expert_mma_gateup_%s_t%d" % (args.config, T))
     alg_step = sum(step_bytes[j] for j in timed_ids) / len(timed_ids)
+    if T <= SMALL_T:
+        alg_gu = sum(gateup_bytes[j] for j in timed_ids) / len(timed_ids)
+        traffic = traffic_from_profile(
+            ["quantized_routed_expert_04_b200/csrc/expert_mma.cu",
+             "quantized_routed_expert_04_b200/csrc/common.cuh"],
+            "expert_mma_gateup_%s_t%d" % (args.config, T))
+        roofline = {"kernel": "expert_mma_kernel<gate/up+SwiGLU>", "bound": "hbm",
+                    "achieved": alg_gu / (avg_gu_ms / 1000.0) / 1e9, "peak": hbm_peak,
+                    "unit": "GB/s", "peak_source": peak_src + " (copy kernel)",
+                    "algorithmic_bytes_per_launch": alg_gu}
+    else:
+        alg_gu = 4.0 * cfg.hidden * cfg.inter * T * (cfg.top_k + S)
+        traffic = traffic_from_profile(
+            ["quantized_routed_expert_04_b200/csrc/prefill_tc.cu",
+             "quantized_routed_expert_04_b200/csrc/common.cuh"],
+            "expert_tc_gateup_%s_t%d" % (args.config, T))
+        roofline = {"kernel": "expert_tc_kernel<gate/up+SwiGLU>", "bound": "tensor",
+                    "achieved": alg_gu / (avg_gu_ms / 1000.0) / 1e12, "peak": tc_peak,
+                    "unit": "TFLOP/s", "peak_source": peak_src + " (dense bf16 GEMM burst; "
+                    "f16 has the same rate)", "algorithmic_flops_per_launch": alg_gu}
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+    roofline["traffic"] = traffic
+    roofline["avg_launch_ms"] = avg_gu_ms
     phase_ms = {k: round(v[1] / max(1, v[0]), 5) for k, v in prof.items() if v[0]}
     launches = sum(v[0] for v in prof.values())
 
@@ -410,11 +430,10 @@ def main():
             "expert_weight_gbs": alg_step / (ms / 1000.0) / 1e9,
             "expert_weight_frac_of_hbm": alg_step / (ms / 1000.0) / 1e9 / hbm_peak,
             "tflops": flops_per_step / (ms / 1000.0) / 1e12,
-            "roofline": {"kernel": "expert_mma_kernel<gate/up+SwiGLU>", "bound": "hbm",
-                         "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "peak_source": peak_src,
-                         "traffic": traffic, "algorithmic_bytes_per_launch": alg_gu,
-                         "avg_launch_ms": avg_gu_ms},
+            "roofline": roofline,
+            "expert_gemm_tflops": (6.0 * cfg.hidden * cfg.inter * T * (cfg.top_k + S) /
+                                   ((prof["gate_up"][1] + prof["down"][1]) /
+                                    max(1, prof["gate_up"][0]) / 1000.0) / 1e12),
             "phase_ms_per_launch": phase_ms,
             "e2e": {"value": whole_job_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": T * cfg.hidden * 2,

@@ -91,6 +91,13 @@ CONFIGS = {
         zipf_beta=1.0,
         description="prefill: hidden 4096, inter 2048, 256 experts top-8 + 1 "
                     "shared, 8192 tokens, Zipf(0.8) router bias"),
+    # the prefill layer's shapes with 32 experts and 2048 tokens: small enough
+    # (about 0.5 GB of blobs) for profiler captures and quick parity runs
+    "prefill_small": LayerConfig(
+        "prefill_small", 4096, 2048, 32, 8, 1, 32, (2048,), bias="zipf", zipf_s=0.8,
+        zipf_beta=1.0,
+        description="prefill-shaped, small: hidden 4096, inter 2048, 32 experts "
+                    "top-8 + 1 shared, 2048 tokens, Zipf(0.8) router bias"),
 }
 
 
