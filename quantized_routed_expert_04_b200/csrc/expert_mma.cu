@@ -11,10 +11,13 @@
 //  * Work item = (active expert, group of <= 16 of its pairs, one 16-row
 //    weight tile): for gate/up, 8 rows of Wg and the same 8 rows of Wu (so a
 //    thread holds gate and up of one (row, pair) and SwiGLU is local); for
-//    down, 16 rows of Wd.  A persistent grid gives each CTA a contiguous range
-//    of items (equal weight bytes per CTA); inside a CTA, item q goes to warp
-//    q mod (warps per CTA), which computes it over the whole K range -- no
-//    cross-warp reduction, no rendezvous.
+//    down, 16 rows of Wd.  The (item, K group) pairs of the pass, laid end to
+//    end, are cut into one equal contiguous range per warp of the persistent
+//    grid (every warp streams the same number of weight bytes, to within one
+//    group).  An item that a cut splits is finished by the last of its
+//    pieces, which adds the pieces' partial sums in piece order (fixed, so
+//    the result does not depend on timing); all other items are computed
+//    whole by one warp, with no cross-warp reduction.
 //  * The blob stores a tile K-group by K-group, so any K chunk of a tile is
 //    one contiguous run of bytes.  Each warp streams its own items' chunks
 //    through a private ring of shared-memory stages: its lane 0 issues one
@@ -56,6 +59,24 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
 // (bulk copy) writes to the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Spin (with back-off and a time limit) until *counter reaches `target`;
+// acquire ordering for the reads that follow.
+__device__ __forceinline__ bool wait_count(const int *counter, int target, int *status) {
+  const uint64_t t0 = global_timer_ns();
+  unsigned ns = 32;
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, STATUS_TIMEOUT);
+      return false;
+    }
+    __nanosleep(ns);
+    if (ns < 512) ns <<= 1;
+  }
 }
 
 struct Item {
@@ -159,46 +180,66 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
   grid_dependency_launch();
 
   const int n_items = item_base[n_active];
-  const int i_begin = (int)((long long)n_items * blockIdx.x / gridDim.x);
-  const int i_end = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
   const int gpc = p.kc / 128;                    // K groups per (full) chunk
   const int groups = p.K / 128;                  // K groups per tile row
-  const int n_chunks = (groups + gpc - 1) / gpc; // the last chunk may be shorter
   const uint32_t q_stage = (uint32_t)p.kc * 8;   // scale offset inside a stage
   const int g = lane >> 2, cq = lane & 3;
 
-  // This warp's items: i_begin + warp, + kMmWarps, ...  Items of unbound
-  // experts are skipped and flagged.
-  auto next_item = [&](int i, int &a_hint) -> int {
-    for (; i < i_end; i += kMmWarps) {
-      while (item_base[a_hint + 1] <= i) ++a_hint;
-      if (at.blob[a_hint]) return i;
+  // This warp's share of the (item, group) sequence: [x_lo, x_hi); the
+  // first r = total mod W warps take q + 1 groups, the others q.
+  const int W = (int)gridDim.x * kMmWarps;
+  const int wg = (int)blockIdx.x * kMmWarps + warp;
+  const int total = n_items * groups;
+  const int q = total / W, r = total - (total / W) * W;
+  auto cut = [&](int w) -> int { return w * q + min(w, r); };
+  auto warp_of = [&](int x) -> int {  // the warp whose share holds x
+    return x < r * (q + 1) ? x / (q + 1) : r + (x - r * (q + 1)) / q;
+  };
+  const int x_lo = cut(wg), x_hi = cut(wg + 1);
+
+  // A piece: groups [g0, g1) of item `item`; x is its start in the sequence.
+  // Pieces of unbound experts are skipped and flagged.
+  struct Piece {
+    int item, g0, g1;
+  };
+  auto piece_at = [&](int x, int &a_hint, Piece &pc) -> bool {
+    while (x < x_hi) {
+      pc.item = x / groups;
+      pc.g0 = x - pc.item * groups;
+      pc.g1 = min(groups, pc.g0 + (x_hi - x));
+      while (item_base[a_hint + 1] <= pc.item) ++a_hint;
+      if (at.blob[a_hint]) return true;
       if (lane == 0) set_status(p.status, STATUS_NOT_BOUND);
+      x += pc.g1 - pc.g0;
     }
-    return i_end;
+    return false;
   };
 
-  // ---- copy issue; sequence number = (own item ordinal) * n_chunks + chunk
+  // ---- copy issue: this warp's pieces in order, gpc groups per stage
   int a_issue = 0;
-  int i_issue = next_item(i_begin + warp, a_issue);
-  int c_issue = 0;
+  Piece pc_issue;
+  int x_issue = x_lo;
+  bool have_issue = piece_at(x_issue, a_issue, pc_issue);
+  int cg_issue = have_issue ? pc_issue.g0 : 0;   // next group to copy
   uint32_t s_issue = 0;
   auto issue_next = [&]() {
-    if (i_issue >= i_end) return;
-    const Item it = decode_item(p, at, item_base, a_issue, i_issue);
+    if (!have_issue) return;
+    const Item it = decode_item(p, at, item_base, a_issue, pc_issue.item);
     const int slot = (int)(s_issue % p.stages);
     uint8_t *dst = ring + slot * p.stage_bytes;
+    const int ng = min(gpc, pc_issue.g1 - cg_issue);
     if (lane == 0) {
-      const size_t g0 = (size_t)it.tau * groups + (size_t)c_issue * gpc;
-      const uint32_t ng = (uint32_t)min(gpc, groups - c_issue * gpc);
-      mbar_arrive_expect_tx(&full[slot], ng * (1024u + 128u));
-      bulk_g2s(dst, it.blob + p.q_off + g0 * 1024, ng * 1024u, &full[slot]);
-      bulk_g2s(dst + q_stage, it.blob + p.s_off + g0 * 128, ng * 128u, &full[slot]);
+      const size_t g0 = (size_t)it.tau * groups + (size_t)cg_issue;
+      mbar_arrive_expect_tx(&full[slot], (uint32_t)ng * (1024u + 128u));
+      bulk_g2s(dst, it.blob + p.q_off + g0 * 1024, (uint32_t)ng * 1024u, &full[slot]);
+      bulk_g2s(dst + q_stage, it.blob + p.s_off + g0 * 128, (uint32_t)ng * 128u, &full[slot]);
     }
     ++s_issue;
-    if (++c_issue == n_chunks) {
-      c_issue = 0;
-      i_issue = next_item(i_issue + kMmWarps, a_issue);
+    cg_issue += ng;
+    if (cg_issue == pc_issue.g1) {
+      x_issue += pc_issue.g1 - pc_issue.g0;
+      have_issue = piece_at(x_issue, a_issue, pc_issue);
+      if (have_issue) cg_issue = pc_issue.g0;
     }
   };
   for (int s = 0; s < p.stages; ++s) issue_next();
@@ -216,6 +257,22 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
     }
     return p.b_src + (size_t)src * p.K;
   };
+  // Output of one (pair n, row g / g + 8) element pair of an item.
+  auto emit = [&](const Item &it, int n, float lo, float hi) {
+    const size_t prow = (size_t)(it.pi0 + n) * p.out_ld;
+    if (kGateUp) {
+      // lo: gate row i, hi: up row i, i = 8 tau + g
+      const float h = lo / (1.0f + expf(-lo)) * hi;
+      const int ii = it.tau * 8 + g;
+      // stored like the packed activations: group of 8 in order 0,4,1,5,2,6,3,7
+      const int pos = (ii & ~7) | (((ii & 3) << 1) | ((ii >> 2) & 1));
+      p.h_out[prow + pos] = __float2half_rn(h);
+    } else {
+      const int r0 = it.tau * 16 + g;
+      p.y_out[prow + r0] = lo;
+      p.y_out[prow + r0 + 8] = hi;
+    }
+  };
   uint4 bb0[NT][4], bb1[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -223,28 +280,31 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
     for (int b = 0; b < 4; ++b) bb0[nt][b] = bb1[nt][b] = make_uint4(0u, 0u, 0u, 0u);
   int pb = 0;  // buffer holding the current group's fragments
   int a = 0;
-  int i = next_item(i_begin + warp, a);
-  if (i < i_end) {
+  Piece pc;
+  int x = x_lo;
+  bool have = piece_at(x, a, pc);
+  if (have) {
     int a_tmp = a;
-    const Item it0 = decode_item(p, at, item_base, a_tmp, i);
+    const Item it0 = decode_item(p, at, item_base, a_tmp, pc.item);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) load_b(bb0[nt], act_row(it0, nt), 0, cq);
+    for (int nt = 0; nt < NT; ++nt) load_b(bb0[nt], act_row(it0, nt), pc.g0 * 128, cq);
   }
   uint32_t s_use = 0;
-  while (i < i_end) {
-    const Item it = decode_item(p, at, item_base, a, i);
+  while (have) {
+    const Item it = decode_item(p, at, item_base, a, pc.item);
     const int ntn = (it.ntok + 7) >> 3;
     int a_nx = a;
-    const int i_nx = next_item(i + kMmWarps, a_nx);
+    Piece pc_nx;
+    const bool have_nx = piece_at(x + (pc.g1 - pc.g0), a_nx, pc_nx);
     const __half *row_cur[NT], *row_nx[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       row_cur[nt] = act_row(it, nt);
       row_nx[nt] = nullptr;
     }
-    if (i_nx < i_end) {
+    if (have_nx) {
       int a_tmp = a_nx;
-      const Item it_nx = decode_item(p, at, item_base, a_tmp, i_nx);
+      const Item it_nx = decode_item(p, at, item_base, a_tmp, pc_nx.item);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) row_nx[nt] = act_row(it_nx, nt);
     }
@@ -254,20 +314,20 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
 #pragma unroll
       for (int v = 0; v < 4; ++v) acc[n][v] = 0.0f;
 
-    for (int c = 0; c < n_chunks; ++c, ++s_use) {
+    for (int cg = pc.g0; cg < pc.g1; ++s_use) {
       const int slot = (int)(s_use % p.stages);
       if (!warp_wait(&full[slot], (s_use / p.stages) & 1u, p.status)) return;
       const uint8_t *stq = ring + slot * p.stage_bytes;
       const uint8_t *sts = stq + q_stage;
-      const int ng = min(gpc, groups - c * gpc);
+      const int ng = min(gpc, pc.g1 - cg);
 #pragma unroll 4
       for (int j = 0; j < ng; ++j) {
-        // fragments of the next group: this item, else the next item
+        // fragments of the next group: this piece, else the next piece
         {
-          const int G_next = c * gpc + j + 1;
-          const bool same = G_next < groups;
-          if (same || i_nx < i_end) {
-            const int k0 = same ? G_next * 128 : 0;
+          const int G_next = cg + j + 1;
+          const bool same = G_next < pc.g1;
+          if (same || have_nx) {
+            const int k0 = (same ? G_next : pc_nx.g0) * 128;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const __half *r = same ? row_cur[nt] : row_nx[nt];
@@ -326,37 +386,80 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
         if (pb == 0) mma_group(bb0); else mma_group(bb1);
         pb ^= 1;
       }
+      cg += ng;
       // the stage's bytes are in registers now: refill it
       fence_proxy_async_smem();
       __syncwarp();
       issue_next();
     }
 
-    // ---- epilogue: this warp holds the complete sums of the item
+    // ---- epilogue
+    if (pc.g0 == 0 && pc.g1 == groups) {
+      // the whole item: this warp holds its complete sums
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      if (nt >= ntn) continue;
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int v = 0; v < 2; ++v) {
-        const int n = nt * 8 + 2 * cq + v;
-        if (n >= it.ntok) continue;
-        const size_t prow = (size_t)(it.pi0 + n) * p.out_ld;
-        if (kGateUp) {
-          // acc[v]: gate row i, acc[v + 2]: up row i, i = 8 tau + g
-          const float gv = acc[nt][v], uv = acc[nt][v + 2];
-          const float h = gv / (1.0f + expf(-gv)) * uv;
-          const int ii = it.tau * 8 + g;
-          // stored like the packed activations: group of 8 in order 0,4,1,5,2,6,3,7
-          const int pos = (ii & ~7) | (((ii & 3) << 1) | ((ii >> 2) & 1));
-          p.h_out[prow + pos] = __float2half_rn(h);
-        } else {
-          const int r0 = it.tau * 16 + g;
-          p.y_out[prow + r0] = acc[nt][v];
-          p.y_out[prow + r0 + 8] = acc[nt][v + 2];
+        for (int v = 0; v < 2; ++v) {
+          const int n = nt * 8 + 2 * cq + v;
+          if (nt < ntn && n < it.ntok) emit(it, n, acc[nt][v], acc[nt][v + 2]);
         }
+    } else {
+      // one piece of an item cut by warp shares.  Its pieces belong to the
+      // warps w_first .. w_last with non-empty shares; w_first's piece comes
+      // at the end of its share, the others at the start of theirs.  Each
+      // other piece stores its partial sums in its warp's slot and counts
+      // itself on w_first's counter (release: fence before the increment);
+      // w_first waits for them (acquire), adds the slots in warp order to
+      // its own sums and emits.
+      const int x_item = pc.item * groups;
+      const int w_first = warp_of(x_item), w_last = warp_of(x_item + groups - 1);
+      if (pc.g0 > 0) {
+        float *mine = p.partial + (size_t)wg * kMmSlotFloats;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int n = nt * 8 + 2 * cq + v;
+            if (nt < ntn && n < it.ntok) {
+              mine[n * 16 + g] = acc[nt][v];
+              mine[n * 16 + g + 8] = acc[nt][v + 2];
+            }
+          }
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(&p.counters[w_first], 1);
+        }
+      } else {
+        int others = 0;
+        for (int w = w_first + 1; w <= w_last; ++w) others += cut(w + 1) > cut(w);
+        int ok = 1;
+        if (lane == 0) ok = wait_count(&p.counters[w_first], others, p.status) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) return;
+        __threadfence();
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int n = nt * 8 + 2 * cq + v;
+            if (nt < ntn && n < it.ntok) {
+              float lo = acc[nt][v], hi = acc[nt][v + 2];
+              for (int w = w_first + 1; w <= w_last; ++w) {
+                if (cut(w + 1) == cut(w)) continue;  // empty share: no piece
+                const float *src = p.partial + (size_t)w * kMmSlotFloats;
+                lo += __ldcg(src + n * 16 + g);
+                hi += __ldcg(src + n * 16 + g + 8);
+              }
+              emit(it, n, lo, hi);
+            }
+          }
+        __syncwarp();
+        if (lane == 0) p.counters[w_first] = 0;  // ready for the next launch
       }
     }
-    i = i_nx;
+    x += pc.g1 - pc.g0;
+    pc = pc_nx;
+    have = have_nx;
     a = a_nx;
   }
 }

@@ -42,12 +42,15 @@ __global__ void combine_kernel(const float *y, const int32_t *idx, const float *
 // ---- expert matmuls for small token counts (expert_mma.cu)
 //
 // One work item = (active expert, group of <= 16 of its pairs, one 16-row
-// weight tile of the blob: 8 gate + 8 up rows, or 16 down rows).
+// weight tile of the blob: 8 gate + 8 up rows, or 16 down rows).  Each warp
+// of the grid takes an equal contiguous share of the (item, K group)
+// sequence; an item cut by a share boundary is finished by its last piece.
 constexpr int kMmMaxStages = 8;                     // stages per warp ring
 constexpr int kMmWarps = 12;                        // warps per CTA, each with its own ring
 constexpr int kMmThreads = 32 * kMmWarps;
 constexpr int kMmMaxGroup = 16;                     // pairs per item (two n8 MMA tiles)
 constexpr int kMmMaxPairs = 4096;                   // pair tokens staged in shared memory
+constexpr int kMmSlotFloats = kMmMaxGroup * 16;     // partial sums of one piece: pairs x rows
 
 struct MmParams {
   ExpertTable table;
@@ -66,6 +69,8 @@ struct MmParams {
   float *y_out;       // down output
   int *status;
   int stage_bytes;    // kc*8 weight bytes + kc scale bytes, rounded to 128
+  float *partial;     // [warps of the grid][kMmSlotFloats] partial sums of cut items
+  int *counters;      // [warps of the grid] pieces arrived per cut item (zero between launches)
 };
 
 template <bool kGateUp, int NT>   // NT: 8-pair MMA tiles per item (1 or 2)

@@ -56,6 +56,9 @@ struct strata_moe {
   __half *h16 = nullptr;
   float *y = nullptr;
   __half *xp = nullptr;     // activations gathered in sorted pair order (large batches)
+  float *partial = nullptr; // decode kernels: partial sums of items cut between warps
+  int *counters = nullptr;  // decode kernels: arrival counters (zero between launches)
+  size_t counters_bytes = 0;
   int *status = nullptr;    // device status word (own allocation)
   int *counter = nullptr;   // last-block counter of the small-batch routing kernel
   int last_bits = 0;
@@ -142,6 +145,9 @@ strata_status grow_workspace(strata_moe *h, int T) {
   const size_t o_h16 = take(sizeof(__half) * P * h->I);
   const size_t o_y = take(sizeof(float) * P * h->H);
   const size_t o_xp = cap > kSmallT ? take(sizeof(__half) * P * h->H) : 0;
+  const size_t n_counters = (size_t)kMmWarps * h->num_sms;
+  const size_t o_partial = take(sizeof(float) * n_counters * kMmSlotFloats);
+  const size_t o_counters = take(sizeof(int) * n_counters);
   void *mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, off);
   if (e != cudaSuccess) {
@@ -168,6 +174,12 @@ strata_status grow_workspace(strata_moe *h, int T) {
   h->h16 = reinterpret_cast<__half *>(b + o_h16);
   h->y = reinterpret_cast<float *>(b + o_y);
   h->xp = cap > kSmallT ? reinterpret_cast<__half *>(b + o_xp) : nullptr;
+  h->partial = reinterpret_cast<float *>(b + o_partial);
+  h->counters = reinterpret_cast<int *>(b + o_counters);
+  h->counters_bytes = sizeof(int) * n_counters;
+  e = cudaMemset(h->counters, 0, h->counters_bytes);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e);
   return STRATA_OK;
 }
 
@@ -180,13 +192,15 @@ ExpertTable make_table(const strata_moe *h) {
   return t;
 }
 
-// Stage size and count of the per-warp rings: K chunks of 512 elements (4 KB
-// of packed weights per copy; the last chunk of a row may be shorter), as
-// many stages as fit.
+// Stage size and count of the per-warp rings: K chunks of up to 512 elements
+// (4 KB of packed weights per copy; halved until three stages fit; a piece's
+// last chunk may be shorter), as many stages as fit.
 void pick_chunk(int K, int *kc_out, int *stages_out) {
   const size_t avail = 232448 - 1024 - mm_fixed_smem_bytes();
   const size_t per_warp = avail / kMmWarps;
-  const int kc = std::min(K, 512);
+  int kc = std::min(K, 512);
+  while (kc > 128 && per_warp / align_up((size_t)kc * 9, 128) < 3)
+    kc = std::max(128, kc / 256 * 128);
   const size_t stage = align_up((size_t)kc * 9, 128);
   *kc_out = kc;
   *stages_out = (int)std::max<size_t>(2, std::min<size_t>(kMmMaxStages, per_warp / stage));
@@ -219,6 +233,8 @@ MmParams mm_params(const strata_moe *h, bool gate_up, const ExpertTable &table, 
   p.y_out = h->y;
   p.status = h->status;
   p.stage_bytes = (int)align_up((size_t)p.kc * 9, 128);
+  p.partial = h->partial;
+  p.counters = h->counters;
   return p;
 }
 
@@ -569,6 +585,9 @@ strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream) {
     return STRATA_ERR_CUDA;
   if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return STRATA_ERR_CUDA;
   h->last_bits = bits;
+  if ((bits & STATUS_TIMEOUT) && h->counters &&
+      cudaMemset(h->counters, 0, h->counters_bytes) != cudaSuccess)
+    return STRATA_ERR_CUDA;
   if (bits & (STATUS_BAD_ROUTING | STATUS_TIMEOUT | STATUS_BOUNDS)) return STRATA_ERR_DEVICE_STATUS;
   if (bits & STATUS_NOT_BOUND) return STRATA_ERR_NOT_BOUND;
   return STRATA_OK;
@@ -650,7 +669,7 @@ strata_status noalloc_scratch_on(int device, unsigned char **out) {
 // (the only thing that must be zero when a call starts), then the regions of
 // the small-batch workspace.
 struct NoAllocLayout {
-  size_t counter, logits, idx, w, meta, ptok, pj, inv, x16, h16, y, total;
+  size_t counter, logits, idx, w, meta, ptok, pj, inv, x16, h16, y, counters, partial, total;
 };
 
 NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
@@ -674,6 +693,8 @@ NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
   L.x16 = take(sizeof(__half) * T * h->H);
   L.h16 = take(sizeof(__half) * P * h->I);
   L.y = take(sizeof(float) * P * h->H);
+  L.counters = take(sizeof(int) * kMmWarps * h->num_sms);
+  L.partial = take(sizeof(float) * kMmWarps * h->num_sms * kMmSlotFloats);
   L.total = off;
   return L;
 }
@@ -688,6 +709,7 @@ class NoAllocWorkspace {
   NoAllocWorkspace(strata_moe *h, unsigned char *base, const NoAllocLayout &L)
       : h_(h), logits_(h->logits), idx_(h->idx), w_(h->w), meta_(h->meta), rt_(h->rt),
         x16_(h->x16), h16_(h->h16), y_(h->y), xp_(h->xp), counter_(h->counter),
+        partial_(h->partial), counters_(h->counters),
         profiling_(h->profiling) {
     const int nid = h->E + h->S;
     h->logits = reinterpret_cast<float *>(base + L.logits);
@@ -706,6 +728,8 @@ class NoAllocWorkspace {
     h->y = reinterpret_cast<float *>(base + L.y);
     h->xp = nullptr;
     h->counter = reinterpret_cast<int *>(base + L.counter);
+    h->counters = reinterpret_cast<int *>(base + L.counters);
+    h->partial = reinterpret_cast<float *>(base + L.partial);
     h->profiling = false;
   }
   ~NoAllocWorkspace() {
@@ -719,6 +743,8 @@ class NoAllocWorkspace {
     h_->y = y_;
     h_->xp = xp_;
     h_->counter = counter_;
+    h_->partial = partial_;
+    h_->counters = counters_;
     h_->profiling = profiling_;
   }
   NoAllocWorkspace(const NoAllocWorkspace &) = delete;
@@ -735,6 +761,8 @@ class NoAllocWorkspace {
   float *y_;
   __half *xp_;
   int *counter_;
+  float *partial_;
+  int *counters_;
   bool profiling_;
 };
 
@@ -759,10 +787,13 @@ extern "C" strata_status strata_moe_forward_noalloc(strata_moe *h, const void *x
   unsigned char *base = nullptr;
   st = noalloc_scratch_on(device, &base);
   if (st != STRATA_OK) return st;
-  // The routing kernel's block counter must start at zero; a call that timed
-  // out may have left it otherwise.  Everything else is written before it is
-  // read.
-  const cudaError_t e = cudaMemsetAsync(base + L.counter, 0, sizeof(int), stream);
+  // The routing kernel's block counter and the decode kernels' arrival
+  // counters must start at zero (a call that timed out may have left them
+  // otherwise).  Everything else is written before it is read.
+  cudaError_t e = cudaMemsetAsync(base + L.counter, 0, sizeof(int), stream);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(base + L.counters, 0,
+                        sizeof(int) * kMmWarps * h->num_sms, stream);
   if (e != cudaSuccess) return cuda_status(e);
   NoAllocWorkspace ws(h, base, L);
   st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream, true);
