@@ -271,20 +271,32 @@ def main():
     E, S = cfg.n_experts, cfg.n_shared
     seed = replica_seed(args.seed, rank)
 
-    # --- the layer, every blob resident (slots bound in a seeded permutation)
+    # --- the layer: every blob resident (slots bound in a seeded permutation),
+    # or, for a layer with fewer slots than experts, an LRU arena filled per
+    # step from a pinned host pool of all experts (copies on a side stream,
+    # timed apart from the layer)
     blobs = synth.make_all_blobs(cfg, args.seed)
-    dev_blobs = torch.from_numpy(blobs).cuda()
     W, b = synth.make_router(cfg, args.seed)
     W_dev = torch.from_numpy(W).cuda()
     b_dev = None if b is None else torch.from_numpy(b).cuda()
-    n_slots = cfg.n_slots if cfg.n_slots == E else E
-    layer = binding.StrataMoE(cfg.hidden, cfg.inter, E, cfg.top_k, S, n_slots)
+    paged = cfg.n_slots < E
+    layer = binding.StrataMoE(cfg.hidden, cfg.inter, E, cfg.top_k, S, cfg.n_slots)
     layer.set_router(W_dev, b_dev)
-    for i in range(S):
-        layer.bind_shared(i, dev_blobs[E + i])
-    perm = synth.make_slot_permutation(cfg, args.seed) if n_slots == E else np.arange(E)
-    for s, e in enumerate(perm):
-        layer.bind_slot(s, int(e), dev_blobs[int(e)])
+    B_e = synth.expert_bytes(cfg.hidden, cfg.inter)
+    if paged:
+        dev_shared = torch.from_numpy(blobs[E:]).cuda()
+        for i in range(S):
+            layer.bind_shared(i, dev_shared[i])
+        pool = torch.from_numpy(np.ascontiguousarray(blobs[:E]).reshape(-1)).pin_memory()
+        arena_mem = torch.empty(cfg.n_slots * B_e, dtype=torch.uint8, device="cuda")
+        arena = binding.Arena(layer, pool, arena_mem)
+        copy_stream = torch.cuda.Stream()
+    else:
+        dev_blobs = torch.from_numpy(blobs).cuda()
+        for i in range(S):
+            layer.bind_shared(i, dev_blobs[E + i])
+        for s, e in enumerate(synth.make_slot_permutation(cfg, args.seed)):
+            layer.bind_slot(s, int(e), dev_blobs[int(e)])
     layer.reserve(T)
 
     steps_total = args.warmup + args.steps
@@ -300,7 +312,6 @@ def main():
     for x in xs:
         layer.route(x, None, idx_t, w_t)
         distinct.append(len(set(idx_t.cpu().numpy().reshape(-1).tolist())))
-    B_e = synth.expert_bytes(cfg.hidden, cfg.inter)
     gateup_bytes = [(d + S) * 2 * cfg.inter * cfg.hidden * 9 // 16 for d in distinct]
     step_bytes = [(d + S) * B_e for d in distinct]
     flops_per_step = 6 * cfg.hidden * cfg.inter * T * (cfg.top_k + S)
@@ -316,8 +327,35 @@ def main():
         flush.fill_(float(i))
         torch.sum(clean, dim=0, out=sink.view(()))
 
-    def step(i):
-        layer.forward(xs[i % n_batches], out)
+    idx_host = torch.empty(T, cfg.top_k, dtype=torch.int32).pin_memory()
+    paging = {"hits": 0, "misses": 0, "bytes": 0, "copy_ms": 0.0, "steps": 0}
+
+    def step(i, inner=None, x=None):
+        """One forward.  Paged: route, read the ids, make them resident,
+        forward with the routing; `inner` (4 events) brackets the two kernel
+        phases so that the copies in between are timed apart."""
+        x = xs[i % n_batches] if x is None else x
+        if not paged:
+            layer.forward(x, out)
+            return
+        if inner:
+            inner[0].record(stream)
+        layer.route(x, None, idx_t, w_t)
+        if inner:
+            inner[1].record(stream)
+        idx_host.copy_(idx_t)
+        hits, misses, nbytes = arena.ensure(idx_host.numpy().reshape(-1), stream=stream,
+                                            copy_stream=copy_stream)
+        if inner:
+            inner[2].record(stream)
+        layer.forward_routed(x, idx_t, w_t, out)
+        if inner:
+            inner[3].record(stream)
+            paging["hits"] += hits
+            paging["misses"] += misses
+            paging["bytes"] += nbytes
+            paging["copy_ms"] += arena.copy_ms()
+            paging["steps"] += 1
 
     for i in range(args.warmup):
         flush_l2(i)
@@ -332,6 +370,7 @@ def main():
     binding.strata_moe_profile_read(layer.h)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    inner = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -340,7 +379,7 @@ def main():
         for i in range(args.steps):
             flush_l2(i)
             ev[i][0].record(stream)
-            step(args.warmup + i)
+            step(args.warmup + i, inner[i] if paged else None)
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
@@ -348,7 +387,10 @@ def main():
         dist.barrier()
     prof = binding.strata_moe_profile_read(layer.h)
     binding.strata_moe_profile(layer.h, False)
-    step_ms = [a.elapsed_time(bb) for a, bb in ev]
+    if paged:  # layer kernels only: routing + forward, not the copies between them
+        step_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in inner]
+    else:
+        step_ms = [a.elapsed_time(bb) for a, bb in ev]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), world, "cuda")
     value = whole_job_tokens_per_s(T, world, ms)
 
@@ -405,7 +447,7 @@ def main():
         flush_l2(i)
         e2e_ev[i][0].record(stream)
         x_stage.copy_(x_host[i % 4], non_blocking=True)
-        layer.forward(x_stage, out)
+        step(i, x=x_stage)   # paged: includes the host routing read and the copies
         out_host.copy_(out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
@@ -442,6 +484,17 @@ def main():
             "clocks": clocks.summary(),
             "wall_s_timed_region": t_wall,
         }
+        if paged:
+            n = max(1, paging["steps"])
+            line["paging"] = {
+                "n_slots": cfg.n_slots, "note": "layer time (value) excludes the expert copies; "
+                "e2e includes them and the host read of the routing",
+                "hits_per_step": paging["hits"] / n, "misses_per_step": paging["misses"] / n,
+                "copy_bytes_per_step": paging["bytes"] / n,
+                "copy_ms_per_step": paging["copy_ms"] / n,
+                "copy_gbs": (paging["bytes"] / max(paging["copy_ms"], 1e-9) / 1e6)}
+            line["data"] = "synthetic (seeded); %d of %d experts resident, the rest in pinned " \
+                           "host memory" % (cfg.n_slots, E)
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line))

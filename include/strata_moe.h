@@ -168,6 +168,54 @@ int strata_moe_last_device_bits(const strata_moe *h);
 strata_status strata_moe_profile(strata_moe *h, int enable);
 strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches, double *ms);
 
+/* ---- Expert arena: least-recently-used residency of routed experts.
+ * The paging layer in front of the slot table (ro99/strata README,
+ * "Residency": routed experts leased into VRAM per step through an LRU cache
+ * from pinned host memory; "Strata on a Mac", "What you need": a fixed arena
+ * of experts, the rest read in as tokens need them).  An arena owns the
+ * layer's slot table: it binds slot s to device memory
+ * arena_dev + s * strata_moe_expert_bytes(hidden, inter).  Results do not
+ * depend on the arena's choices, only copy traffic does. */
+typedef struct strata_arena strata_arena; /* opaque */
+
+typedef struct {
+  int hits;     /* requested experts that were already resident */
+  int misses;   /* requested experts copied in by this call */
+  size_t bytes; /* bytes copied host -> device by this call */
+} strata_arena_stats;
+
+/* Create an arena for `layer` (which must outlive it).  host_pool: host
+ * memory holding all n_experts blobs back to back in expert order
+ * (strata_moe_expert_bytes apart), ideally pinned (pageable memory makes the
+ * copies synchronous); arena_dev: device memory for n_slots blobs, 256-byte
+ * aligned.  Both stay owned by the caller and must outlive the arena.  All
+ * slots of the layer are emptied.  Errors: INVALID_ARG, OOM, CUDA. */
+strata_status strata_arena_create(strata_moe *layer, const void *host_pool, void *arena_dev,
+                                  strata_arena **out);
+void strata_arena_destroy(strata_arena *a);
+
+/* Make the experts ids[0..n) (host int32, repeats allowed) resident before the
+ * work that `stream` runs next.  Resident ones are hits and become most
+ * recently used; each miss is copied (one cudaMemcpyAsync on copy_stream) into
+ * the lowest empty slot, else into the least recently used slot not asked for
+ * by this call (ties: lowest slot), and bound there.  copy_stream first waits
+ * for the work already queued on `stream` (an evicted expert may still be read
+ * there); `stream` then waits for the copies.  stats (may be NULL) receives
+ * hits, misses and bytes.  Host-side and asynchronous; the layer's slot
+ * table changes at once, so enqueue the forward that uses these experts on
+ * `stream` after this call.  Errors: INVALID_ARG (an id out of range),
+ * TOO_MANY_EXPERTS (more distinct ids than slots; nothing changes), CUDA. */
+strata_status strata_arena_ensure(strata_arena *a, const int32_t *ids, int n,
+                                  strata_stream_t stream, strata_stream_t copy_stream,
+                                  strata_arena_stats *stats);
+
+/* Wait for the copies of the last ensure call and return their device time in
+ * milliseconds (0 if it copied nothing).  Errors: INVALID_ARG, CUDA. */
+strata_status strata_arena_copy_ms(strata_arena *a, float *ms);
+
+/* Slot holding expert_id, -1 if it is not resident, -2 if out of range. */
+int strata_arena_slot_of(const strata_arena *a, int expert_id);
+
 /* Size of the fixed device scratch of strata_moe_forward_noalloc, and the
  * most tokens one call of it takes. */
 #define STRATA_NOALLOC_SCRATCH_BYTES (16u << 20)

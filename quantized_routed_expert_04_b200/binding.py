@@ -32,6 +32,10 @@ class Status(enum.IntEnum):
     SCRATCH_LIMIT = 9
 
 
+class ArenaStats(ctypes.Structure):
+    _fields_ = [("hits", ctypes.c_int), ("misses", ctypes.c_int), ("bytes", ctypes.c_size_t)]
+
+
 class StrataError(RuntimeError):
     def __init__(self, status, where=""):
         self.status = Status(status)
@@ -64,6 +68,11 @@ def load_library():
             "strata_moe_profile": (I, [P, I]),
             "strata_moe_profile_read": (I, [P, I, P, P]),
             "strata_status_str": (ctypes.c_char_p, [I]),
+            "strata_arena_create": (I, [P, P, P, ctypes.POINTER(P)]),
+            "strata_arena_destroy": (None, [P]),
+            "strata_arena_ensure": (I, [P, P, I, P, P, ctypes.POINTER(ArenaStats)]),
+            "strata_arena_copy_ms": (I, [P, ctypes.POINTER(ctypes.c_float)]),
+            "strata_arena_slot_of": (I, [P, I]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -182,6 +191,66 @@ def strata_moe_profile_read(h):
 
 def strata_status_str(st):
     return _load().strata_status_str(int(st)).decode()
+
+
+def strata_arena_create(layer_h, host_pool, arena_dev):
+    a = ctypes.c_void_p()
+    _check(_load().strata_arena_create(layer_h, _addr(host_pool), _addr(arena_dev),
+                                       ctypes.byref(a)), "strata_arena_create")
+    return a.value
+
+
+def strata_arena_destroy(a):
+    _load().strata_arena_destroy(a)
+
+
+def strata_arena_ensure(a, ids, stream=None, copy_stream=None):
+    """ids: a sequence of expert ids (host).  Returns (hits, misses, bytes)."""
+    import numpy as np
+    arr = np.ascontiguousarray(np.asarray(ids, dtype=np.int32).reshape(-1))
+    st = ArenaStats()
+    _check(_load().strata_arena_ensure(a, arr.ctypes.data, int(arr.size), _stream(stream),
+                                       _stream(copy_stream), ctypes.byref(st)),
+           "strata_arena_ensure")
+    return st.hits, st.misses, int(st.bytes)
+
+
+def strata_arena_copy_ms(a):
+    ms = ctypes.c_float()
+    _check(_load().strata_arena_copy_ms(a, ctypes.byref(ms)), "strata_arena_copy_ms")
+    return ms.value
+
+
+def strata_arena_slot_of(a, expert_id):
+    return int(_load().strata_arena_slot_of(a, expert_id))
+
+
+class Arena:
+    """Owning wrapper of an expert arena over a StrataMoE layer."""
+
+    def __init__(self, layer, host_pool, arena_dev):
+        self.layer, self.host_pool, self.arena_dev = layer, host_pool, arena_dev
+        self.a = strata_arena_create(layer.h, host_pool, arena_dev)
+
+    def ensure(self, ids, stream=None, copy_stream=None):
+        return strata_arena_ensure(self.a, ids, stream, copy_stream)
+
+    def copy_ms(self):
+        return strata_arena_copy_ms(self.a)
+
+    def slot_of(self, expert_id):
+        return strata_arena_slot_of(self.a, expert_id)
+
+    def close(self):
+        if self.a:
+            strata_arena_destroy(self.a)
+            self.a = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class StrataMoE:

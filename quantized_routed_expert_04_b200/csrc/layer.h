@@ -60,3 +60,9 @@ struct Routing {
 };
 
 }  // namespace strata
+
+struct strata_moe;
+// Shape of a layer handle (for the arena, which sees the handle only through
+// the public calls): hidden, inter, routed experts, arena slots, device.
+void strata_handle_shape(const strata_moe *h, int *hidden, int *inter, int *n_experts,
+                         int *n_slots, int *device);

@@ -514,6 +514,19 @@ strata_status strata_moe_bind_slot(strata_moe *h, int slot, int expert_id, const
   return STRATA_OK;
 }
 
+}  // extern "C"
+
+void strata_handle_shape(const strata_moe *h, int *hidden, int *inter, int *n_experts,
+                         int *n_slots, int *device) {
+  *hidden = h->H;
+  *inter = h->I;
+  *n_experts = h->E;
+  *n_slots = h->n_slots;
+  *device = h->device;
+}
+
+extern "C" {
+
 int strata_moe_slot_expert(const strata_moe *h, int slot) {
   if (!h || slot < 0 || slot >= h->n_slots) return -2;
   return h->slot_expert[slot];
