@@ -65,58 +65,97 @@ __global__ void router_gemv_kernel(const __nv_bfloat16 *__restrict__ x,
 }
 
 // ---------------------------------------------------------------- router GEMM
-// 64 tokens x 64 experts per block; each thread owns 4 x 4 logits and adds
-// products in ascending h, in double.  Used for large batches (prefill).
-constexpr int kRT = 64, kRE = 64, kRK = 32;
+// Large batches (prefill): logits of 128 tokens x 64 experts per block on the
+// fp64 tensor-core path (mma.m8n8k4, f64 in and out).  The bf16 x fp32
+// products are exact in fp64 and every sum is an fp64 sum, rounded once to
+// fp32 at the end; the order of the fp64 additions differs from a plain
+// ascending loop, which moves a logit by at most about 1e-11 relative before
+// that rounding.  8 warps as 4 (tokens) x 2 (experts), each 32 x 32 = 4 x 4
+// tiles of 8 x 8; K staged 16 at a time in shared memory as doubles, the
+// next K slice prefetched into registers during the MMAs.
+constexpr int kRT = 128, kRE = 64, kRK = 16;
+constexpr int kRXL = kRT + 8, kRWL = kRE + 8;   // padded rows (2-way bank spread)
+
+__device__ __forceinline__ void dmma_8x8x4(double &d0, double &d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1)
+               : "d"(a), "d"(b));
+}
 
 __global__ void __launch_bounds__(256) router_gemm_kernel(
     const __nv_bfloat16 *__restrict__ x, const float *__restrict__ W,
     const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits) {
   grid_dependency_wait();
-  __shared__ float xs[kRK][kRT + 1];
-  __shared__ float ws[kRK][kRE + 1];
+  __shared__ double xs[kRK][kRXL];
+  __shared__ double ws[kRK][kRWL];
   const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  double acc[4][4];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wt = (warp & 3) * 32, we = (warp >> 2) * 32;   // warp tile origin in the block
+  // global -> register staging: one 16-byte piece of x and of W per thread
+  const int xr = tid >> 1, xc = (tid & 1) * 8;              // token row, k offset (8 bf16)
+  const int wr = tid >> 2, wc = (tid & 3) * 4;              // expert row, k offset (4 fp32)
+  const bool x_ok = t0 + xr < T, w_ok = e0 + wr < E;
+  const __nv_bfloat16 *xp = x + (size_t)(x_ok ? t0 + xr : 0) * H + xc;
+  const float *wp = W + (size_t)(w_ok ? e0 + wr : 0) * H + wc;
+  uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+  float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (x_ok) xv = *reinterpret_cast<const uint4 *>(xp);
+  if (w_ok) wv = *reinterpret_cast<const float4 *>(wp);
+
+  double acc[4][4][2];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+
   for (int k0 = 0; k0 < H; k0 += kRK) {
-    for (int v = tid; v < kRT * kRK; v += 256) {
-      const int r = v / kRK, c = v % kRK;
-      const int t = t0 + r;
-      xs[c][r] = t < T ? __bfloat162float(x[(size_t)t * H + k0 + c]) : 0.0f;
-      const int e = e0 + r;
-      ws[c][r] = e < E ? W[(size_t)e * H + k0 + c] : 0.0f;
+    {
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xv);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(h2[q]);
+        xs[xc + 2 * q][xr] = (double)f.x;
+        xs[xc + 2 * q + 1][xr] = (double)f.y;
+      }
+      ws[wc + 0][wr] = (double)wv.x;
+      ws[wc + 1][wr] = (double)wv.y;
+      ws[wc + 2][wr] = (double)wv.z;
+      ws[wc + 3][wr] = (double)wv.w;
     }
     __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kRK; ++kk) {
+    if (k0 + kRK < H) {
+      if (x_ok) xv = *reinterpret_cast<const uint4 *>(xp + k0 + kRK);
+      if (w_ok) wv = *reinterpret_cast<const float4 *>(wp + k0 + kRK);
+    }
+#pragma unroll
+    for (int kk = 0; kk < kRK; kk += 4) {
       double a[4], b[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
+      for (int i = 0; i < 4; ++i) a[i] = xs[kk + (lane & 3)][wt + 8 * i + (lane >> 2)];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = ws[kk][tx * 4 + j];
+      for (int j = 0; j < 4; ++j) b[j] = ws[kk + (lane & 3)][we + 8 * j + (lane >> 2)];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
     }
     __syncthreads();
   }
+  // lane holds rows (lane >> 2) and columns 2 (lane & 3) + {0, 1} of each tile
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
+    const int t = t0 + wt + 8 * i + (lane >> 2);
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e >= E) continue;
-      double v = acc[i][j];
-      if (bias) v += (double)bias[e];
-      logits[(size_t)t * E + e] = (float)v;
-    }
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int e = e0 + we + 8 * j + 2 * (lane & 3) + c;
+        if (e >= E) continue;
+        double v = acc[i][j][c];
+        if (bias) v += (double)bias[e];
+        logits[(size_t)t * E + e] = (float)v;
+      }
   }
 }
 

@@ -393,7 +393,7 @@ strata_status run_router(strata_moe *h, const void *x, int T, float *logits, int
                  false, p);
     return cuda_status(e);
   }
-  e = launch(h, PH_ROUTER, router_gemm_kernel, dim3((T + 63) / 64, (h->E + 63) / 64), dim3(256), 0,
+  e = launch(h, PH_ROUTER, router_gemm_kernel, dim3((T + 127) / 128, (h->E + 63) / 64), dim3(256), 0,
              stream, false, xb, h->router_W, h->router_b, T, h->H, h->E, logits);
   if (e == cudaSuccess)
     e = launch(h, PH_TOPK, topk_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, true, logits, T,
