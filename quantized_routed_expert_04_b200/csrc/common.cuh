@@ -54,22 +54,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Wait for the barrier phase, backing off with nanosleep between polls (for
-// waits off the critical path, e.g. a producer waiting for a free stage).
-__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, int *status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_timer_ns();
-  unsigned ns = 32;
-  while (true) {
-    __nanosleep(ns);
-    if (ns < 256) ns <<= 1;
-    if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      set_status(status, STATUS_TIMEOUT);
-      return false;
-    }
-  }
-}
 
 // try_wait with a suspend-time hint: the thread sleeps until the phase
 // completes or about 1 ms passes, instead of spinning.
@@ -120,19 +104,7 @@ __device__ __forceinline__ void grid_dependency_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---------------------------------------------------------------- loads
-__device__ __forceinline__ uint32_t ld_nc_u32(const void *p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
 
-// ---------------------------------------------------------------- tensor core (legacy)
-__device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
 
 // D = A * B + C, A 16x16 f16 (row), B 16x8 f16 (col), C/D 16x8 f32.
 // (Not volatile: it has no side effects, so the compiler may interleave

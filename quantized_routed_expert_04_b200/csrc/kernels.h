@@ -9,8 +9,6 @@
 namespace strata {
 
 // ---- routing (route.cu)
-__global__ void router_gemv_kernel(const __nv_bfloat16 *x, const float *W, const float *bias,
-                                   int T, int H, int E, float *logits);
 __global__ void router_gemm_kernel(const __nv_bfloat16 *x, const float *W, const float *bias,
                                    int T, int H, int E, float *logits);
 __global__ void topk_kernel(const float *logits, int T, int E, int k, int32_t *idx, float *w);

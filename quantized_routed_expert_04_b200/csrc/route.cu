@@ -20,50 +20,6 @@
 
 namespace strata {
 
-// ---------------------------------------------------------------- router GEMV
-// One warp per expert row, all tokens in groups of kTokGroup; each lane sums
-// its strided share of h in double, then a fixed xor-shuffle tree adds the
-// lanes.  Used for small batches (decode).
-constexpr int kTokGroup = 8;
-
-__global__ void router_gemv_kernel(const __nv_bfloat16 *__restrict__ x,
-                                   const float *__restrict__ W, const float *__restrict__ bias,
-                                   int T, int H, int E, float *__restrict__ logits) {
-  grid_dependency_wait();
-  const int lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (e >= E) return;
-  const float *wr = W + (size_t)e * H;
-  for (int t0 = 0; t0 < T; t0 += kTokGroup) {
-    const int nt = min(kTokGroup, T - t0);
-    double acc[kTokGroup];
-#pragma unroll
-    for (int i = 0; i < kTokGroup; ++i) acc[i] = 0.0;
-    for (int h = lane * 2; h < H; h += 64) {
-      const float2 wv = *reinterpret_cast<const float2 *>(wr + h);
-#pragma unroll
-      for (int i = 0; i < kTokGroup; ++i) {
-        if (i < nt) {
-          const __nv_bfloat162 xv =
-              *reinterpret_cast<const __nv_bfloat162 *>(x + (size_t)(t0 + i) * H + h);
-          const float2 xf = __bfloat1622float2(xv);
-          acc[i] = fma((double)xf.x, (double)wv.x, acc[i]);
-          acc[i] = fma((double)xf.y, (double)wv.y, acc[i]);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kTokGroup; ++i) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-    }
-    if (lane == 0) {
-      const double b = bias ? (double)bias[e] : 0.0;
-      for (int i = 0; i < nt; ++i) logits[(size_t)(t0 + i) * E + e] = (float)(acc[i] + b);
-    }
-  }
-}
-
 // ---------------------------------------------------------------- router GEMM
 // Large batches (prefill): logits of 128 tokens x 64 experts per block on the
 // fp64 tensor-core path (mma.m8n8k4, f64 in and out).  The bf16 x fp32
