@@ -308,11 +308,10 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) row_nx[nt] = act_row(it_nx, nt);
     }
-    float acc[NT][4];
+    // acc[nt][0] = (row g: pair 2c, 2c + 1), acc[nt][1] = (row g + 8: same pairs)
+    float2 acc[NT][2];
 #pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) acc[n][v] = 0.0f;
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = make_float2(0.0f, 0.0f);
 
     for (int cg = pc.g0; cg < pc.g1; ++s_use) {
       const int slot = (int)(s_use % p.stages);
@@ -374,11 +373,11 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
                 mma_16816(d[b], a1, bv[nt][b].z, bv[nt][b].w, d[b]);
               }
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                acc[nt][0] = fmaf(sc0[b], d[b][0], acc[nt][0]);
-                acc[nt][1] = fmaf(sc0[b], d[b][1], acc[nt][1]);
-                acc[nt][2] = fmaf(sc1[b], d[b][2], acc[nt][2]);
-                acc[nt][3] = fmaf(sc1[b], d[b][3], acc[nt][3]);
+              for (int b = 0; b < 4; ++b) {  // paired fp32 FMAs (same rounding as two fmaf)
+                acc[nt][0] = __ffma2_rn(make_float2(sc0[b], sc0[b]), make_float2(d[b][0], d[b][1]),
+                                        acc[nt][0]);
+                acc[nt][1] = __ffma2_rn(make_float2(sc1[b], sc1[b]), make_float2(d[b][2], d[b][3]),
+                                        acc[nt][1]);
               }
             }
           }
@@ -401,7 +400,7 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
           const int n = nt * 8 + 2 * cq + v;
-          if (nt < ntn && n < it.ntok) emit(it, n, acc[nt][v], acc[nt][v + 2]);
+          if (nt < ntn && n < it.ntok) emit(it, n, (v ? acc[nt][0].y : acc[nt][0].x), (v ? acc[nt][1].y : acc[nt][1].x));
         }
     } else {
       // one piece of an item cut by warp shares.  Its pieces belong to the
@@ -421,8 +420,8 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
           for (int v = 0; v < 2; ++v) {
             const int n = nt * 8 + 2 * cq + v;
             if (nt < ntn && n < it.ntok) {
-              mine[n * 16 + g] = acc[nt][v];
-              mine[n * 16 + g + 8] = acc[nt][v + 2];
+              mine[n * 16 + g] = v ? acc[nt][0].y : acc[nt][0].x;
+              mine[n * 16 + g + 8] = v ? acc[nt][1].y : acc[nt][1].x;
             }
           }
         __syncwarp();
@@ -443,7 +442,8 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
           for (int v = 0; v < 2; ++v) {
             const int n = nt * 8 + 2 * cq + v;
             if (nt < ntn && n < it.ntok) {
-              float lo = acc[nt][v], hi = acc[nt][v + 2];
+              float lo = v ? acc[nt][0].y : acc[nt][0].x;
+              float hi = v ? acc[nt][1].y : acc[nt][1].x;
               for (int w = w_first + 1; w <= w_last; ++w) {
                 if (cut(w + 1) == cut(w)) continue;  // empty share: no piece
                 const float *src = p.partial + (size_t)w * kMmSlotFloats;
