@@ -20,9 +20,7 @@
 //               shorter tiles;
 //   last warp   weight producer: per four K groups (of 128) one bulk copy per
 //               blob tile of packed weights and one of scales (its own warp,
-//               so the weight ring runs ahead of the activations).
-// The copy engine's per-operation cost, not bytes, limits this kernel when
-// the copies are small, so both producers move few, large pieces.
+//               so the weight ring runs ahead of the activations);
 //   warp 1      MMA: allocates all 512 TMEM columns (two 256-column
 //               accumulator buffers), and one thread issues 4 tcgen05.mma
 //               (M=128, N=pairs rounded up to 16, K=16) per atom, then
@@ -34,8 +32,10 @@
 //               transposed through shared memory, stored.
 // Both operands are staged one 64-wide swizzle atom at a time in a ring of
 // three stages with one "full" barrier (dequant arrivals + activation bytes)
-// and one "empty" barrier (MMA commit) per stage; packed weights are six K
-// groups deep.
+// and one "empty" barrier (MMA commit) per stage; packed weights sit in two
+// stages of four K groups.  The copy engine's per-operation cost, not bytes,
+// limits this kernel when the copies are small, so both producers move few,
+// large pieces.
 // N = 256 matters: one M=128 MMA costs about the same issue time at N = 128
 // as at N = 256, so the wide tile nearly doubles tensor throughput.
 // Every wait is bounded; on a timeout the status word is set and the roles
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint64_t *pk_full = bars, *pk_empty = pk_full + kPkStages;
-  // full[s]: the 8 dequant warps' arrivals plus the activation TMA bytes;
+  // full[s]: the dequant warps' arrivals plus the activation TMA bytes;
   // empty[s]: the MMAs that read stage s have completed
   uint64_t *full = pk_empty + kPkStages, *empty = full + kStages;
   uint64_t *acc_full = empty + kStages, *acc_empty = acc_full + 2;
