@@ -50,6 +50,8 @@ def _load():
         lib.oracle_expert_bytes.argtypes = [i, i]
         lib.oracle_route.restype = i
         lib.oracle_route.argtypes = [P, i, i, P, P, i, i, P, P, P]
+        lib.oracle_route_sigmoid.restype = i
+        lib.oracle_route_sigmoid.argtypes = [P, i, i, P, P, P, ctypes.c_float, i, i, P, P, P]
         lib.oracle_expert_ffn.restype = i
         lib.oracle_expert_ffn.argtypes = [P, i, i, P, i, P, P, P, P]
         lib.oracle_forward_routed.restype = i
@@ -96,6 +98,25 @@ def route(x_bf16: np.ndarray, W: np.ndarray, bias, top_k: int):
                               _ptr(logits), _ptr(idx), _ptr(w))
     if st != OK:
         raise ValueError("oracle_route status %d" % st)
+    return logits, idx, w
+
+
+def route_sigmoid(x_bf16: np.ndarray, W: np.ndarray, bias, corr, scale: float, top_k: int):
+    """Sigmoid router with correction bias `corr` (fp32 [E] or None) and routed
+    scale.  Returns (logits fp32 [T][E], idx int32 [T][k], w fp32 [T][k])."""
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    b = _c(bias, np.float32)
+    c = _c(corr, np.float32)
+    T, H = x.shape
+    E = W.shape[0]
+    logits = np.zeros((T, E), np.float32)
+    idx = np.zeros((T, top_k), np.int32)
+    w = np.zeros((T, top_k), np.float32)
+    st = _load().oracle_route_sigmoid(_ptr(x), T, H, _ptr(W), _ptr(b), _ptr(c), float(scale), E,
+                                      top_k, _ptr(logits), _ptr(idx), _ptr(w))
+    if st != OK:
+        raise ValueError("oracle_route_sigmoid status %d" % st)
     return logits, idx, w
 
 

@@ -242,6 +242,46 @@ int oracle_route(const uint16_t *x, int T, int H, const float *Wr, const float *
   return ORC_OK;
 }
 
+// Sigmoid router with a correction bias and a routed scale (the "sigmoid
+// top-10 routing with a correction bias and a 2.5x routed scale" of
+// ro99/strata README, model notes under the model table).  Logits as in
+// oracle_route; score s_e = 1 / (1 + exp(-l_e)) evaluated in double and
+// rounded to fp32; selection key = s_e + corr[e] (fp32; corr may be null =
+// zeros); the k largest keys, lower index first among equal keys; weights =
+// s_e / (sum of the selected scores, added in selection order) * scale, fp32.
+int oracle_route_sigmoid(const uint16_t *x, int T, int H, const float *Wr, const float *bias,
+                         const float *corr, float scale, int E, int k, float *logits,
+                         int32_t *idx, float *w) {
+  if (T < 0 || H <= 0 || E <= 0 || k <= 0 || k > E) return ORC_BAD_ARG;
+  std::vector<float> l(E), sc(E), key(E);
+  std::vector<char> taken(E);
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += (double)bf16_value(x[(size_t)t * H + h]) * (double)Wr[(size_t)e * H + h];
+      if (bias) acc += (double)bias[e];
+      l[e] = (float)acc;
+      if (logits) logits[(size_t)t * E + e] = l[e];
+      sc[e] = (float)(1.0 / (1.0 + std::exp(-(double)l[e])));
+      key[e] = corr ? sc[e] + corr[e] : sc[e];
+    }
+    std::fill(taken.begin(), taken.end(), 0);
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e)
+        if (!taken[e] && (best < 0 || key[e] > key[best])) best = e;
+      taken[best] = 1;
+      idx[(size_t)t * k + j] = best;
+    }
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) sum = sum + sc[idx[(size_t)t * k + j]];
+    for (int j = 0; j < k; ++j)
+      w[(size_t)t * k + j] = sc[idx[(size_t)t * k + j]] / sum * scale;
+  }
+  return ORC_OK;
+}
+
 // One expert on n tokens given as fp32 activations.  Any of g, u, h may be
 // null; y is [n][H].
 int oracle_expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,

@@ -345,3 +345,59 @@ def test_wide_zipf_share():
     _, idx, _ = oracle.route(x, W, b, cfg.top_k)
     share = np.mean(ranks[idx.reshape(-1)] <= 64)
     assert 0.78 <= share <= 0.82, share
+
+
+# ------------------------------------------------------------ sigmoid routing
+# (sigmoid top-k with a correction bias and a routed scale)
+
+def test_route_sigmoid_hand_case():
+    # x = 0, so every logit is its bias: 0 -> score exactly 0.5.  The
+    # correction bias alone decides the selection; the weights are
+    # 0.5 / (0.5 + 0.5) * 2.5 = 1.25 exactly.
+    E, H, k = 4, 64, 2
+    x = np.zeros((1, H), np.uint16)
+    W = np.ones((E, H), np.float32)
+    corr = np.array([0.0, 0.25, -0.25, 0.125], np.float32)
+    logits, idx, w = oracle.route_sigmoid(x, W, np.zeros(E, np.float32), corr, 2.5, k)
+    assert logits.tolist() == [[0.0] * E]
+    assert idx.tolist() == [[1, 3]]
+    assert w.tolist() == [[1.25, 1.25]]
+    # a large negative logit has a tiny score: a big correction still selects
+    # it (keys 0.5, 0.75, 0.25, 0.625), but its share of the weight is tiny
+    bias = np.array([0.0, -30.0, 0.0, 0.0], np.float32)
+    corr2 = np.array([0.0, 0.75, -0.25, 0.125], np.float32)
+    _, idx, w = oracle.route_sigmoid(x, W, bias, corr2, 1.0, k)
+    assert idx.tolist() == [[1, 3]]
+    tiny = 1.0 / (1.0 + np.exp(30.0))
+    assert w[0, 0] == pytest.approx(tiny / (tiny + 0.5), rel=1e-5)
+    assert w[0, 1] == pytest.approx(0.5 / (tiny + 0.5), rel=1e-6)
+
+
+def test_route_sigmoid_without_correction_selects_like_softmax():
+    # the sigmoid is increasing, so without a correction bias the selection is
+    # the top-k of the logits, as in the softmax router
+    cfg = synth.custom_config("sg", 256, 128, 16, 4)
+    x = synth.make_x(cfg, 12, seed=5)
+    W, _ = synth.make_router(cfg, seed=5)
+    _, idx_s, _ = oracle.route(x, W, None, 4)
+    logits, idx_g, w_g = oracle.route_sigmoid(x, W, None, None, 1.0, 4)
+    assert idx_g.tolist() == idx_s.tolist()
+    sc = 1.0 / (1.0 + np.exp(-logits.astype(np.float64)))
+    sel = np.take_along_axis(sc, idx_g.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w_g, sel / sel.sum(axis=1, keepdims=True), rtol=2e-6)
+    np.testing.assert_allclose(w_g.sum(axis=1), 1.0, rtol=2e-6)
+
+
+def test_route_sigmoid_subset_topk_of_keys():
+    # selection = the subset with the largest sum of keys (score + correction)
+    E, k, H = 7, 3, 128
+    rng = np.random.default_rng(11)
+    x = synth.f32_to_bf16_bits(rng.standard_normal((6, H)).astype(np.float32))
+    W = (rng.standard_normal((E, H)) / np.sqrt(H)).astype(np.float32)
+    corr = (rng.standard_normal(E) * 0.2).astype(np.float32)
+    logits, idx, w = oracle.route_sigmoid(x, W, None, corr, 2.5, k)
+    for t in range(x.shape[0]):
+        sc = (1.0 / (1.0 + np.exp(-logits[t].astype(np.float64)))).astype(np.float32)
+        key = (sc + corr).astype(np.float32)
+        assert idx[t].tolist() == naive.topk_by_subsets(key, k)
+        assert float(w[t].sum()) == pytest.approx(2.5, rel=1e-6)
