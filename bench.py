@@ -67,7 +67,9 @@ def parse():
 def workload_desc(cfg, T):
     return {"workload": "%s, %d tokens" % (cfg.description, T), "hidden": cfg.hidden,
             "inter": cfg.inter, "n_experts": cfg.n_experts, "top_k": cfg.top_k,
-            "n_shared": cfg.n_shared, "n_slots": cfg.n_slots, "tokens": T}
+            "n_shared": cfg.n_shared, "n_slots": cfg.n_slots, "tokens": T,
+            "routing": cfg.routing if cfg.routing == "softmax" else
+            "%s (correction bias, routed scale %g)" % (cfg.routing, cfg.routed_scale)}
 
 
 def dist_env():
@@ -154,11 +156,14 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- oracle leg
-def oracle_step_time(cfg, blobs, W, b, x_bits):
+def oracle_step_time(cfg, blobs, W, b, x_bits, corr=None):
     import oracle
     E, S = cfg.n_experts, cfg.n_shared
     t0 = time.perf_counter()
-    _, idx, w = oracle.route(x_bits, W, b, cfg.top_k)
+    if cfg.routing == "sigmoid":
+        _, idx, w = oracle.route_sigmoid(x_bits, W, b, corr, cfg.routed_scale, cfg.top_k)
+    else:
+        _, idx, w = oracle.route(x_bits, W, b, cfg.top_k)
     st, _ = oracle.forward_routed(x_bits, cfg.hidden, cfg.inter, E, cfg.top_k, np.arange(E),
                                   [blobs[e] for e in range(E)], [blobs[E + i] for i in range(S)],
                                   idx, w)
@@ -172,14 +177,14 @@ def cpu_sample_tokens(cfg, T):
     return T if T <= 16 else 8
 
 
-def run_cpu_baseline(cfg, blobs, W, b, T, seed, budget_s=20.0, max_steps=8):
+def run_cpu_baseline(cfg, blobs, W, b, T, seed, budget_s=20.0, max_steps=8, corr=None):
     n = cpu_sample_tokens(cfg, T)
     total, toks, steps = 0.0, 0, 0
     while steps < max_steps and (total < budget_s or steps == 0):
         x = synth.make_x(cfg, T, seed, step=10_000 + steps)
         if n < T:
             x = x[np.linspace(0, T - 1, n).astype(int)]
-        total += oracle_step_time(cfg, blobs, W, b, x)
+        total += oracle_step_time(cfg, blobs, W, b, x, corr)
         toks += n
         steps += 1
         if total / steps * (steps + 1) > budget_s * 1.5:
@@ -198,18 +203,19 @@ def reference_arm(args):
     T = args.tokens
     blobs = synth.make_all_blobs(cfg, args.seed)
     W, b = synth.make_router(cfg, args.seed)
+    corr = synth.make_correction_bias(cfg, args.seed) if cfg.routing == "sigmoid" else None
     n = cpu_sample_tokens(cfg, T)
     per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup if args.warmup < 3 else 1):
         x = synth.make_x(cfg, T, args.seed, step=20_000 + i)[:n]
-        oracle_step_time(cfg, blobs, W, b, x)
+        oracle_step_time(cfg, blobs, W, b, x, corr)
     times = []
     t_start = time.perf_counter()
     for s in range(args.steps):
         x = synth.make_x(cfg, T, args.seed, step=s)
         if n < T:
             x = x[np.linspace(0, T - 1, n).astype(int)]
-        times.append(oracle_step_time(cfg, blobs, W, b, x))
+        times.append(oracle_step_time(cfg, blobs, W, b, x, corr))
         if time.perf_counter() - t_start > per_step_budget * args.steps:
             break
     k = len(times)
@@ -282,6 +288,11 @@ def main():
     paged = cfg.n_slots < E
     layer = binding.StrataMoE(cfg.hidden, cfg.inter, E, cfg.top_k, S, cfg.n_slots)
     layer.set_router(W_dev, b_dev)
+    corr = None
+    if cfg.routing == "sigmoid":
+        corr = synth.make_correction_bias(cfg, args.seed)
+        corr_dev = torch.from_numpy(corr).cuda()
+        layer.set_routing(binding.ROUTE_SIGMOID, corr_dev, cfg.routed_scale)
     B_e = synth.expert_bytes(cfg.hidden, cfg.inter)
     if paged:
         dev_shared = torch.from_numpy(blobs[E:]).cuda()
@@ -469,7 +480,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = run_cpu_baseline(cfg, blobs, W, b, T, args.seed)
+        cpu = run_cpu_baseline(cfg, blobs, W, b, T, args.seed, corr=corr)
 
     if rank == 0:
         line = {

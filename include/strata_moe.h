@@ -107,6 +107,23 @@ size_t strata_moe_expert_bytes(int hidden, int inter);
  * aligned.  Errors: INVALID_ARG. */
 strata_status strata_moe_set_router(strata_moe *h, const float *W_dev, const float *bias_dev);
 
+/* Routing function (default: softmax).
+ * STRATA_ROUTE_SOFTMAX: the description at the top of this file; corr_dev
+ *   must be NULL and routed_scale 1.
+ * STRATA_ROUTE_SIGMOID: the "sigmoid top-k routing with a correction bias and
+ *   a routed scale" of ro99/strata README (model notes under the model
+ *   table): score[e] = 1 / (1 + exp(-logit[e])) (evaluated in double, rounded
+ *   to fp32); the top_k experts by score[e] + corr[e] (fp32; ties: lower id;
+ *   corr_dev: device fp32 [n_experts] or NULL for zeros) in descending order;
+ *   weights w[j] = score[j] / (sum of the selected scores, added in that
+ *   order) * routed_scale.  Shared experts keep weight 1.
+ * corr_dev is read by later calls (caller-owned, must stay valid).
+ * Errors: INVALID_ARG (unknown mode, routed_scale not positive and finite,
+ * misaligned corr_dev, or corr/scale given with softmax). */
+enum { STRATA_ROUTE_SOFTMAX = 0, STRATA_ROUTE_SIGMOID = 1 };
+strata_status strata_moe_set_routing(strata_moe *h, int mode, const float *corr_dev,
+                                     float routed_scale);
+
 /* Bind shared expert i (0 <= i < n_shared) to the blob at device_ptr
  * (256-byte aligned, strata_moe_expert_bytes long).  Errors: INVALID_ARG. */
 strata_status strata_moe_bind_shared(strata_moe *h, int i, const void *device_ptr);

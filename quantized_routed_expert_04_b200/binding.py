@@ -56,6 +56,7 @@ def load_library():
             "strata_moe_expert_bytes": (Z, [I, I]),
             "strata_moe_set_router": (I, [P, P, P]),
             "strata_moe_bind_shared": (I, [P, I, P]),
+            "strata_moe_set_routing": (I, [P, I, P, ctypes.c_float]),
             "strata_moe_bind_slot": (I, [P, I, I, P]),
             "strata_moe_slot_expert": (I, [P, I]),
             "strata_moe_reserve": (I, [P, I]),
@@ -124,6 +125,14 @@ def strata_moe_expert_bytes(hidden, inter):
 
 def strata_moe_set_router(h, W, bias=None):
     _check(_load().strata_moe_set_router(h, _addr(W), _addr(bias)), "strata_moe_set_router")
+
+
+ROUTE_SOFTMAX, ROUTE_SIGMOID = 0, 1
+
+
+def strata_moe_set_routing(h, mode, corr=None, routed_scale=1.0):
+    _check(_load().strata_moe_set_routing(h, int(mode), _addr(corr), float(routed_scale)),
+           "strata_moe_set_routing")
 
 
 def strata_moe_bind_shared(h, i, blob):
@@ -274,6 +283,9 @@ class StrataMoE:
 
     def set_router(self, W, bias=None):
         strata_moe_set_router(self.h, W, bias)
+
+    def set_routing(self, mode, corr=None, routed_scale=1.0):
+        strata_moe_set_routing(self.h, mode, corr, routed_scale)
 
     def bind_shared(self, i, blob):
         strata_moe_bind_shared(self.h, i, blob)

@@ -11,7 +11,15 @@ namespace strata {
 // ---- routing (route.cu)
 __global__ void router_gemm_kernel(const __nv_bfloat16 *x, const float *W, const float *bias,
                                    int T, int H, int E, float *logits);
-__global__ void topk_kernel(const float *logits, int T, int E, int k, int32_t *idx, float *w);
+// Routing function: softmax (sigmoid = 0) or sigmoid scores with an optional
+// correction bias on the selection key and a routed scale on the weights.
+struct RouteMode {
+  int sigmoid;
+  const float *corr;  // [E] or null
+  float scale;
+};
+__global__ void topk_kernel(const float *logits, int T, int E, int k, RouteMode mode,
+                            int32_t *idx, float *w);
 __global__ void pack_x_kernel(const __nv_bfloat16 *x, int n8, __half *x16);
 __global__ void bucket_count_kernel(const int32_t *idx, int T, int k, int E, int *cnt,
                                     int *status);
@@ -29,6 +37,7 @@ struct SmallRouteParams {
   __half *x16;
   int *counter;    // last-block counter, zero between launches
   int *status;
+  RouteMode mode;
 };
 template <bool kRoute, bool kBucket>
 __global__ void route_small_kernel(SmallRouteParams p);

@@ -116,59 +116,86 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
 }
 
 // ---------------------------------------------------------------- top-k
-// One warp per token.  Lane l holds logits l, l+32, ...; k rounds of a warp
-// arg-max (larger logit wins, equal logits: lower id wins).
-__global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int k,
-                            int32_t *__restrict__ idx, float *__restrict__ w) {
-  grid_dependency_wait();
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
+// One warp per token.  Lane l holds experts l, l+32, ...; k rounds of a warp
+// arg-max of the selection key (larger wins, equal keys: lower id wins).
+// Softmax routing: key = logit, weights = exp(l_j - l_0) / sum_j (the
+// renormalised softmax of the selected experts).  Sigmoid routing: score =
+// 1 / (1 + exp(-l)) in double rounded to fp32, key = score + correction,
+// weights = score_j / (sum of the selected scores in selection order) *
+// routed scale.  Lane j (< k) returns selection j in sel_e / sel_w.
+__device__ void select_topk_warp(const float *__restrict__ logit_row, int E, int k,
+                                 const RouteMode &mode, int lane, int &sel_e, float &sel_w) {
   constexpr int kPer = kMaxExperts / 32;
-  float v[kPer];
+  float key[kPer], val[kPer];   // val: logit (softmax) or score (sigmoid)
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? logits[(size_t)t * E + e] : -INFINITY;
+    const float l = e < E ? __ldcg(logit_row + e) : -INFINITY;
+    if (mode.sigmoid && e < E) {
+      val[i] = (float)(1.0 / (1.0 + exp(-(double)l)));
+      key[i] = mode.corr ? __fadd_rn(val[i], mode.corr[e]) : val[i];
+    } else {
+      val[i] = l;
+      key[i] = l;
+    }
   }
   unsigned taken = 0;
-  float sel_l[kMaxTopK];
-  int sel_e[kMaxTopK];
+  float v0 = 0.0f, z = 0.0f, my_v = 0.0f;
+  int my_e = 0;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
+    float bk = -INFINITY;
     int be = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
-        bv = v[i];
+      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || key[i] > bk)) {
+        bk = key[i];
         be = e;
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-        bv = ov;
+      if (oe != 0x7fffffff && (be == 0x7fffffff || ok > bk || (ok == bk && oe < be))) {
+        bk = ok;
         be = oe;
       }
     }
+    // the winner's logit or score, from the lane that holds it
+    float mine = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (i == (be >> 5)) mine = val[i];
+    const float bv = __shfl_sync(0xffffffffu, mine, be & 31);
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    sel_l[j] = bv;
-    sel_e[j] = be;
+    if (mode.sigmoid) {
+      z = __fadd_rn(z, bv);
+    } else {
+      if (j == 0) v0 = bv;
+      z += expf(bv - v0);
+    }
+    if (lane == j) {  // lane j keeps selection j (k <= 32)
+      my_v = bv;
+      my_e = be;
+    }
   }
-  if (lane == 0) {
-    float z = 0.0f;
-    float p[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-      p[j] = expf(sel_l[j] - sel_l[0]);
-      z += p[j];
-    }
-    for (int j = 0; j < k; ++j) {
-      idx[(size_t)t * k + j] = sel_e[j];
-      w[(size_t)t * k + j] = p[j] / z;
-    }
+  sel_e = my_e;
+  sel_w = mode.sigmoid ? __fmul_rn(__fdiv_rn(my_v, z), mode.scale) : expf(my_v - v0) / z;
+}
+
+__global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int k, RouteMode mode,
+                            int32_t *__restrict__ idx, float *__restrict__ w) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int e;
+  float wt;
+  select_topk_warp(logits + (size_t)t * E, E, k, mode, lane, e, wt);
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = e;
+    w[(size_t)t * k + lane] = wt;
   }
 }
 
@@ -346,51 +373,16 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
 // buckets the pairs.  The last block resets the counter for the next launch.
 namespace {
 
-__device__ void topk_token_warp(const float *__restrict__ logit_row, int E, int k, int lane,
-                                int32_t *idx_out, float *w_out, int *s_idx) {
-  constexpr int kPer = kMaxExperts / 32;
-  float v[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? __ldcg(logit_row + e) : -INFINITY;
-  }
-  unsigned taken = 0;
-  float l0 = 0.0f, z = 0.0f, my_l = 0.0f;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
-        bv = v[i];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (j == 0) l0 = bv;
-    const float pj = expf(bv - l0);
-    z += pj;
-    if (lane == j) {  // lane j keeps selection j (k <= 32)
-      my_l = bv;
-      my_e = be;
-    }
-  }
+__device__ void topk_token_warp(const float *__restrict__ logit_row, int E, int k,
+                                const RouteMode &mode, int lane, int32_t *idx_out, float *w_out,
+                                int *s_idx) {
+  int e;
+  float wt;
+  select_topk_warp(logit_row, E, k, mode, lane, e, wt);
   if (lane < k) {
-    idx_out[lane] = my_e;
-    w_out[lane] = expf(my_l - l0) / z;
-    if (s_idx) s_idx[lane] = my_e;
+    idx_out[lane] = e;
+    w_out[lane] = wt;
+    if (s_idx) s_idx[lane] = e;
   }
 }
 
@@ -555,7 +547,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteParams p) {
   }
   if (kRoute) {
     for (int t = warp; t < T; t += 8)
-      topk_token_warp(p.logits + (size_t)t * E, E, k, lane, p.idx + (size_t)t * k,
+      topk_token_warp(p.logits + (size_t)t * E, E, k, p.mode, lane, p.idx + (size_t)t * k,
                       p.w + (size_t)t * k, kBucket ? s_idx + t * k : nullptr);
   } else {
     for (int q = tid; q < T * k; q += blockDim.x) s_idx[q] = p.idx[q];

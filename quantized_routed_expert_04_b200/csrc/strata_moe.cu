@@ -42,6 +42,7 @@ struct strata_moe {
   std::vector<const void *> shared_ptr;    // per shared expert
   const float *router_W = nullptr;
   const float *router_b = nullptr;
+  RouteMode mode{0, nullptr, 1.0f};
 
   // workspace
   int cap_tokens = 0;
@@ -375,6 +376,7 @@ SmallRouteParams small_params(strata_moe *h, const void *x, int T, float *logits
   p.x16 = h->x16;
   p.counter = h->counter;
   p.status = h->status;
+  p.mode = h->mode;
   return p;
 }
 
@@ -397,7 +399,7 @@ strata_status run_router(strata_moe *h, const void *x, int T, float *logits, int
              stream, false, xb, h->router_W, h->router_b, T, h->H, h->E, logits);
   if (e == cudaSuccess)
     e = launch(h, PH_TOPK, topk_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, true, logits, T,
-               h->E, h->k, idx, w);
+               h->E, h->k, h->mode, idx, w);
   return cuda_status(e);
 }
 
@@ -483,6 +485,20 @@ strata_status strata_moe_set_router(strata_moe *h, const float *W_dev, const flo
     return STRATA_ERR_INVALID_ARG;
   h->router_W = W_dev;
   h->router_b = bias_dev;
+  return STRATA_OK;
+}
+
+strata_status strata_moe_set_routing(strata_moe *h, int mode, const float *corr_dev,
+                                     float routed_scale) {
+  if (!h || (mode != STRATA_ROUTE_SOFTMAX && mode != STRATA_ROUTE_SIGMOID))
+    return STRATA_ERR_INVALID_ARG;
+  if (!(routed_scale > 0.0f) || !(routed_scale < 3.0e38f)) return STRATA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(corr_dev) & 3) return STRATA_ERR_INVALID_ARG;
+  if (mode == STRATA_ROUTE_SOFTMAX && (corr_dev || routed_scale != 1.0f))
+    return STRATA_ERR_INVALID_ARG;
+  h->mode.sigmoid = mode == STRATA_ROUTE_SIGMOID;
+  h->mode.corr = corr_dev;
+  h->mode.scale = routed_scale;
   return STRATA_OK;
 }
 

@@ -60,6 +60,8 @@ class LayerConfig:
     zipf_s: float = 0.0         # Zipf exponent of the bias
     zipf_beta: float = 1.0      # multiplier on the Zipf log-pmf
     description: str = ""
+    routing: str = "softmax"    # "softmax" | "sigmoid" (with correction bias)
+    routed_scale: float = 1.0
 
 
 # beta for the wide layer: the value at which ~80% of the routed hits of the
@@ -91,6 +93,13 @@ CONFIGS = {
         zipf_beta=1.0,
         description="prefill: hidden 4096, inter 2048, 256 experts top-8 + 1 "
                     "shared, 8192 tokens, Zipf(0.8) router bias"),
+    # the wide-expert layer's shapes, all experts resident, routed like the
+    # pages' sigmoid models: sigmoid scores, a per-expert correction bias on
+    # the selection, a 2.5x routed scale
+    "sigmoid": LayerConfig(
+        "sigmoid", 4096, 1024, 256, 10, 0, 256, (1, 4), routing="sigmoid", routed_scale=2.5,
+        description="sigmoid-routed decode: hidden 4096, inter 1024, 256 experts top-10, "
+                    "correction bias ~N(0, 0.05^2), routed scale 2.5"),
     # the prefill layer's shapes with 32 experts and 2048 tokens: small enough
     # (about 0.5 GB of blobs) for profiler captures and quick parity runs
     "prefill_small": LayerConfig(
@@ -214,6 +223,7 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 # seeded draws; every stream is keyed by (seed, purpose, index)
 
 _STREAM_X, _STREAM_ROUTER, _STREAM_BIAS, _STREAM_EXPERT, _STREAM_SLOTS, _STREAM_RANK = range(6)
+_STREAM_CORR = 6
 
 
 def _rng(seed: int, stream: int, index: int = 0) -> np.random.Generator:
@@ -248,6 +258,13 @@ def make_router(cfg: LayerConfig, seed: int = 0):
     else:
         raise ValueError(cfg.bias)
     return W, b
+
+
+def make_correction_bias(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
+    """Per-expert correction bias of the sigmoid router, fp32 [E] ~ N(0, 0.05^2)
+    (same order as the scores' spread near 0.5, so it reorders experts)."""
+    r = _rng(seed, _STREAM_CORR)
+    return (r.standard_normal(cfg.n_experts) * 0.05).astype(np.float32)
 
 
 def make_expert_blob(cfg: LayerConfig, expert: int, seed: int = 0) -> np.ndarray:
