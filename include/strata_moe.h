@@ -51,7 +51,10 @@
  * route call takes a snapshot of the slot table when it is enqueued, so a
  * later bind affects only later calls.  Rebinding a slot whose blob is still
  * read by enqueued work is the caller's hazard, as for any stream-ordered
- * buffer.
+ * buffer.  A handle (and an arena) must not be used from several host threads
+ * at once.  A route or forward call with more tokens than the workspace holds
+ * grows it first (cudaMalloc/cudaFree and a device synchronisation); use
+ * strata_moe_reserve to do that up front.
  *
  * Errors: a call that finds a problem on the host returns a status and
  * enqueues nothing.  Problems only the device can see (a routed expert with
