@@ -26,9 +26,9 @@
 //               (M=128, N=pairs rounded up to 16, K=16) per atom, then
 //               commits to the stage barriers and, at the end of a tile, to
 //               the accumulator;
-//   warps 2-5   dequant: int4 -> exact f16 integers -> times the fp16 scale
+//   warps 2-9   dequant: int4 -> exact f16 integers -> times the fp16 scale
 //               (one f16 rounding) -> the K-major 128-byte-swizzled A layout;
-//   warps 6-9   epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
+//   warps 10-13 epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
 //               transposed through shared memory, stored.
 // Both operands are staged one 64-wide swizzle atom at a time in a ring of
 // three stages with one "full" barrier (dequant arrivals + activation bytes)
@@ -54,7 +54,7 @@ constexpr int kTcN = 256;          // pairs per tile (max MMA N used)
 constexpr int kPkStages = 2;       // packed-weight stages (four K groups each)
 constexpr int kPkGroups = 4;
 constexpr int kStages = 3;         // operand stages: one 64-wide atom of A and of B each
-constexpr int kDqWarps = 4;
+constexpr int kDqWarps = 8;
 constexpr int kDqRows = kTcM / kDqWarps;    // weight rows per dequant warp
 static_assert(kDqRows % 8 == 0, "dequant warps cover whole 8-row groups");
 constexpr int kPkWarp = 2 + kDqWarps + 4;   // the last warp
