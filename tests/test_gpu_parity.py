@@ -113,6 +113,23 @@ def test_forward_ragged_token_groups(T):
     lay.close()
 
 
+@pytest.mark.parametrize("E,k,S,T", [
+    (8, 8, 0, 4),     # top_k = n_experts: every expert takes every token
+    (1, 1, 1, 5),     # one routed expert (weight 1) plus a shared one
+    (8, 2, 0, 65),    # one token past the small-batch path: tensor-core path
+    (8, 2, 1, 64),    # the largest small batch
+])
+def test_forward_degenerate_shapes(E, k, S, T):
+    cfg = synth.custom_config("deg", 256, 256, E, k, n_shared=S, tokens=(T,))
+    lay = GpuLayer(cfg)
+    x = synth.make_x(cfg, T, step=4)
+    st, out = lay.forward(x)
+    assert int(st[0]) == 0
+    ref, _, _ = oracle_reference(cfg, lay.blobs, lay.W, lay.b, x)
+    assert_within_tolerance(out, ref, "E=%d k=%d S=%d T=%d" % (E, k, S, T))
+    lay.close()
+
+
 def test_forward_prefill_sampled_tokens():
     """Prefill size (8192 tokens, 256 experts + 1 shared), in the launch
     configuration the benchmark times; 12 sampled tokens checked against the
