@@ -74,3 +74,25 @@ def test_library_is_sm100a_only():
         text = open(os.path.join(build.BUILD, f)).read()
         targets = set(re.findall(r"for '(sm_\w+)'", text))
         assert targets <= {"sm_100a"}, (f, targets)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback: without the built library the binding raises
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "libstrata_moe.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.load_library()
+
+
+def test_product_code_never_uses_the_oracle():
+    # the oracle is test infrastructure: the package, its C sources and the
+    # header must not import it, load its library or call its functions
+    use = re.compile(r"(import\s+oracle|from\s+oracle|liboracle|oracle_\w+\s*\(|oracle\.\w+\()")
+    offenders = []
+    for base, _, files in os.walk(os.path.join(ROOT, "quantized_routed_expert_04_b200")):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                if use.search(open(os.path.join(base, f)).read()):
+                    offenders.append(os.path.relpath(os.path.join(base, f), ROOT))
+    assert not offenders, offenders
+    assert not use.search(open(os.path.join(ROOT, "include", "strata_moe.h")).read())
