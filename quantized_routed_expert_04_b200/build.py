@@ -10,6 +10,7 @@ _build/ptxas_<name>.log.
 from __future__ import annotations
 
 import concurrent.futures
+import fcntl
 import glob
 import os
 import subprocess
@@ -58,9 +59,23 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile and link if a source is newer than the library.  Several
+    processes may call this at once (one per GPU): a file lock lets one build
+    while the others wait, then find the library up to date."""
     if not force and up_to_date():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        try:
+            if not force and up_to_date():
+                return LIB
+            return _build_locked(verbose)
+        finally:
+            fcntl.flock(lock, fcntl.LOCK_UN)
+
+
+def _build_locked(verbose: bool) -> str:
     srcs = _sources()
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(_compile, srcs))
