@@ -6,7 +6,7 @@ import numpy as np
 
 from quantized_routed_expert_04_b200 import synth
 
-# BASELINE tolerance of the layer output (errors computed in fp32/fp64):
+# Tolerance of the layer output (errors computed in fp32/fp64):
 #   max |out - ref| <= 2e-2 * max |ref|  and  sum |out - ref| / sum |ref| <= 2e-3
 TOL_MAX = 2e-2
 TOL_MEAN = 2e-3
