@@ -9,11 +9,12 @@
  *      probabilities divided by their sum -> weights w[t][j];
  *   2. finds each selected expert's weights through an expert-id -> slot
  *      table over a fixed-size arena of expert blobs (ro99/strata README,
- *      "Residency": routed experts leased into VRAM through an LRU cache;
+ *      "Residency": the routed experts of a step are kept in GPU memory
+ *      under LRU replacement;
  *      "Strata on a Mac", "What you need": an arena of the most-used experts
  *      with the rest read as tokens need them);
- *   3. runs the expert FFN on 4-bit block-quantised weights ("INT4 ...
- *      W4A16 execution", ro99/strata README, model table):
+ *   3. runs the expert FFN on 4-bit block-quantised weights with 16-bit
+ *      activations (the int4 format of ro99/strata README, model table):
  *      h = silu(Wg x) * (Wu x), y = Wd h, silu(z) = z / (1 + exp(-z));
  *   4. writes out[t] = sum_j w[t][j] * y[t][j] + sum_s y_shared[t][s].
  * The output does not depend on which slot holds which expert, nor on
@@ -113,9 +114,9 @@ strata_status strata_moe_set_router(strata_moe *h, const float *W_dev, const flo
 /* Routing function (default: softmax).
  * STRATA_ROUTE_SOFTMAX: the description at the top of this file; corr_dev
  *   must be NULL and routed_scale 1.
- * STRATA_ROUTE_SIGMOID: the "sigmoid top-k routing with a correction bias and
- *   a routed scale" of ro99/strata README (model notes under the model
- *   table): score[e] = 1 / (1 + exp(-logit[e])) (evaluated in double, rounded
+ * STRATA_ROUTE_SIGMOID: sigmoid scores, a per-expert correction bias on the
+ *   selection and a scale on the routed weights, as ro99/strata README
+ *   describes for some models (notes under the model table): score[e] = 1 / (1 + exp(-logit[e])) (evaluated in double, rounded
  *   to fp32); the top_k experts by score[e] + corr[e] (fp32; ties: lower id;
  *   corr_dev: device fp32 [n_experts] or NULL for zeros) in descending order;
  *   weights w[j] = score[j] / (sum of the selected scores, added in that
@@ -190,9 +191,10 @@ strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches
 
 /* ---- Expert arena: least-recently-used residency of routed experts.
  * The paging layer in front of the slot table (ro99/strata README,
- * "Residency": routed experts leased into VRAM per step through an LRU cache
- * from pinned host memory; "Strata on a Mac", "What you need": a fixed arena
- * of experts, the rest read in as tokens need them).  An arena owns the
+ * "Residency": the routed experts of each step kept in GPU memory under LRU
+ * replacement and copied in from pinned host memory; "Strata on a Mac",
+ * "What you need": a fixed arena of experts, the rest read in as tokens need
+ * them).  An arena owns the
  * layer's slot table: it binds slot s to device memory
  * arena_dev + s * strata_moe_expert_bytes(hidden, inter).  Results do not
  * depend on the arena's choices, only copy traffic does. */

@@ -8,7 +8,7 @@
 // beyond what the definition states.
 //
 // What it computes, and the passages it follows:
-//  * Routing: "route each token to its top-k experts" with an fp32 router
+//  * Routing: each token goes to its k best experts by an fp32 router
 //    GEMV, softmax, top-k with lowest-index tie-break and renormalisation
 //    (the layer statement this library implements; the fused router dispatch
 //    of Strata "docs/MAC.md", section "Switches", two opt-ins paragraph).
@@ -17,10 +17,12 @@
 //    in double, the sum is rounded once to an fp32 logit; top-k compares the
 //    fp32 logits; softmax is fp32 with max subtraction over all experts; the
 //    selected probabilities are divided by their sum.
-//  * Expert lookup through a slot table ("routed experts ... leased into VRAM
-//    per decode step through an LRU cache", ro99/strata README, "Residency").
-//  * Expert FFN on W4A16 weights ("INT4 ... W4A16 execution", ro99/strata
-//    README, model table), read from the tiled blob format described at
+//  * Expert lookup through a slot table (the engine keeps the routed experts
+//    of each decode step in GPU memory under LRU replacement: ro99/strata
+//    README, "Residency").
+//  * Expert FFN on 4-bit weights with 16-bit activations (the int4 weight
+//    format of ro99/strata README, model table), read from the tiled blob
+//    format described at
 //    place_of(): w = float(fp16 scale) * q, exact in fp32; gate and
 //    up dot products in fp32 in ascending K; h = silu(g) * u with
 //    silu(z) = z / (1 + exp(-z)) in fp32; down projection in fp32 ascending K.

@@ -2,8 +2,9 @@
 // decides which experts occupy the layer's slots and copies missing blobs in
 // from a host pool.
 //
-// What it follows: ro99/strata README, "Residency" (routed experts leased
-// into VRAM per decode step through an LRU cache, from pinned host memory);
+// What it follows: ro99/strata README, "Residency" (the routed experts of
+// each decode step are kept in GPU memory under LRU replacement and copied
+// in from pinned host memory);
 // "Strata on a Mac", "What you need" (a fixed arena of the most-used experts,
 // the rest read in as tokens need them).  The layer's output does not depend
 // on which slot holds an expert, so the policy only changes copy traffic,

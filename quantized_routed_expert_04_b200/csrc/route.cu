@@ -1,7 +1,8 @@
 // Routing, bucketing, activation packing and the weighted combine.
 //
-// Router ("the router GEMV and moe_route", "Strata on a Mac", "Switches",
-// two opt-ins paragraph): logit = x . Wr[e] + b[e] with x bf16 and Wr fp32;
+// Router (the fused router dispatch that "Strata on a Mac", "Switches",
+// describes among its two opt-ins): logit = x . Wr[e] + b[e] with x bf16 and
+// Wr fp32;
 // every product is exact in double and the sum is kept in double, then
 // rounded once to fp32.  Top-k takes the largest fp32 logits, lower expert id
 // first among equal ones; the weights are the softmax probabilities of the
