@@ -25,6 +25,7 @@ _SRC = os.path.join(_HERE, "oracle.cpp")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 OK, BAD_ARG, NOT_BOUND, SLOT_CONFLICT = 0, 1, 2, 3
+FORMATS = {"int4": 0, "nvfp4": 1}   # weight formats of an expert blob
 
 _lib = None
 
@@ -54,6 +55,12 @@ def _load():
         lib.oracle_route_sigmoid.argtypes = [P, i, i, P, P, P, ctypes.c_float, i, i, P, P, P]
         lib.oracle_expert_ffn.restype = i
         lib.oracle_expert_ffn.argtypes = [P, i, i, P, i, P, P, P, P]
+        lib.oracle_expert_bytes_fmt.restype = ctypes.c_size_t
+        lib.oracle_expert_bytes_fmt.argtypes = [i, i, i]
+        lib.oracle_expert_ffn_fmt.restype = i
+        lib.oracle_expert_ffn_fmt.argtypes = [P, i, i, i, P, i, P, P, P, P]
+        lib.oracle_forward_routed_fmt.restype = i
+        lib.oracle_forward_routed_fmt.argtypes = [P, i, i, i, i, i, i, P, P, i, P, P, P, P, i]
         lib.oracle_forward_routed.restype = i
         lib.oracle_forward_routed.argtypes = [P, i, i, i, i, i, i, P, P, i, P, P, P, P]
         lib.oracle_forward.restype = i
@@ -77,8 +84,8 @@ def _ptr_array(blobs):
     return arr
 
 
-def expert_bytes(hidden: int, inter: int) -> int:
-    return int(_load().oracle_expert_bytes(hidden, inter))
+def expert_bytes(hidden: int, inter: int, fmt: str = "int4") -> int:
+    return int(_load().oracle_expert_bytes_fmt(hidden, inter, FORMATS[fmt]))
 
 
 def route(x_bf16: np.ndarray, W: np.ndarray, bias, top_k: int):
@@ -120,7 +127,7 @@ def route_sigmoid(x_bf16: np.ndarray, W: np.ndarray, bias, corr, scale: float, t
     return logits, idx, w
 
 
-def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray):
+def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray, fmt: str = "int4"):
     """One expert on fp32 activations x [n][H].  Returns (g, u, h, y)."""
     blob = _c(blob, np.uint8)
     x = _c(x, np.float32)
@@ -129,15 +136,15 @@ def expert_ffn(blob: np.ndarray, hidden: int, inter: int, x: np.ndarray):
     u = np.zeros((n, inter), np.float32)
     h = np.zeros((n, inter), np.float32)
     y = np.zeros((n, hidden), np.float32)
-    st = _load().oracle_expert_ffn(_ptr(blob), hidden, inter, _ptr(x), n,
-                                   _ptr(g), _ptr(u), _ptr(h), _ptr(y))
+    st = _load().oracle_expert_ffn_fmt(_ptr(blob), hidden, inter, FORMATS[fmt], _ptr(x), n,
+                                       _ptr(g), _ptr(u), _ptr(h), _ptr(y))
     if st != OK:
         raise ValueError("oracle_expert_ffn status %d" % st)
     return g, u, h, y
 
 
 def forward_routed(x_bf16, hidden, inter, n_experts, top_k, slot_expert, slot_blobs,
-                   shared_blobs, idx, w):
+                   shared_blobs, idx, w, fmt: str = "int4"):
     """Layer output (fp32 [T][H]) for given routing; returns (status, out).
 
     slot_expert: int [n_slots] expert id per slot (-1 = empty); slot_blobs:
@@ -152,9 +159,9 @@ def forward_routed(x_bf16, hidden, inter, n_experts, top_k, slot_expert, slot_bl
     idx = _c(idx, np.int32)
     w = _c(w, np.float32)
     out = np.zeros((T, hidden), np.float32)
-    st = _load().oracle_forward_routed(
+    st = _load().oracle_forward_routed_fmt(
         _ptr(x), T, hidden, inter, n_experts, top_k, S, _ptr(se), _ptr_array(slot_blobs),
-        len(se), _ptr_array(shared_blobs), _ptr(idx), _ptr(w), _ptr(out))
+        len(se), _ptr_array(shared_blobs), _ptr(idx), _ptr(w), _ptr(out), FORMATS[fmt])
     return st, out
 
 

@@ -52,19 +52,30 @@ enum {
 
 size_t round_up_256(size_t v) { return (v + 255) / 256 * 256; }
 
+// Weight formats of an expert blob.
+//  FMT_INT4:  4-bit two's-complement integers, one fp16 scale per 32 along K.
+//  FMT_NVFP4: 4-bit E2M1 floats, one E4M3 scale per 16 along K, one fp32
+//             global scale per matrix (the NVFP4 routed-expert format of
+//             ro99/strata README, model table); weights are used with 16-bit
+//             activations as for int4.
+enum Format { FMT_INT4 = 0, FMT_NVFP4 = 1 };
+
 // Section offsets of one expert blob, in bytes from its start:
-// gate+up weights, down weights, gate+up scales, down scales.
+// gate+up weights, down weights, gate+up scales, down scales, and for NVFP4
+// a 256-byte section of three fp32 global scales (gate, up, down).
 struct Layout {
-  size_t guq, dq, gus, ds, total;
+  size_t guq, dq, gus, ds, glob, total;
 };
 
-Layout layout_of(int H, int I) {
+Layout layout_of(int H, int I, int fmt = FMT_INT4) {
   Layout L;
   size_t off = 0;
   L.guq = off; off = round_up_256(off + (size_t)I * H);
   L.dq = off;  off = round_up_256(off + (size_t)H * I / 2);
   L.gus = off; off = round_up_256(off + (size_t)I * H / 8);
   L.ds = off;  off = round_up_256(off + (size_t)H * I / 16);
+  L.glob = off;
+  if (fmt == FMT_NVFP4) off = round_up_256(off + 3 * sizeof(float));
   L.total = off;
   return L;
 }
@@ -95,6 +106,28 @@ float f16_value(uint16_t bits) {
   return (float)(sign ? -v : v);
 }
 
+// E2M1 (sign, 2-bit exponent with bias 1, 1-bit mantissa), from the format's
+// definition: exponent 0 is subnormal (0 or 0.5), else 2^(e-1) * (1 + m/2).
+float e2m1_value(int code) {
+  const int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  const double v = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+  return (float)(sign ? -v : v);
+}
+
+// E4M3 (sign, 4-bit exponent with bias 7, 3-bit mantissa; no infinities,
+// exponent 15 with mantissa 7 is NaN), from the format's definition.
+float e4m3_value(uint8_t byte) {
+  const int sign = (byte >> 7) & 1, e = (byte >> 3) & 0xF, m = byte & 7;
+  double v;
+  if (e == 0)
+    v = std::ldexp((double)m / 8.0, -6);
+  else if (e == 15 && m == 7)
+    v = NAN;
+  else
+    v = std::ldexp(1.0 + m / 8.0, e - 7);
+  return (float)(sign ? -v : v);
+}
+
 // The three matrices of an expert and where their rows live.  A section is
 // split into tiles of 16 rows; gate row i is row i % 8 of tile i / 8 and up
 // row i is row 8 + i % 8 of the same tile; down row r is row r % 16 of tile
@@ -102,18 +135,24 @@ float f16_value(uint16_t bits) {
 // 16 rows of 64 bytes; element k of a row sits in group k / 128, block
 // b = (k % 128) / 32, word w = (k % 32) / 8, nibble m = k % 8, at byte
 // 16 w + 4 b + m / 2 of the row's 64 bytes (low nibble for even m).  Scales:
-// per tile, group, row: four fp16 values, one per block.
+// per tile, group, row: four fp16 values, one per block (INT4), or eight
+// E4M3 bytes, scale i for elements 16 i .. 16 i + 15 of the group (NVFP4;
+// the same 8 bytes per row and group).
 enum Matrix { GATE, UP, DOWN };
 
 struct RowPlace {
   const uint8_t *q;      // section start
   const uint16_t *s;     // scale section start
   int K, tile, trow;
+  float glob;            // NVFP4 global scale of the matrix
 };
 
-RowPlace place_of(const uint8_t *blob, int H, int I, Matrix mat, int row) {
-  Layout L = layout_of(H, I);
+RowPlace place_of(const uint8_t *blob, int H, int I, Matrix mat, int row,
+                  int fmt = FMT_INT4) {
+  Layout L = layout_of(H, I, fmt);
   RowPlace p;
+  p.glob = 1.0f;
+  if (fmt == FMT_NVFP4) std::memcpy(&p.glob, blob + L.glob + sizeof(float) * (int)mat, sizeof(float));
   if (mat == DOWN) {
     p.q = blob + L.dq;
     p.s = (const uint16_t *)(blob + L.ds);
@@ -130,12 +169,24 @@ RowPlace place_of(const uint8_t *blob, int H, int I, Matrix mat, int row) {
   return p;
 }
 
-int int4_at(const RowPlace &p, int k) {
+// The 4-bit code of element k (both formats place codes alike).
+int nibble_at(const RowPlace &p, int k) {
   const int j = k / 128, b = (k % 128) / 32, w = (k % 32) / 8, m = k % 8;
   const size_t row_base = (((size_t)p.tile * (p.K / 128) + j) * 16 + p.trow) * 64;
   const uint8_t byte = p.q[row_base + 16 * w + 4 * b + m / 2];
-  const int n = (m % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+  return (m % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+}
+
+int int4_at(const RowPlace &p, int k) {
+  const int n = nibble_at(p, k);
   return n >= 8 ? n - 16 : n;
+}
+
+// NVFP4 group scale of element k: E4M3 byte (k % 128) / 16 of the row's 8.
+float e4m3_scale_at(const RowPlace &p, int k) {
+  const int j = k / 128, i = (k % 128) / 16;
+  const uint8_t *s8 = reinterpret_cast<const uint8_t *>(p.s);
+  return e4m3_value(s8[(((size_t)p.tile * (p.K / 128) + j) * 16 + p.trow) * 8 + i]);
 }
 
 float scale_at(const RowPlace &p, int k) {
@@ -144,8 +195,18 @@ float scale_at(const RowPlace &p, int k) {
 }
 
 // One dequantised row of an expert matrix (K = H for gate/up, I for down).
-void dequant_row(const uint8_t *blob, int H, int I, Matrix mat, int row, float *out) {
-  const RowPlace p = place_of(blob, H, I, mat, row);
+// INT4: w = float(fp16 scale) * q, exact in fp32.  NVFP4: w = (e2m1 value *
+// E4M3 scale, exact in fp32) * fp32 global scale, rounded once.
+void dequant_row(const uint8_t *blob, int H, int I, Matrix mat, int row, float *out,
+                 int fmt = FMT_INT4) {
+  const RowPlace p = place_of(blob, H, I, mat, row, fmt);
+  if (fmt == FMT_NVFP4) {
+    for (int k = 0; k < p.K; ++k) {
+      const float v = e2m1_value(nibble_at(p, k)) * e4m3_scale_at(p, k);
+      out[k] = v * p.glob;
+    }
+    return;
+  }
   for (int b0 = 0; b0 < p.K; b0 += 32) {
     const float scale = scale_at(p, b0);
     for (int k = b0; k < b0 + 32; ++k) out[k] = scale * (float)int4_at(p, k);
@@ -157,11 +218,11 @@ float silu(float z) { return z / (1.0f + std::exp(-z)); }
 // y[n][H] = FFN(x[n][H]) for n tokens through one expert blob.
 // Optional g, u, h outputs are [n][I].
 void expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
-                float *g_out, float *u_out, float *h_out, float *y) {
+                float *g_out, float *u_out, float *h_out, float *y, int fmt = FMT_INT4) {
   std::vector<float> wg(H), wu(H), wd(I), h((size_t)n * I);
   for (int i = 0; i < I; ++i) {
-    dequant_row(blob, H, I, GATE, i, wg.data());
-    dequant_row(blob, H, I, UP, i, wu.data());
+    dequant_row(blob, H, I, GATE, i, wg.data(), fmt);
+    dequant_row(blob, H, I, UP, i, wu.data(), fmt);
     for (int t = 0; t < n; ++t) {
       const float *xt = x + (size_t)t * H;
       float g = 0.0f, u = 0.0f;
@@ -177,7 +238,7 @@ void expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
     }
   }
   for (int r = 0; r < H; ++r) {
-    dequant_row(blob, H, I, DOWN, r, wd.data());
+    dequant_row(blob, H, I, DOWN, r, wd.data(), fmt);
     for (int t = 0; t < n; ++t) {
       const float *ht = h.data() + (size_t)t * I;
       float acc = 0.0f;
@@ -200,6 +261,7 @@ const uint8_t *lookup(const int32_t *slot_expert, const uint8_t *const *slot_blo
 extern "C" {
 
 size_t oracle_expert_bytes(int H, int I) { return layout_of(H, I).total; }
+size_t oracle_expert_bytes_fmt(int H, int I, int fmt) { return layout_of(H, I, fmt).total; }
 
 // Router for T tokens.  x: bf16 bits [T][H]; Wr: fp32 [E][H]; bias: fp32 [E]
 // or null.  Outputs: logits fp32 [T][E] (may be null), idx [T][k], w [T][k].
@@ -286,23 +348,30 @@ int oracle_route_sigmoid(const uint16_t *x, int T, int H, const float *Wr, const
 
 // One expert on n tokens given as fp32 activations.  Any of g, u, h may be
 // null; y is [n][H].
+int oracle_expert_ffn_fmt(const uint8_t *blob, int H, int I, int fmt, const float *x, int n,
+                          float *g, float *u, float *h, float *y) {
+  if (!blob || H <= 0 || I <= 0 || H % 128 || I % 128 || n < 0) return ORC_BAD_ARG;
+  if (fmt != FMT_INT4 && fmt != FMT_NVFP4) return ORC_BAD_ARG;
+  expert_ffn(blob, H, I, x, n, g, u, h, y, fmt);
+  return ORC_OK;
+}
+
 int oracle_expert_ffn(const uint8_t *blob, int H, int I, const float *x, int n,
                       float *g, float *u, float *h, float *y) {
-  if (!blob || H <= 0 || I <= 0 || H % 128 || I % 128 || n < 0) return ORC_BAD_ARG;
-  expert_ffn(blob, H, I, x, n, g, u, h, y);
-  return ORC_OK;
+  return oracle_expert_ffn_fmt(blob, H, I, FMT_INT4, x, n, g, u, h, y);
 }
 
 // Layer output for T tokens with routing given.  Experts are found through
 // the slot table (slot s holds expert slot_expert[s] at slot_blob[s]; -1 or a
 // null blob = empty).  out: fp32 [T][H].  A token whose routed expert is not
 // bound gets a zero output row and the call returns ORC_NOT_BOUND.
-int oracle_forward_routed(const uint16_t *x, int T, int H, int I, int E, int k, int S,
-                          const int32_t *slot_expert, const uint8_t *const *slot_blob,
-                          int n_slots, const uint8_t *const *shared_blob,
-                          const int32_t *idx, const float *w, float *out) {
+int oracle_forward_routed_fmt(const uint16_t *x, int T, int H, int I, int E, int k, int S,
+                              const int32_t *slot_expert, const uint8_t *const *slot_blob,
+                              int n_slots, const uint8_t *const *shared_blob,
+                              const int32_t *idx, const float *w, float *out, int fmt) {
   if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || S < 0 || n_slots < 0)
     return ORC_BAD_ARG;
+  if (fmt != FMT_INT4 && fmt != FMT_NVFP4) return ORC_BAD_ARG;
   if (H % 128 || I % 128) return ORC_BAD_ARG;
   // the same expert in two slots is a conflict
   for (int a = 0; a < n_slots; ++a)
@@ -341,7 +410,7 @@ int oracle_forward_routed(const uint16_t *x, int T, int H, int I, int E, int k, 
     yout.assign((size_t)n * H, 0.0f);
     for (int a = 0; a < n; ++a)
       std::memcpy(&xin[(size_t)a * H], &xf[(size_t)uses[a].first * H], sizeof(float) * H);
-    expert_ffn(blob, H, I, xin.data(), n, nullptr, nullptr, nullptr, yout.data());
+    expert_ffn(blob, H, I, xin.data(), n, nullptr, nullptr, nullptr, yout.data(), fmt);
     for (int a = 0; a < n; ++a)
       std::memcpy(&y[((size_t)uses[a].first * (k + S) + uses[a].second) * H],
                   &yout[(size_t)a * H], sizeof(float) * H);
@@ -364,6 +433,14 @@ int oracle_forward_routed(const uint16_t *x, int T, int H, int I, int E, int k, 
     }
   }
   return status;
+}
+
+int oracle_forward_routed(const uint16_t *x, int T, int H, int I, int E, int k, int S,
+                          const int32_t *slot_expert, const uint8_t *const *slot_blob,
+                          int n_slots, const uint8_t *const *shared_blob,
+                          const int32_t *idx, const float *w, float *out) {
+  return oracle_forward_routed_fmt(x, T, H, I, E, k, S, slot_expert, slot_blob, n_slots,
+                                   shared_blob, idx, w, out, FMT_INT4);
 }
 
 // Router followed by the routed layer.  idx/w/logits outputs may be null.

@@ -125,10 +125,13 @@ def _align256(v: int) -> int:
     return (v + 255) // 256 * 256
 
 
-def blob_layout(hidden: int, inter: int) -> dict:
-    """Byte offsets of the four sections and the blob size."""
+def blob_layout(hidden: int, inter: int, fmt: str = "int4") -> dict:
+    """Byte offsets of the sections and the blob size.  NVFP4 adds a 256-byte
+    section of three fp32 global scales (gate, up, down)."""
     H, I = hidden, inter
     sizes = [("guq", I * H), ("dq", H * I // 2), ("gus", I * H // 8), ("ds", H * I // 16)]
+    if fmt == "nvfp4":
+        sizes.append(("glob", 12))
     off, out = 0, {}
     for name, size in sizes:
         out[name] = off
@@ -137,8 +140,8 @@ def blob_layout(hidden: int, inter: int) -> dict:
     return out
 
 
-def expert_bytes(hidden: int, inter: int) -> int:
-    return blob_layout(hidden, inter)["total"]
+def expert_bytes(hidden: int, inter: int, fmt: str = "int4") -> int:
+    return blob_layout(hidden, inter, fmt)["total"]
 
 
 def _check_int4(q):
@@ -172,6 +175,22 @@ def pack_tile_scales(s_tiles: np.ndarray) -> np.ndarray:
     s = np.asarray(s_tiles, np.float16)
     t, r, nb = s.shape
     return s.reshape(t, 16, nb // 4, 4).transpose(0, 2, 1, 3).copy()
+
+
+def pack_tile_codes(c_tiles: np.ndarray) -> np.ndarray:
+    """4-bit codes (0..15) [tiles][16][K] -> u8 [tiles][K/128][16][64], placed
+    like the int4 values (NVFP4 stores E2M1 codes in the same nibbles)."""
+    c = np.asarray(c_tiles)
+    if c.min(initial=0) < 0 or c.max(initial=0) > 15:
+        raise ValueError("codes must lie in [0, 15]")
+    return pack_tiles(np.where(c >= 8, c - 16, c))
+
+
+def pack_tile_scales_e4m3(s_tiles: np.ndarray) -> np.ndarray:
+    """E4M3 scale bytes [tiles][16][K/16] -> u8 [tiles][K/128][16][8]."""
+    s = np.asarray(s_tiles, np.uint8)
+    t, r, ng = s.shape
+    return s.reshape(t, 16, ng // 8, 8).transpose(0, 2, 1, 3).copy()
 
 
 def gate_up_tiles(wg: np.ndarray, wu: np.ndarray) -> np.ndarray:
@@ -224,6 +243,7 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 _STREAM_X, _STREAM_ROUTER, _STREAM_BIAS, _STREAM_EXPERT, _STREAM_SLOTS, _STREAM_RANK = range(6)
 _STREAM_CORR = 6
+_STREAM_EXPERT_FP4 = 7
 
 
 def _rng(seed: int, stream: int, index: int = 0) -> np.random.Generator:
@@ -258,6 +278,49 @@ def make_router(cfg: LayerConfig, seed: int = 0):
     else:
         raise ValueError(cfg.bias)
     return W, b
+
+
+def build_blob_nvfp4(hidden, inter, gc, uc, dc, gs, us, ds, glob) -> np.ndarray:
+    """Assemble one NVFP4 expert blob.  gc, uc: E2M1 codes [I][H]; dc: [H][I];
+    gs, us: E4M3 scale bytes [I][H/16]; ds: [H][I/16]; glob: three fp32 global
+    scales (gate, up, down)."""
+    H, I = hidden, inter
+    lay = blob_layout(H, I, "nvfp4")
+    blob = np.zeros(lay["total"], np.uint8)
+
+    def put(name, arr):
+        raw = np.ascontiguousarray(arr).view(np.uint8).reshape(-1)
+        blob[lay[name]:lay[name] + raw.size] = raw
+
+    put("guq", pack_tile_codes(gate_up_tiles(np.asarray(gc).reshape(I, H),
+                                             np.asarray(uc).reshape(I, H))))
+    put("dq", pack_tile_codes(down_tiles(np.asarray(dc).reshape(H, I))))
+    put("gus", pack_tile_scales_e4m3(gate_up_tiles(np.asarray(gs).reshape(I, H // 16),
+                                                   np.asarray(us).reshape(I, H // 16))))
+    put("ds", pack_tile_scales_e4m3(down_tiles(np.asarray(ds).reshape(H, I // 16))))
+    put("glob", np.asarray(glob, np.float32))
+    return blob
+
+
+# E4M3 scale bytes drawn for synthetic NVFP4 experts: exponent field 3..6 with
+# any mantissa, i.e. values in [2^-4, 1.875 * 2^-1].
+_E4M3_SCALE_CODES = np.array([(e << 3) | m for e in range(3, 7) for m in range(8)], np.uint8)
+
+
+def make_expert_blob_nvfp4(cfg: LayerConfig, expert: int, seed: int = 0) -> np.ndarray:
+    """One NVFP4 expert blob: uniform random E2M1 codes (random bytes), scale
+    bytes uniform over _E4M3_SCALE_CODES, global scales U[0.02, 0.08]."""
+    H, I = cfg.hidden, cfg.inter
+    lay = blob_layout(H, I, "nvfp4")
+    r = _rng(seed, _STREAM_EXPERT_FP4, expert)
+    blob = np.zeros(lay["total"], np.uint8)
+    for name, nbytes in (("guq", I * H), ("dq", H * I // 2)):
+        blob[lay[name]:lay[name] + nbytes] = np.frombuffer(r.bytes(nbytes), np.uint8)
+    for name, count in (("gus", I * H // 8), ("ds", H * I // 16)):
+        blob[lay[name]:lay[name] + count] = r.choice(_E4M3_SCALE_CODES, size=count)
+    glob = r.uniform(0.02, 0.08, size=3).astype(np.float32)
+    blob[lay["glob"]:lay["glob"] + 12] = glob.view(np.uint8)
+    return blob
 
 
 def make_correction_bias(cfg: LayerConfig, seed: int = 0) -> np.ndarray:

@@ -50,6 +50,50 @@ def dense_expert(blob: np.ndarray, H: int, I: int):
     return Wg, Wu, Wd
 
 
+# E2M1 magnitudes by (exponent, mantissa) code: the eight values of the
+# format, written out by hand.
+E2M1_MAGNITUDES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def unpack_codes(raw: np.ndarray, tiles: int, K: int) -> np.ndarray:
+    """u8 bytes of a tiled section -> 4-bit codes [tiles][16][K] (0..15)."""
+    signed = unpack_tiles(raw, tiles, K)
+    return np.where(signed < 0, signed + 16, signed)
+
+
+def e2m1_values(codes: np.ndarray) -> np.ndarray:
+    mag = np.asarray(E2M1_MAGNITUDES)[codes & 7]
+    return np.where(codes & 8, -mag, mag)
+
+
+def e4m3_values(raw: np.ndarray) -> np.ndarray:
+    """E4M3 bytes -> float64, decoded by torch's float8_e4m3fn type."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(raw, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def tile_scales_e4m3(raw: np.ndarray, tiles: int, K: int) -> np.ndarray:
+    """E4M3 bytes of a tiled scale section -> float64 [tiles][16][K/16]."""
+    s = e4m3_values(np.asarray(raw, np.uint8)).reshape(tiles, K // 128, 16, 8)
+    return s.transpose(0, 2, 1, 3).reshape(tiles, 16, K // 16)
+
+
+def dense_expert_nvfp4(blob: np.ndarray, H: int, I: int):
+    """(Wg, Wu, Wd) of an NVFP4 blob in float64 (before the fp32 rounding)."""
+    lay = synth.blob_layout(H, I, "nvfp4")
+    glob = np.asarray(blob[lay["glob"]:lay["glob"] + 12]).view(np.float32).astype(np.float64)
+    gu = e2m1_values(unpack_codes(blob[lay["guq"]:lay["guq"] + I * H], I // 8, H))
+    gus = tile_scales_e4m3(blob[lay["gus"]:lay["gus"] + I * H // 8], I // 8, H)
+    d = e2m1_values(unpack_codes(blob[lay["dq"]:lay["dq"] + H * I // 2], H // 16, I))
+    ds = tile_scales_e4m3(blob[lay["ds"]:lay["ds"] + H * I // 16], H // 16, I)
+    w_gu = gu * np.repeat(gus, 16, axis=2)
+    Wg = w_gu[:, :8, :].reshape(I, H) * glob[0]
+    Wu = w_gu[:, 8:, :].reshape(I, H) * glob[1]
+    Wd = (d * np.repeat(ds, 16, axis=2)).reshape(H, I) * glob[2]
+    return Wg, Wu, Wd
+
+
 def ffn64(dense, x: np.ndarray) -> np.ndarray:
     Wg, Wu, Wd = dense
     g = Wg @ x

@@ -401,3 +401,85 @@ def test_route_sigmoid_subset_topk_of_keys():
         key = (sc + corr).astype(np.float32)
         assert idx[t].tolist() == naive.topk_by_subsets(key, k)
         assert float(w[t].sum()) == pytest.approx(2.5, rel=1e-6)
+
+
+# ------------------------------------------------------------ NVFP4 experts
+# (E2M1 codes in the int4 nibble places, one E4M3 scale per 16 along K, one
+# fp32 global scale per matrix)
+
+def _nvfp4_blob(H, I, gc=None, gs=None, glob=(1.0, 1.0, 1.0)):
+    gc = np.zeros((I, H), np.int64) if gc is None else gc
+    gs = np.full((I, H // 16), 0x38, np.uint8) if gs is None else gs   # 0x38 = 1.0
+    zc = np.zeros((I, H), np.int64)
+    return synth.build_blob_nvfp4(H, I, gc, zc, np.zeros((H, I), np.int64), gs,
+                                  np.full((I, H // 16), 0x38, np.uint8),
+                                  np.full((H, I // 16), 0x38, np.uint8), glob)
+
+
+def test_nvfp4_blob_size():
+    for H, I in [(128, 128), (4096, 1024)]:
+        assert oracle.expert_bytes(H, I, "nvfp4") == oracle.expert_bytes(H, I) + 256
+        assert oracle.expert_bytes(H, I, "nvfp4") == synth.expert_bytes(H, I, "nvfp4")
+
+
+def test_nvfp4_e2m1_codes_hand_table():
+    H, I = 128, 128
+    gc = np.zeros((I, H), np.int64)
+    gc[0, :16] = np.arange(16)
+    blob = _nvfp4_blob(H, I, gc=gc)
+    x = np.eye(H, dtype=np.float32)[:16]                 # one-hot activations
+    g, _, _, _ = oracle.expert_ffn(blob, H, I, x, fmt="nvfp4")
+    want = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+    assert g[:, 0].tolist() == want
+
+
+def test_nvfp4_e4m3_scales_match_library_decoder():
+    H, I = 2048, 128
+    gc = np.full((I, H), 2, np.int64)                    # E2M1 code 2 = 1.0
+    gs = np.full((I, H // 16), 0x38, np.uint8)
+    codes = np.arange(256, dtype=np.int64)
+    codes[(codes & 0x7F) == 0x7F] = 0x38                 # the two NaN encodings
+    gs[0, :128] = codes[:128]
+    gs[1, :128] = codes[128:]
+    blob = _nvfp4_blob(H, I, gc=gc, gs=gs)
+    x = np.eye(H, dtype=np.float32)[::16]                # first element of each group
+    g, _, _, _ = oracle.expert_ffn(blob, H, I, x, fmt="nvfp4")
+    got = np.concatenate([g[:, 0], g[:, 1]])
+    np.testing.assert_array_equal(got, naive.e4m3_values(codes.astype(np.uint8)).astype(np.float32))
+
+
+def test_nvfp4_weights_are_code_times_scale_times_global():
+    H, I = 256, 128
+    rng = np.random.default_rng(21)
+    gc = rng.integers(0, 16, size=(I, H))
+    gs = rng.choice(np.array([(e << 3) | m for e in range(1, 15) for m in range(8)], np.uint8),
+                    size=(I, H // 16))
+    glob = (0.0371, 1.0, 1.0)
+    blob = _nvfp4_blob(H, I, gc=gc, gs=gs, glob=glob)
+    x = np.eye(H, dtype=np.float32)
+    g, _, _, _ = oracle.expert_ffn(blob, H, I, x, fmt="nvfp4")
+    Wg, _, _ = naive.dense_expert_nvfp4(blob, H, I)
+    np.testing.assert_array_equal(g.T, Wg.astype(np.float32))   # one rounding, exact otherwise
+
+
+@pytest.mark.parametrize("E,k,S,T", [(4, 2, 1, 3), (3, 3, 0, 2)])
+def test_nvfp4_layer_matches_naive_fp64(E, k, S, T):
+    H, I = 128, 128
+    cfg = synth.custom_config("fp4", H, I, E, k, n_shared=S, tokens=(T,))
+    blobs = [synth.make_expert_blob_nvfp4(cfg, e, seed=4) for e in range(E + S)]
+    W, b = synth.make_router(cfg, seed=4)
+    x = synth.make_x(cfg, T, seed=4)
+    _, idx, w = oracle.route(x, W, b, k)
+    st, out = oracle.forward_routed(x, H, I, E, k, np.arange(E), blobs[:E], blobs[E:], idx, w,
+                                    fmt="nvfp4")
+    assert st == oracle.OK
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    dense = [naive.dense_expert_nvfp4(bl, H, I) for bl in blobs]
+    ref = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            ref[t] += float(w[t, j]) * naive.ffn64(dense[idx[t, j]], xf[t])
+        for s in range(S):
+            ref[t] += naive.ffn64(dense[E + s], xf[t])
+    err = np.abs(out - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
