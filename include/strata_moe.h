@@ -226,7 +226,9 @@ void strata_arena_destroy(strata_arena *a);
  * hits, misses and bytes.  Host-side and asynchronous; the layer's slot
  * table changes at once, so enqueue the forward that uses these experts on
  * `stream` after this call.  Errors: INVALID_ARG (an id out of range),
- * TOO_MANY_EXPERTS (more distinct ids than slots; nothing changes), CUDA. */
+ * TOO_MANY_EXPERTS (more distinct ids than slots; nothing changes), CUDA (a
+ * copy could not be enqueued; the slots bound before the failure stay
+ * bound, and their copies may still be in flight on copy_stream). */
 strata_status strata_arena_ensure(strata_arena *a, const int32_t *ids, int n,
                                   strata_stream_t stream, strata_stream_t copy_stream,
                                   strata_arena_stats *stats);
