@@ -89,10 +89,16 @@ typedef enum {
   STRATA_ERR_OOM = 6,              /* workspace allocation failed */
   STRATA_ERR_CUDA = 7,             /* a CUDA runtime call failed */
   STRATA_ERR_DEVICE_STATUS = 8,    /* another device-side error (bad routing, timeout) */
-  STRATA_ERR_SCRATCH_LIMIT = 9     /* too large for strata_moe_forward_noalloc's fixed scratch */
+  STRATA_ERR_SCRATCH_LIMIT = 9,    /* too large for strata_moe_forward_noalloc's fixed scratch */
+  STRATA_ERR_RANGE = 10            /* a value left the f16 range (device-detected; see forward) */
 } strata_status;
 
 /* Create a layer on the current CUDA device.
+ * The layer is the routed mixture-of-experts block that the pages put on the
+ * hot path of decode and prefill (ro99/strata README, "Residency" and
+ * "Kernels"; "Strata on a Mac", "What you need"): n_experts routed experts of
+ * which each token uses top_k, plus n_shared always-on experts, all of one
+ * SwiGLU shape, over an arena of n_slots expert slots.
  * hidden, inter: H and I, multiples of 128.  n_experts: 1..256.
  * top_k: 1..min(32, n_experts).  n_shared: 0..4 always-on experts of the same
  * shape.  n_slots: arena slots, top_k..n_experts.  On success *out owns a
@@ -132,7 +138,10 @@ strata_status strata_moe_set_routing(strata_moe *h, int mode, const float *corr_
  * (256-byte aligned, strata_moe_expert_bytes long).  Errors: INVALID_ARG. */
 strata_status strata_moe_bind_shared(strata_moe *h, int i, const void *device_ptr);
 
-/* Put expert_id's blob at device_ptr into slot `slot` (0 <= slot < n_slots);
+/* The expert-id -> slot table over the arena (ro99/strata README,
+ * "Residency": routed experts kept in GPU memory under LRU replacement; "Strata
+ * on a Mac", "What you need": a fixed-size arena of the most-used experts).
+ * Put expert_id's blob at device_ptr into slot `slot` (0 <= slot < n_slots);
  * expert_id == -1 empties the slot (device_ptr ignored).  device_ptr must be
  * 256-byte aligned.  Errors: INVALID_ARG (range, alignment, NULL),
  * SLOT_CONFLICT (expert_id already sits in another slot). */
@@ -146,7 +155,10 @@ int strata_moe_slot_expert(const strata_moe *h, int slot);
  * (for example before capturing them in a CUDA graph).  Errors: OOM, CUDA. */
 strata_status strata_moe_reserve(strata_moe *h, int max_tokens);
 
-/* Routing only.  x_bf16: device bf16 [n_tokens][hidden].  logits_out: device
+/* Routing only: step 1 of the description at the top of this file (the
+ * router that "Strata on a Mac", "Switches", fuses into one dispatch with its
+ * top-k: logits, then the top_k experts and their renormalised weights).
+ * x_bf16: device bf16 [n_tokens][hidden].  logits_out: device
  * fp32 [n_tokens][n_experts] or NULL.  idx_out: device int32
  * [n_tokens][top_k], experts in descending logit order (ties: lower id
  * first).  w_out: device fp32 [n_tokens][top_k], the renormalised softmax
@@ -154,11 +166,24 @@ strata_status strata_moe_reserve(strata_moe *h, int max_tokens);
 strata_status strata_moe_route(strata_moe *h, const void *x_bf16, int n_tokens, float *logits_out,
                                int32_t *idx_out, float *w_out, strata_stream_t stream);
 
-/* The whole layer.  x_bf16: device bf16 [n_tokens][hidden]; out_bf16: device
- * bf16 [n_tokens][hidden] (round to nearest even of the fp32 combine).
- * Asynchronous on `stream`.  Host errors: INVALID_ARG (including no router
- * set or a shared expert not bound), OOM, CUDA.  Device errors (see
- * strata_moe_get_status): NOT_BOUND. */
+/* The whole layer: steps 1-4 of the description at the top of this file
+ * (ro99/strata README, "Kernels": the W4A16 routed-expert FFN; "How these
+ * numbers are measured", "Fidelity (paged vs resident output)": the output
+ * does not depend on the slot table).  x_bf16: device bf16
+ * [n_tokens][hidden]; out_bf16: device bf16 [n_tokens][hidden] (round to
+ * nearest even of the fp32 combine).  Asynchronous on `stream`.
+ * Range: the kernels feed the tensor cores f16 operands, so activations and
+ * the SwiGLU output h must stay below 65520 in magnitude (larger values round
+ * to an f16 infinity), and with more than 64 tokens (the tensor-core path,
+ * which dequantises each weight to f16(q * scale)) every fp16 scale of a
+ * routed or shared expert must be below 8192 in magnitude (8 * 8192 would
+ * overflow).  A value beyond these limits is detected on the device and
+ * reported as STRATA_ERR_RANGE by strata_moe_get_status (the affected outputs
+ * are then not meaningful); with up to 64 tokens scales of any finite fp16
+ * value are applied exactly in fp32.
+ * Host errors: INVALID_ARG (including no router set or a shared expert not
+ * bound), OOM, CUDA.  Device errors (see strata_moe_get_status): NOT_BOUND,
+ * RANGE, DEVICE_STATUS (a wait that timed out). */
 strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens, void *out_bf16,
                                  strata_stream_t stream);
 
@@ -171,12 +196,14 @@ strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n
                                         strata_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the device status word: STRATA_OK,
- * STRATA_ERR_NOT_BOUND, STRATA_ERR_DEVICE_STATUS, or STRATA_ERR_CUDA if the
- * stream itself failed. */
+ * STRATA_ERR_NOT_BOUND, STRATA_ERR_RANGE, STRATA_ERR_DEVICE_STATUS (in that
+ * order of precedence, lowest last), or STRATA_ERR_CUDA if the stream itself
+ * failed. */
 strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream);
 
 /* Raw device status bits of the last get_status call (1 = not bound,
- * 2 = bad routing id, 4 = wait timeout, 8 = bounds), for diagnostics. */
+ * 2 = bad routing id, 4 = wait timeout, 8 = bounds, 16 = f16 range), for
+ * diagnostics. */
 int strata_moe_last_device_bits(const strata_moe *h);
 
 /* Per-kernel timing for measurement.  enable != 0 makes every later call
@@ -228,7 +255,9 @@ void strata_arena_destroy(strata_arena *a);
  * `stream` after this call.  Errors: INVALID_ARG (an id out of range),
  * TOO_MANY_EXPERTS (more distinct ids than slots; nothing changes), CUDA (a
  * copy could not be enqueued; the slots bound before the failure stay
- * bound, and their copies may still be in flight on copy_stream). */
+ * bound, and their copies may still be in flight on copy_stream, while the
+ * slot chosen for the failed copy keeps its old expert, in the arena and in
+ * the layer's table alike). */
 strata_status strata_arena_ensure(strata_arena *a, const int32_t *ids, int n,
                                   strata_stream_t stream, strata_stream_t copy_stream,
                                   strata_arena_stats *stats);
@@ -258,9 +287,12 @@ int strata_arena_slot_of(const strata_arena *a, int expert_id);
  * handle's workspace, and the call allocates nothing: no cudaMalloc, cudaFree
  * or other allocating routine.  n_tokens may be at most
  * STRATA_NOALLOC_MAX_TOKENS, and the workspace for n_tokens = T must fit the
- * array: with P = T * (top_k + n_shared) and N = n_experts + n_shared, about
- *     4*T*n_experts + 8*T*top_k + 4*(3N + 2) + 12*P + 2*T*hidden
- *       + 2*P*inter + 4*P*hidden  bytes (each term rounded up to 256);
+ * array: with P = T * (top_k + n_shared), N = n_experts + n_shared and M the
+ * device's multiprocessor count, about
+ *     256 + 4*T*n_experts + 8*T*top_k + 4*(3N + 2) + 12*P + 2*T*hidden
+ *       + 2*P*inter + 4*P*hidden + 12*M*(4 + 1024)  bytes
+ * (each term rounded up to 256; the last term is the decode kernels'
+ * per-warp arrival counters and partial sums, 1.8 MB on 148 multiprocessors);
  * a request beyond either limit returns STRATA_ERR_SCRATCH_LIMIT and
  * enqueues nothing.  The current device must be the handle's device
  * (otherwise INVALID_ARG).  The first call on a device looks up the array's

@@ -30,6 +30,7 @@ class Status(enum.IntEnum):
     CUDA = 7
     DEVICE_STATUS = 8
     SCRATCH_LIMIT = 9
+    RANGE = 10
 
 
 class ArenaStats(ctypes.Structure):

@@ -145,12 +145,14 @@ strata_status strata_arena_ensure(strata_arena *a, const int32_t *ids, int n,
       if (a->wanted[held] && a->last_use[s] == a->tick) continue;
       if (victim < 0 || a->last_use[s] < a->last_use[victim]) victim = s;
     }
-    const int old = a->expert_in[victim];
-    if (old >= 0) a->slot_of[old] = -1;
+    // the victim's bookkeeping changes only once its copy is enqueued: a copy
+    // that cannot be enqueued leaves the victim bound to its old expert
     uint8_t *dst = a->arena + (size_t)victim * a->blob_bytes;
     err = cudaMemcpyAsync(dst, a->pool + (size_t)e * a->blob_bytes, a->blob_bytes,
                           cudaMemcpyHostToDevice, copy_stream);
     if (err != cudaSuccess) break;
+    const int old = a->expert_in[victim];
+    if (old >= 0) a->slot_of[old] = -1;
     const strata_status st = strata_moe_bind_slot(a->layer, victim, e, dst);
     if (st != STRATA_OK) {
       clear_wanted();

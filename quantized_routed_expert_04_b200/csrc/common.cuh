@@ -3,6 +3,7 @@
 // mma.sync, lop3, griddepcontrol, tcgen05).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -14,6 +15,26 @@ namespace strata {
 // ---------------------------------------------------------------- status word
 __device__ __forceinline__ void set_status(int *status, int bit) {
   if (status) atomicOr(status, bit);
+}
+
+// Eight bf16 activations -> eight f16 stored in the order 0,4,1,5,2,6,3,7
+// (the order in which int4x8_to_f16 produces weight pairs, so that one
+// 16-byte load gives a thread its four mma B-fragment registers).  Sets
+// `overflow` if a finite or infinite input rounds to an f16 infinity.
+__device__ __forceinline__ uint4 pack8_bf16_to_f16(uint4 raw, bool &overflow) {
+  const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+  const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
+  const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
+  const float m = fmaxf(fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))),
+                        fmaxf(fmaxf(fabsf(f2.x), fabsf(f2.y)), fmaxf(fabsf(f3.x), fabsf(f3.y))));
+  overflow = m >= kF16Overflow;
+  uint4 o;
+  __half2 h;
+  h = __floats2half2_rn(f0.x, f2.x); o.x = *reinterpret_cast<uint32_t *>(&h);
+  h = __floats2half2_rn(f0.y, f2.y); o.y = *reinterpret_cast<uint32_t *>(&h);
+  h = __floats2half2_rn(f1.x, f3.x); o.z = *reinterpret_cast<uint32_t *>(&h);
+  h = __floats2half2_rn(f1.y, f3.y); o.w = *reinterpret_cast<uint32_t *>(&h);
+  return o;
 }
 
 // ---------------------------------------------------------------- addresses
@@ -132,10 +153,14 @@ __device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cas
 // Eight int4 values packed in one 32-bit word (element e in bits 4e..4e+3,
 // two's complement) -> four f16x2 registers holding the exact integers
 //   out[0] = (q0, q4), out[1] = (q1, q5), out[2] = (q2, q6), out[3] = (q3, q7)
-// (low half first).  A nibble n with its sign bit flipped is n' = q + 8 in
-// [0, 15]; OR-ing it into the mantissa of 1024.0 gives 1024 + n' (low nibble
-// position) or 1024 + 16 n' (next nibble position), both exact in f16, and
-// one f16 subtract (or multiply-add by 1/16) recovers q exactly.
+// (low half first).  This is the published magic-number conversion of
+// low-bit integers to f16 with one lop3 per pair (Kim et al., "Who Says
+// Elephants Can't Run: Bringing Large Scale MoE Models into Cloud Scale
+// Production", 2022), here in a two's-complement form: a nibble n with its
+// sign bit flipped is n' = q + 8 in [0, 15]; the same lop3 that masks it ORs
+// it into the mantissa of 1024.0 and flips the sign bit, giving 1024 + n'
+// (low nibble position) or 1024 + 16 n' (next nibble position), both exact
+// in f16, and one f16 subtract (or multiply-add by 1/16) recovers q exactly.
 __device__ __forceinline__ void int4x8_to_f16(uint32_t w, uint32_t out[4]) {
   const uint32_t w8 = w >> 8;
   const uint32_t a = and_xor(w, 0x000F000Fu, 0x64086408u);

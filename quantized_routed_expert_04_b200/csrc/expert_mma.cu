@@ -266,6 +266,7 @@ __global__ void __launch_bounds__(kMmThreads, 1) expert_mma_kernel(MmParams p) {
       const int ii = it.tau * 8 + g;
       // stored like the packed activations: group of 8 in order 0,4,1,5,2,6,3,7
       const int pos = (ii & ~7) | (((ii & 3) << 1) | ((ii >> 2) & 1));
+      if (fabsf(h) >= kF16Overflow) set_status(p.status, STATUS_RANGE);
       p.h_out[prow + pos] = __float2half_rn(h);
     } else {
       const int r0 = it.tau * 16 + g;

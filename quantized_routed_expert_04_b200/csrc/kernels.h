@@ -20,7 +20,7 @@ struct RouteMode {
 };
 __global__ void topk_kernel(const float *logits, int T, int E, int k, RouteMode mode,
                             int32_t *idx, float *w);
-__global__ void pack_x_kernel(const __nv_bfloat16 *x, int n8, __half *x16);
+__global__ void pack_x_kernel(const __nv_bfloat16 *x, int n8, __half *x16, int *status);
 __global__ void bucket_count_kernel(const int32_t *idx, int T, int k, int E, int *cnt,
                                     int *status);
 __global__ void bucket_fill_kernel(const int32_t *idx, int T, int k, int E, int S, Routing rt);

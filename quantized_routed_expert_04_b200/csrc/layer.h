@@ -20,7 +20,12 @@ enum : int {
   STATUS_BAD_ROUTING = 2,    // forward_routed got an expert id out of range
   STATUS_TIMEOUT = 4,        // a bounded wait in a kernel gave up
   STATUS_BOUNDS = 8,         // a computed offset fell outside its buffer
+  STATUS_RANGE = 16,         // a value left the f16 range of the tensor-core operands
 };
+
+// Smallest magnitude that round-to-nearest-even turns into an f16 infinity
+// (65504 is the largest finite f16; half-way to the next power step rounds up).
+constexpr float kF16Overflow = 65520.0f;
 
 // Byte offsets of the four sections of an expert blob: gate+up weights,
 // down weights, gate+up scales, down scales (see include/strata_moe.h).

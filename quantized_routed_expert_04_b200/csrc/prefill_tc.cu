@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = lane >> 2;
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
     uint32_t pk_cnt = 0, st = 0, ph = 0;
-    bool ok = true;
+    bool ok = true, big_scale = false;
     int a = 0;
     for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
       for (int g = 0; g < G && ok; ++g) {
@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 pq + j * (kPkGroups * 1024) + gi * 1024 + tr * 64 + w * 16 + atom * 8);
             const uint32_t sv = *reinterpret_cast<const uint32_t *>(
                 psc + j * (kPkGroups * 128) + gi * 128 + tr * 8 + atom * 4);
+            // |scale| >= 8192 (or not finite): q * scale can overflow f16
+            big_scale |= __vcmpgeu2(sv & 0x7FFF7FFFu, 0x70007000u) != 0u;
             const uint32_t words[2] = {qv.x, qv.y};
             const __half2 sc[2] = {__half2half2(__low2half(bits_h2(sv))),
                                    __half2half2(__high2half(bits_h2(sv)))};
@@ -360,12 +362,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
+    if (__any_sync(0xffffffffu, big_scale) && lane == 0) set_status(p.status, STATUS_RANGE);
   } else if (warp < kPkWarp) {
     // -------------------------------------------------------- epilogue
     const int qd = warp & 3;  // TMEM lane quarter of this warp
     float *stage = reinterpret_cast<float *>(smem + kOffEpi + (warp - 2 - kDqWarps) * 1024);
     uint32_t t_cnt_local = 0;
-    bool ok = true;
+    bool ok = true, big_h = false;
     int a = 0;
     for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
       const Unit un = decode(u, a);
@@ -385,7 +388,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float up = __shfl_xor_sync(0xffffffffu, v[t], 8);
             if (gate) {
               const float gv = v[t];
-              hs[t * 16 + pos16] = __float2half_rn(gv / (1.0f + expf(-gv)) * up);
+              const float hv = gv / (1.0f + expf(-gv)) * up;
+              big_h |= fabsf(hv) >= kF16Overflow;
+              hs[t * 16 + pos16] = __float2half_rn(hv);
             }
           }
           __syncwarp();
@@ -428,6 +433,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
       ++t_cnt_local;
     }
+    if (__any_sync(0xffffffffu, big_h) && lane == 0) set_status(p.status, STATUS_RANGE);
   }
 
   tc_fence_before();

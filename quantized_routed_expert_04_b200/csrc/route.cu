@@ -201,25 +201,16 @@ __global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int 
 }
 
 // ---------------------------------------------------------------- activation pack
-// x bf16 -> f16 with each group of 8 stored in the order 0,4,1,5,2,6,3,7 (the
-// order in which the int4 unpacking produces weight pairs, so one 16-byte
-// load gives a thread its four mma B-fragment registers).
+// x bf16 -> f16 (pack8_bf16_to_f16: groups of 8 in the order 0,4,1,5,2,6,3,7);
+// an activation beyond the f16 range sets STATUS_RANGE.
 __global__ void pack_x_kernel(const __nv_bfloat16 *__restrict__ x, int n8,
-                              __half *__restrict__ x16) {
+                              __half *__restrict__ x16, int *status) {
   grid_dependency_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
-  const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)i * 8);
-  const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-  const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
-  const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
-  // elements: 0=f0.x 1=f0.y 2=f1.x 3=f1.y 4=f2.x 5=f2.y 6=f3.x 7=f3.y
-  uint4 o;
-  __half2 h;
-  h = __floats2half2_rn(f0.x, f2.x); o.x = h2_bits(h);
-  h = __floats2half2_rn(f0.y, f2.y); o.y = h2_bits(h);
-  h = __floats2half2_rn(f1.x, f3.x); o.z = h2_bits(h);
-  h = __floats2half2_rn(f1.y, f3.y); o.w = h2_bits(h);
+  bool over;
+  const uint4 o = pack8_bf16_to_f16(*reinterpret_cast<const uint4 *>(x + (size_t)i * 8), over);
+  if (over) set_status(status, STATUS_RANGE);
   *reinterpret_cast<uint4 *>(x16 + (size_t)i * 8) = o;
 }
 
@@ -459,19 +450,15 @@ __device__ void bucket_block(const int *s_idx, int T, int k, int E, int S, const
 }
 
 __device__ void pack_x_range(const __nv_bfloat16 *__restrict__ x, __half *__restrict__ x16, int g0,
-                             int g1) {
+                             int g1, int *status) {
+  bool any = false;
   for (int i = g0 + (int)threadIdx.x; i < g1; i += blockDim.x) {
-    const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)i * 8);
-    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-    const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
-    const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
-    uint4 o;
-    o.x = h2_bits(__floats2half2_rn(f0.x, f2.x));
-    o.y = h2_bits(__floats2half2_rn(f0.y, f2.y));
-    o.z = h2_bits(__floats2half2_rn(f1.x, f3.x));
-    o.w = h2_bits(__floats2half2_rn(f1.y, f3.y));
+    bool over;
+    const uint4 o = pack8_bf16_to_f16(*reinterpret_cast<const uint4 *>(x + (size_t)i * 8), over);
+    any |= over;
     *reinterpret_cast<uint4 *>(x16 + (size_t)i * 8) = o;
   }
+  if (any) set_status(status, STATUS_RANGE);
 }
 
 }  // namespace
@@ -489,7 +476,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteParams p) {
   if (kBucket) {
     const int n8 = T * H / 8;
     pack_x_range(p.x, p.x16, (int)((long long)n8 * blockIdx.x / gridDim.x),
-                 (int)((long long)n8 * (blockIdx.x + 1) / gridDim.x));
+                 (int)((long long)n8 * (blockIdx.x + 1) / gridDim.x), p.status);
   }
   if (kRoute) {
     const int e = blockIdx.x;

@@ -327,7 +327,7 @@ strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *id
     const auto *xb = static_cast<const __nv_bfloat16 *>(x);
     const int n8 = T * h->H / 8;
     e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb,
-               n8, h->x16);
+               n8, h->x16, h->status);
     if (e == cudaSuccess)
       e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
                  stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
@@ -420,6 +420,8 @@ const char *strata_status_str(strata_status s) {
     case STRATA_ERR_DEVICE_STATUS: return "device-side error";
     case STRATA_ERR_SCRATCH_LIMIT:
       return "request larger than the fixed scratch of strata_moe_forward_noalloc";
+    case STRATA_ERR_RANGE:
+      return "a value left the f16 range of the tensor-core operands";
   }
   return "unknown status";
 }
@@ -618,6 +620,7 @@ strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream) {
       cudaMemset(h->counters, 0, h->counters_bytes) != cudaSuccess)
     return STRATA_ERR_CUDA;
   if (bits & (STATUS_BAD_ROUTING | STATUS_TIMEOUT | STATUS_BOUNDS)) return STRATA_ERR_DEVICE_STATUS;
+  if (bits & STATUS_RANGE) return STRATA_ERR_RANGE;
   if (bits & STATUS_NOT_BOUND) return STRATA_ERR_NOT_BOUND;
   return STRATA_OK;
 }

@@ -108,6 +108,33 @@ class GpuLayer:
         self.layer.close()
 
 
+def oracle_reference_parallel(cfg, blobs, W, b, x_bits, idx=None, w=None, n_threads=None):
+    """oracle_reference split over token chunks run in threads (the oracle's
+    C calls release the interpreter lock, so the chunks run in parallel on
+    the host cores).  Each token's output depends only on that token, so the
+    result equals the single call's.  Returns (out, idx, w)."""
+    import concurrent.futures
+    import os
+
+    import oracle
+    T = x_bits.shape[0]
+    if idx is None:
+        _, idx, w = oracle.route(x_bits, W, b, cfg.top_k)
+    n = max(1, min(T, n_threads or os.cpu_count() or 1))
+    bounds = np.linspace(0, T, n + 1).astype(int)
+    out = np.zeros((T, cfg.hidden), np.float32)
+
+    def run(i):
+        lo, hi = bounds[i], bounds[i + 1]
+        if hi > lo:
+            out[lo:hi] = oracle_reference(cfg, blobs, W, b, x_bits[lo:hi], idx[lo:hi],
+                                          w[lo:hi])[0]
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(run, range(n)))
+    return out, idx, w
+
+
 def oracle_reference(cfg, blobs, W, b, x_bits, idx=None, w=None):
     """Oracle output (fp32 [T][H]) with every expert bound; routing computed
     by the oracle unless idx/w are given.  Returns (out, idx, w)."""

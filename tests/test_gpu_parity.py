@@ -130,21 +130,6 @@ def test_forward_degenerate_shapes(E, k, S, T):
     lay.close()
 
 
-def test_forward_prefill_sampled_tokens():
-    """Prefill size (8192 tokens, 256 experts + 1 shared), in the launch
-    configuration the benchmark times; 12 sampled tokens checked against the
-    oracle one by one (routing checked on all tokens separately)."""
-    cfg = synth.CONFIGS["prefill"]
-    lay = GpuLayer(cfg)
-    x = synth.make_x(cfg, 8192)
-    st, out = lay.forward(x)
-    assert st[0] == 0
-    rows = np.random.default_rng(0).choice(8192, 12, replace=False)
-    ref, _, _ = oracle_reference(cfg, lay.blobs, lay.W, lay.b, x[rows])
-    assert_within_tolerance(out[rows], ref, "prefill sampled")
-    lay.close()
-
-
 # ------------------------------------------------------------------ invariants
 # "How these numbers are measured", Fidelity: paged output is bit-identical to
 # resident output.

@@ -96,3 +96,7 @@ def test_reference_arm_line(monkeypatch):
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert np.isfinite(line["ms_per_step"])
+    # both arms describe the workload with the same config object
+    from quantized_routed_expert_04_b200 import synth
+    assert line["config"] == bench.config_desc(synth.CONFIGS["tiny"], 4, 1)
+    assert line["cpu_baseline"]["host_cpu_count"] == os.cpu_count()
