@@ -313,7 +313,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "decode": ["quantized_routed_expert_04_b200/csrc/expert_mma.cu",
+    "decode": ["quantized_routed_expert_04_b200/csrc/decode_fused.cu",
                "quantized_routed_expert_04_b200/csrc/common.cuh"],
     "prefill": ["quantized_routed_expert_04_b200/csrc/prefill_tc.cu",
                 "quantized_routed_expert_04_b200/csrc/common.cuh"],
@@ -496,8 +496,8 @@ def measure(wl, steps, warmup, world, clocks, peaks, flush_l2, seed, config_name
                              "peak": peaks["hbm"], "unit": "GB/s",
                              "peak_source": peaks["source"] + " (copy kernel)",
                              "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg}
-        traffic_key, kfiles = "expert_mma_gateup_%s_t%d" % (config_name, T), \
-            KERNEL_SOURCES["decode"]
+        traffic_key, kfiles, traffic_kernel = "decode_fused_%s_t%d" % (config_name, T), \
+            KERNEL_SOURCES["decode"], "fused"
     else:
         flops_pair = 6.0 * H * I
         P = T * (cfg.top_k + S)
@@ -516,8 +516,8 @@ def measure(wl, steps, warmup, world, clocks, peaks, flush_l2, seed, config_name
         gu, dn = prof.get("gate_up", (0, 0.0)), prof.get("down", (0, 0.0))
         if gu[0]:
             rec["expert_gemm_tflops"] = flops_pair * P / ((gu[1] + dn[1]) / gu[0] / 1000.0) / 1e12
-        traffic_key, kfiles = "expert_tc_gateup_%s_t%d" % (config_name, T), \
-            KERNEL_SOURCES["prefill"]
+        traffic_key, kfiles, traffic_kernel = "expert_tc_gateup_%s_t%d" % (config_name, T), \
+            KERNEL_SOURCES["prefill"], "gate_up"
     for r in rooflines.values():
         r["frac"] = r["achieved"] / r["peak"]
         r["timing"] = ("CUDA events around every launch, in a pass of %d of the timed steps run "
@@ -525,7 +525,8 @@ def measure(wl, steps, warmup, world, clocks, peaks, flush_l2, seed, config_name
     if rooflines:
         dom = max(rooflines, key=lambda k: rooflines[k]["avg_launch_ms"])
         roof = dict(rooflines[dom], kernel=dom)
-        roof["traffic"] = traffic_from_profile(kfiles, traffic_key) if dom == "gate_up" else None
+        roof["traffic"] = (traffic_from_profile(kfiles, traffic_key) if dom == traffic_kernel
+                           else None)
         rec["roofline"] = roof
         rec["rooflines"] = rooflines
 

@@ -206,12 +206,27 @@ strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream);
  * diagnostics. */
 int strata_moe_last_device_bits(const strata_moe *h);
 
+/* Limit, in nanoseconds, of every wait of the small-batch (up to 64 tokens)
+ * kernel that depends on other multiprocessors or on copies in flight: its
+ * grid barriers and its ring stages (default STRATA_DEFAULT_WAIT_NS, 2 s).
+ * A wait that runs out sets the device status (STRATA_ERR_DEVICE_STATUS,
+ * bit 4) and the kernel winds down: every copy it issued still lands (that
+ * wait keeps the default limit) and every grid barrier is still passed, so no
+ * other multiprocessor waits on it; that call's outputs are not meaningful,
+ * and strata_moe_get_status resets the kernel's counters so that the next
+ * call is clean.  0 makes every wait that is not already satisfied give up at
+ * once (a way to exercise this path).  The tensor-core (more than 64 tokens)
+ * kernels keep the default.  Errors: INVALID_ARG. */
+#define STRATA_DEFAULT_WAIT_NS 2000000000ull
+strata_status strata_moe_set_wait_limit(strata_moe *h, unsigned long long ns);
+
 /* Per-kernel timing for measurement.  enable != 0 makes every later call
  * record a CUDA event pair around each kernel on the call's stream;
  * strata_moe_profile_read synchronises those events and returns, per phase,
  * the number of launches and their summed milliseconds, then clears them.
  * Phases: 0 router, 1 top-k, 2 bucketing, 3 activation pack, 4 gate/up+SwiGLU,
- * 5 down projection, 6 combine, 7 prefill gather.  n_phases <= 8.
+ * 5 down projection, 6 combine, 7 prefill gather, 8 the whole small-batch
+ * layer (one launch).  n_phases <= 9.
  * Errors: INVALID_ARG, CUDA. */
 strata_status strata_moe_profile(strata_moe *h, int enable);
 strata_status strata_moe_profile_read(strata_moe *h, int n_phases, int *launches, double *ms);
@@ -289,10 +304,11 @@ int strata_arena_slot_of(const strata_arena *a, int expert_id);
  * STRATA_NOALLOC_MAX_TOKENS, and the workspace for n_tokens = T must fit the
  * array: with P = T * (top_k + n_shared), N = n_experts + n_shared and M the
  * device's multiprocessor count, about
- *     256 + 4*T*n_experts + 8*T*top_k + 4*(3N + 2) + 12*P + 2*T*hidden
- *       + 2*P*inter + 4*P*hidden + 12*M*(4 + 1024)  bytes
- * (each term rounded up to 256; the last term is the decode kernels'
- * per-warp arrival counters and partial sums, 1.8 MB on 148 multiprocessors);
+ *     4*T*n_experts + 8*T*top_k + 4*(3N + 2) + 12*P + 2*T*hidden
+ *       + 2*P*inter + 4*P*hidden + 4*(4 + 24*M + hidden/16) + 24576*M  bytes
+ * (each term rounded up to 256; the last two terms are the decode kernel's
+ * barrier, cut-item and tile counters and its two partial-sum slots per warp,
+ * 3.7 MB on 148 multiprocessors);
  * a request beyond either limit returns STRATA_ERR_SCRATCH_LIMIT and
  * enqueues nothing.  The current device must be the handle's device
  * (otherwise INVALID_ARG).  The first call on a device looks up the array's

@@ -68,6 +68,7 @@ def load_library():
             "strata_moe_get_status": (I, [P, P]),
             "strata_moe_last_device_bits": (I, [P]),
             "strata_moe_profile": (I, [P, I]),
+            "strata_moe_set_wait_limit": (I, [P, ctypes.c_ulonglong]),
             "strata_moe_profile_read": (I, [P, I, P, P]),
             "strata_status_str": (ctypes.c_char_p, [I]),
             "strata_arena_create": (I, [P, P, P, ctypes.POINTER(P)]),
@@ -183,11 +184,18 @@ def strata_moe_get_status(h, stream=None):
     return Status(st), int(_load().strata_moe_last_device_bits(h))
 
 
+DEFAULT_WAIT_NS = 2_000_000_000
+
+
+def strata_moe_set_wait_limit(h, ns):
+    _check(_load().strata_moe_set_wait_limit(h, int(ns)), "strata_moe_set_wait_limit")
+
+
 def strata_moe_profile(h, enable):
     _check(_load().strata_moe_profile(h, 1 if enable else 0), "strata_moe_profile")
 
 
-PHASES = ("router", "topk", "bucket", "pack", "gate_up", "down", "combine", "gather")
+PHASES = ("router", "topk", "bucket", "pack", "gate_up", "down", "combine", "gather", "fused")
 
 
 def strata_moe_profile_read(h):
@@ -311,3 +319,6 @@ class StrataMoE:
 
     def status(self, stream=None):
         return strata_moe_get_status(self.h, stream)
+
+    def set_wait_limit(self, ns):
+        strata_moe_set_wait_limit(self.h, ns)

@@ -24,66 +24,61 @@ __global__ void pack_x_kernel(const __nv_bfloat16 *x, int n8, __half *x16, int *
 __global__ void bucket_count_kernel(const int32_t *idx, int T, int k, int E, int *cnt,
                                     int *status);
 __global__ void bucket_fill_kernel(const int32_t *idx, int T, int k, int E, int S, Routing rt);
-// Routing of small batches in one launch (see route.cu).
+// Routing only of small batches in one launch (see route.cu).
 constexpr int kSmallT = 64;
 struct SmallRouteParams {
   const __nv_bfloat16 *x;
   const float *W, *bias;
-  int T, H, E, k, S;
-  float *logits;   // [T][E] written (kRoute)
-  int32_t *idx;    // [T][k] written (kRoute) or read
-  float *w;        // [T][k] written (kRoute)
-  Routing rt;
-  __half *x16;
+  int T, H, E, k;
+  float *logits;   // [T][E]
+  int32_t *idx;    // [T][k]
+  float *w;        // [T][k]
   int *counter;    // last-block counter, zero between launches
-  int *status;
   RouteMode mode;
 };
-template <bool kRoute, bool kBucket>
 __global__ void route_small_kernel(SmallRouteParams p);
 
 __global__ void combine_kernel(const float *y, const int32_t *idx, const float *w,
                                const int *inv, ExpertTable table, int T, int H, int k, int S,
                                int E, __nv_bfloat16 *out);
 
-// ---- expert matmuls for small token counts (expert_mma.cu)
+// ---- the whole small-batch layer in one persistent launch (decode_fused.cu)
 //
 // One work item = (active expert, group of <= 16 of its pairs, one 16-row
-// weight tile of the blob: 8 gate + 8 up rows, or 16 down rows).  Each warp
-// of the grid takes an equal contiguous share of the (item, K group)
-// sequence; an item cut by a share boundary is finished by its last piece.
+// weight tile: 8 gate + 8 up rows, or 16 down rows).
+constexpr int kFusedWarps = 12;                     // warps per CTA, each with its own ring
 constexpr int kMmMaxStages = 8;                     // stages per warp ring
-constexpr int kMmWarps = 12;                        // warps per CTA, each with its own ring
-constexpr int kMmThreads = 32 * kMmWarps;
 constexpr int kMmMaxGroup = 16;                     // pairs per item (two n8 MMA tiles)
-constexpr int kMmMaxPairs = 4096;                   // pair tokens staged in shared memory
 constexpr int kMmSlotFloats = kMmMaxGroup * 16;     // partial sums of one piece: pairs x rows
-
-struct MmParams {
+struct FusedParams {
   ExpertTable table;
-  Routing rt;
-  int E;
-  int K;              // reduction length: H (gate/up) or I (down)
-  int kc;             // K elements per stage (multiple of 128, divides K)
-  int tiles;          // tiles per expert: I/8 (gate/up) or H/16 (down)
-  int group;          // pairs per item: 8 or 16
-  int n_ids;          // E + S
-  int stages;         // stages per warp ring (<= kMmMaxStages)
-  size_t q_off, s_off;  // weight and scale sections (gate+up or down)
-  const __half *b_src;  // gate/up: packed x16 [T][H]; down: h16 [P][I]
-  int out_ld;         // row length of the output (I for h16, H for y)
-  __half *h_out;      // gate/up output, packed like x16
-  float *y_out;       // down output
+  const __nv_bfloat16 *x;   // [T][H]
+  const float *W, *bias;    // router
+  RouteMode mode;
+  const int32_t *idx_in;    // routing given (forward_routed), else null
+  const float *w_in;
+  int T, H, I, E, k, S;
+  size_t guq, gus, dq, ds;  // blob sections
+  int kc;                   // K elements per ring stage (multiple of 128)
+  int stages, stage_bytes;  // per-warp ring
+  int group;                // pairs per item: 8 or 16
+  unsigned long long wait_ns;  // limit of every wait that depends on other warps or copies
+  size_t smem_tables;       // offset of the routing tables in dynamic shared memory
+  float *logits;            // [T][E]
+  int32_t *idx;             // [T][k] (used when more tokens than warps per CTA)
+  float *w;                 // [T][k]
+  __half *x16, *h16;        // packed activations [T][H], SwiGLU output [P][I]
+  float *y;                 // [P][H]
+  float *partial;           // [warps of the grid][2][kMmSlotFloats]
+  int *cut_cnt;             // [2][warps of the grid]   } zero between launches
+  int *tile_cnt;            // [H/16]                   } (each resets what it
+  int *bar;                 // [4] grid barriers, exit  }  used)
   int *status;
-  int stage_bytes;    // kc*8 weight bytes + kc scale bytes, rounded to 128
-  float *partial;     // [warps of the grid][kMmSlotFloats] partial sums of cut items
-  int *counters;      // [warps of the grid] pieces arrived per cut item (zero between launches)
+  __nv_bfloat16 *out;       // [T][H]
 };
-
-template <bool kGateUp, int NT>   // NT: 8-pair MMA tiles per item (1 or 2)
-__global__ void expert_mma_kernel(MmParams p);
-
-size_t mm_smem_bytes(const MmParams &p);
+template <int NT>   // NT: 8-pair MMA tiles per item (1 or 2)
+__global__ void decode_fused_kernel(FusedParams p);
+size_t fused_table_bytes(int T, int k, int S);
 
 // ---- expert matmuls for many tokens per expert (prefill_tc.cu)
 struct TcParams {
@@ -107,6 +102,5 @@ __global__ void gather_rows_kernel(const __half *x16, const int *pair_tok, const
                                    int H, int P_cap, __half *xp);
 size_t tc_smem_bytes();
 int tc_threads();
-size_t mm_fixed_smem_bytes();
 
 }  // namespace strata

@@ -9,15 +9,16 @@
 // selected experts divided by their sum, computed directly as
 // exp(l_j - l_max) / sum_j exp(l_j - l_max).
 //
-// Bucketing sorts the (token, j) pairs by expert id, then token, with no
-// atomics in the ordering (each expert's block walks the pairs in order), so
-// the layout -- and every result downstream -- is a pure function of the
-// routing, independent of slots and of scheduling.
+// Bucketing (large batches) sorts the (token, j) pairs by expert id, then
+// token, with no atomics in the ordering (each expert's block walks the pairs
+// in order), so the layout -- and every result downstream -- is a pure
+// function of the routing, independent of slots and of scheduling.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace strata {
 
@@ -117,74 +118,6 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
 }
 
 // ---------------------------------------------------------------- top-k
-// One warp per token.  Lane l holds experts l, l+32, ...; k rounds of a warp
-// arg-max of the selection key (larger wins, equal keys: lower id wins).
-// Softmax routing: key = logit, weights = exp(l_j - l_0) / sum_j (the
-// renormalised softmax of the selected experts).  Sigmoid routing: score =
-// 1 / (1 + exp(-l)) in double rounded to fp32, key = score + correction,
-// weights = score_j / (sum of the selected scores in selection order) *
-// routed scale.  Lane j (< k) returns selection j in sel_e / sel_w.
-__device__ void select_topk_warp(const float *__restrict__ logit_row, int E, int k,
-                                 const RouteMode &mode, int lane, int &sel_e, float &sel_w) {
-  constexpr int kPer = kMaxExperts / 32;
-  float key[kPer], val[kPer];   // val: logit (softmax) or score (sigmoid)
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane + 32 * i;
-    const float l = e < E ? __ldcg(logit_row + e) : -INFINITY;
-    if (mode.sigmoid && e < E) {
-      val[i] = (float)(1.0 / (1.0 + exp(-(double)l)));
-      key[i] = mode.corr ? __fadd_rn(val[i], mode.corr[e]) : val[i];
-    } else {
-      val[i] = l;
-      key[i] = l;
-    }
-  }
-  unsigned taken = 0;
-  float v0 = 0.0f, z = 0.0f, my_v = 0.0f;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || key[i] > bk)) {
-        bk = key[i];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (oe != 0x7fffffff && (be == 0x7fffffff || ok > bk || (ok == bk && oe < be))) {
-        bk = ok;
-        be = oe;
-      }
-    }
-    // the winner's logit or score, from the lane that holds it
-    float mine = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (i == (be >> 5)) mine = val[i];
-    const float bv = __shfl_sync(0xffffffffu, mine, be & 31);
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (mode.sigmoid) {
-      z = __fadd_rn(z, bv);
-    } else {
-      if (j == 0) v0 = bv;
-      z += expf(bv - v0);
-    }
-    if (lane == j) {  // lane j keeps selection j (k <= 32)
-      my_v = bv;
-      my_e = be;
-    }
-  }
-  sel_e = my_e;
-  sel_w = mode.sigmoid ? __fmul_rn(__fdiv_rn(my_v, z), mode.scale) : expf(my_v - v0) / z;
-}
-
 __global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int k, RouteMode mode,
                             int32_t *__restrict__ idx, float *__restrict__ w) {
   grid_dependency_wait();
@@ -356,129 +289,19 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
 }
 
 // ---------------------------------------------------------------- small batches
-// Routing of up to kSmallT tokens in one launch (decode).  Every block
-// computes the logits of one expert (8 warps split h; per-warp double sums
-// added in a fixed order) and packs a slice of the activations; the last
-// block to finish -- found with a device counter, each block's writes released
-// by a fence before its counter increment and acquired by the last block with
-// a fence after it -- takes the top-k of every token and, for a forward call,
-// buckets the pairs.  The last block resets the counter for the next launch.
-namespace {
-
-__device__ void topk_token_warp(const float *__restrict__ logit_row, int E, int k,
-                                const RouteMode &mode, int lane, int32_t *idx_out, float *w_out,
-                                int *s_idx) {
-  int e;
-  float wt;
-  select_topk_warp(logit_row, E, k, mode, lane, e, wt);
-  if (lane < k) {
-    idx_out[lane] = e;
-    w_out[lane] = wt;
-    if (s_idx) s_idx[lane] = e;
-  }
-}
-
-// Bucketing of T*k routed pairs (ids in s_idx, shared memory) plus S shared
-// experts by one block of 256 threads.
-__device__ void bucket_block(const int *s_idx, int T, int k, int E, int S, const Routing &rt,
-                             int *status, int *s_cnt, int *s_off) {
-  const int tid = threadIdx.x;
-  const int nid = E + S;
-  const int n = T * k;
-  const int kS = k + S;
-  for (int i = tid; i < nid; i += blockDim.x) s_cnt[i] = i < E ? 0 : T;
-  __syncthreads();
-  for (int p = tid; p < n; p += blockDim.x) {
-    const int e = s_idx[p];
-    if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
-  }
-  __syncthreads();
-  if (tid < 32) {
-    int carry = 0, acarry = 0;
-    for (int i0 = 0; i0 < nid; i0 += 32) {
-      const int i = i0 + tid;
-      const int c = i < nid ? s_cnt[i] : 0;
-      const int f = c > 0;
-      int inc = c, finc = f;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int a = __shfl_up_sync(0xffffffffu, inc, o);
-        const int b = __shfl_up_sync(0xffffffffu, finc, o);
-        if (tid >= o) {
-          inc += a;
-          finc += b;
-        }
-      }
-      if (i < nid) {
-        const int off = carry + inc - c;
-        s_off[i] = off;
-        rt.off[i] = off;
-        rt.cnt[i] = c;
-        if (f) rt.active[acarry + finc - 1] = i;
-      }
-      carry += __shfl_sync(0xffffffffu, inc, 31);
-      acarry += __shfl_sync(0xffffffffu, finc, 31);
-    }
-    if (tid == 0) {
-      rt.off[nid] = carry;
-      *rt.n_active = acarry;
-    }
-  }
-  __syncthreads();
-  for (int p = tid; p < n; p += blockDim.x) {
-    const int e = s_idx[p];
-    const int t = p / k, j = p - (p / k) * k;
-    if (e < 0 || e >= E) {
-      set_status(status, STATUS_BAD_ROUTING);
-      rt.inv[(size_t)t * kS + j] = -1;
-      continue;
-    }
-    int rank = 0;
-    for (int q = 0; q < p; ++q) rank += (s_idx[q] == e);
-    const int pos = s_off[e] + rank;
-    rt.pair_tok[pos] = t;
-    rt.pair_j[pos] = j;
-    rt.inv[(size_t)t * kS + j] = pos;
-  }
-  for (int q = tid; q < T * S; q += blockDim.x) {
-    const int s = q / T, t = q - (q / T) * T;
-    const int pos = s_off[E + s] + t;
-    rt.pair_tok[pos] = t;
-    rt.pair_j[pos] = k + s;
-    rt.inv[(size_t)t * kS + k + s] = pos;
-  }
-}
-
-__device__ void pack_x_range(const __nv_bfloat16 *__restrict__ x, __half *__restrict__ x16, int g0,
-                             int g1, int *status) {
-  bool any = false;
-  for (int i = g0 + (int)threadIdx.x; i < g1; i += blockDim.x) {
-    bool over;
-    const uint4 o = pack8_bf16_to_f16(*reinterpret_cast<const uint4 *>(x + (size_t)i * 8), over);
-    any |= over;
-    *reinterpret_cast<uint4 *>(x16 + (size_t)i * 8) = o;
-  }
-  if (any) set_status(status, STATUS_RANGE);
-}
-
-}  // namespace
-
-template <bool kRoute, bool kBucket>
+// Routing only (strata_moe_route) of up to kSmallT tokens in one launch.
+// Every block computes the logits of one expert (8 warps split h; per-warp
+// double sums added in a fixed order); the last block to finish -- found with
+// a device counter, each block's writes released by a fence before its
+// counter increment and acquired by the last block with a fence after it --
+// takes the top-k of every token and resets the counter for the next launch.
 __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteParams p) {
   grid_dependency_wait();
   __shared__ double s_part[8][kSmallT];
-  __shared__ int s_idx[kSmallT * kMaxTopK];
-  __shared__ int s_cnt[kMaxIds], s_off[kMaxIds];
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, H = p.H, E = p.E, k = p.k;
-
-  if (kBucket) {
-    const int n8 = T * H / 8;
-    pack_x_range(p.x, p.x16, (int)((long long)n8 * blockIdx.x / gridDim.x),
-                 (int)((long long)n8 * (blockIdx.x + 1) / gridDim.x), p.status);
-  }
-  if (kRoute) {
+  {
     const int e = blockIdx.x;
     const float *wr = p.W + (size_t)e * H;
     const int span = H / 8;
@@ -533,20 +356,16 @@ __global__ void __launch_bounds__(256) route_small_kernel(SmallRouteParams p) {
     if (!s_last) return;
     __threadfence();
   }
-  if (kRoute) {
-    for (int t = warp; t < T; t += 8)
-      topk_token_warp(p.logits + (size_t)t * E, E, k, p.mode, lane, p.idx + (size_t)t * k,
-                      p.w + (size_t)t * k, kBucket ? s_idx + t * k : nullptr);
-  } else {
-    for (int q = tid; q < T * k; q += blockDim.x) s_idx[q] = p.idx[q];
+  for (int t = warp; t < T; t += 8) {
+    int e;
+    float wt;
+    select_topk_warp(p.logits + (size_t)t * E, E, k, p.mode, lane, e, wt);
+    if (lane < k) {
+      p.idx[(size_t)t * k + lane] = e;
+      p.w[(size_t)t * k + lane] = wt;
+    }
   }
-  __syncthreads();
-  if (kBucket) bucket_block(s_idx, T, k, E, p.S, p.rt, p.status, s_cnt, s_off);
   if (tid == 0 && gridDim.x > 1) *p.counter = 0;
 }
-
-template __global__ void route_small_kernel<true, true>(SmallRouteParams);
-template __global__ void route_small_kernel<true, false>(SmallRouteParams);
-template __global__ void route_small_kernel<false, true>(SmallRouteParams);
 
 }  // namespace strata

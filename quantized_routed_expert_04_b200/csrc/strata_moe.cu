@@ -21,8 +21,10 @@ using namespace strata;
 
 namespace {
 
-constexpr int kPhases = 8;
-enum Phase { PH_ROUTER = 0, PH_TOPK, PH_BUCKET, PH_PACK, PH_GATEUP, PH_DOWN, PH_COMBINE, PH_GATHER };
+constexpr int kPhases = 9;
+enum Phase {
+  PH_ROUTER = 0, PH_TOPK, PH_BUCKET, PH_PACK, PH_GATEUP, PH_DOWN, PH_COMBINE, PH_GATHER, PH_FUSED
+};
 
 struct EventPair {
   int phase;
@@ -57,9 +59,10 @@ struct strata_moe {
   __half *h16 = nullptr;
   float *y = nullptr;
   __half *xp = nullptr;     // activations gathered in sorted pair order (large batches)
-  float *partial = nullptr; // decode kernels: partial sums of items cut between warps
-  int *counters = nullptr;  // decode kernels: arrival counters (zero between launches)
+  float *partial = nullptr; // decode kernel: partial sums of items cut between warps
+  int *counters = nullptr;  // decode kernel: barrier, cut-item and tile counters (zero between launches)
   size_t counters_bytes = 0;
+  unsigned long long wait_ns = STRATA_DEFAULT_WAIT_NS;  // limit of the decode kernel's waits
   int *status = nullptr;    // device status word (own allocation)
   int *counter = nullptr;   // last-block counter of the small-batch routing kernel
   int last_bits = 0;
@@ -123,6 +126,16 @@ cudaError_t launch(strata_moe *h, int phase, void (*kern)(Exp...), dim3 grid, di
   return err;
 }
 
+// Decode kernel workspace: two partial-sum slots per warp of the grid; the
+// counters: 4 barrier/exit counters, one cut-item counter per warp and phase,
+// one tile counter per 16 output rows.
+size_t fused_partial_bytes(const strata_moe *h) {
+  return sizeof(float) * 2 * (size_t)kFusedWarps * h->num_sms * kMmSlotFloats;
+}
+size_t fused_counter_bytes(const strata_moe *h) {
+  return sizeof(int) * (4 + 2 * (size_t)kFusedWarps * h->num_sms + (size_t)h->H / 16);
+}
+
 strata_status grow_workspace(strata_moe *h, int T) {
   if (T <= h->cap_tokens) return STRATA_OK;
   const int cap = std::max(T, 2 * h->cap_tokens);
@@ -146,9 +159,8 @@ strata_status grow_workspace(strata_moe *h, int T) {
   const size_t o_h16 = take(sizeof(__half) * P * h->I);
   const size_t o_y = take(sizeof(float) * P * h->H);
   const size_t o_xp = cap > kSmallT ? take(sizeof(__half) * P * h->H) : 0;
-  const size_t n_counters = (size_t)kMmWarps * h->num_sms;
-  const size_t o_partial = take(sizeof(float) * n_counters * kMmSlotFloats);
-  const size_t o_counters = take(sizeof(int) * n_counters);
+  const size_t o_partial = take(fused_partial_bytes(h));
+  const size_t o_counters = take(fused_counter_bytes(h));
   void *mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, off);
   if (e != cudaSuccess) {
@@ -177,7 +189,7 @@ strata_status grow_workspace(strata_moe *h, int T) {
   h->xp = cap > kSmallT ? reinterpret_cast<__half *>(b + o_xp) : nullptr;
   h->partial = reinterpret_cast<float *>(b + o_partial);
   h->counters = reinterpret_cast<int *>(b + o_counters);
-  h->counters_bytes = sizeof(int) * n_counters;
+  h->counters_bytes = fused_counter_bytes(h);
   e = cudaMemset(h->counters, 0, h->counters_bytes);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e);
@@ -191,52 +203,6 @@ ExpertTable make_table(const strata_moe *h) {
     if (h->slot_expert[s] >= 0) t.ptr[h->slot_expert[s]] = static_cast<const uint8_t *>(h->slot_ptr[s]);
   for (int i = 0; i < h->S; ++i) t.ptr[h->E + i] = static_cast<const uint8_t *>(h->shared_ptr[i]);
   return t;
-}
-
-// Stage size and count of the per-warp rings: K chunks of up to 512 elements
-// (4 KB of packed weights per copy; halved until three stages fit; a piece's
-// last chunk may be shorter), as many stages as fit.
-void pick_chunk(int K, int *kc_out, int *stages_out) {
-  const size_t avail = 232448 - 1024 - mm_fixed_smem_bytes();
-  const size_t per_warp = avail / kMmWarps;
-  int kc = std::min(K, 512);
-  while (kc > 128 && per_warp / align_up((size_t)kc * 9, 128) < 3)
-    kc = std::max(128, kc / 256 * 128);
-  const size_t stage = align_up((size_t)kc * 9, 128);
-  *kc_out = kc;
-  *stages_out = (int)std::max<size_t>(2, std::min<size_t>(kMmMaxStages, per_warp / stage));
-}
-
-MmParams mm_params(const strata_moe *h, bool gate_up, const ExpertTable &table, int T) {
-  MmParams p;
-  std::memset(&p, 0, sizeof p);
-  p.table = table;
-  p.rt = h->rt;
-  p.E = h->E;
-  p.K = gate_up ? h->H : h->I;
-  pick_chunk(p.K, &p.kc, &p.stages);
-  p.group = T <= 8 ? 8 : kMmMaxGroup;
-  p.n_ids = h->E + h->S;
-  if (gate_up) {
-    p.tiles = h->I / 8;
-    p.q_off = h->layout.guq;
-    p.s_off = h->layout.gus;
-    p.b_src = h->x16;
-    p.out_ld = h->I;
-  } else {
-    p.tiles = h->H / 16;
-    p.q_off = h->layout.dq;
-    p.s_off = h->layout.ds;
-    p.b_src = h->h16;
-    p.out_ld = h->H;
-  }
-  p.h_out = h->h16;
-  p.y_out = h->y;
-  p.status = h->status;
-  p.stage_bytes = (int)align_up((size_t)p.kc * 9, 128);
-  p.partial = h->partial;
-  p.counters = h->counters;
-  return p;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -311,47 +277,29 @@ strata_status check_common(strata_moe *h, const void *x, int T, cudaStream_t) {
   return STRATA_OK;
 }
 
-// Bucketing + the expert passes + combine, given idx/w in device memory.
-// routed_small: the small-batch routing kernel already bucketed the pairs and
-// packed the activations.
+// Large batches (T > 64): bucketing + the tensor-core expert passes + combine,
+// given idx/w in device memory.
 strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *idx, const float *w,
-                          void *out, cudaStream_t stream, bool routed_small) {
+                          void *out, cudaStream_t stream) {
   const ExpertTable table = make_table(h);
   const int kS = h->k + h->S;
   const int nid = h->E + h->S;
-  cudaError_t e = cudaSuccess;
-  if (!routed_small) {
-    e = cudaMemsetAsync(h->rt.cnt, 0, sizeof(int) * nid, stream);
-    if (e == cudaSuccess) e = cudaMemsetAsync(h->rt.inv, 0xFF, sizeof(int) * (size_t)T * kS, stream);
-    if (e != cudaSuccess) return cuda_status(e);
-    const auto *xb = static_cast<const __nv_bfloat16 *>(x);
-    const int n8 = T * h->H / 8;
-    e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb,
-               n8, h->x16, h->status);
-    if (e == cudaSuccess)
-      e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
-                 stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
-    if (e == cudaSuccess)
-      e = launch(h, PH_BUCKET, bucket_fill_kernel, dim3(nid), dim3(256), 0, stream, true, idx, T,
-                 h->k, h->E, h->S, h->rt);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
-  if (T > kSmallT) {
-    const strata_status st = run_tc_experts(h, T, table, stream);
-    if (st != STRATA_OK) return st;
-  }
-  for (int pass = 0; pass < 2 && T <= kSmallT; ++pass) {
-    const bool gu = pass == 0;
-    MmParams p = mm_params(h, gu, table, T);
-    const size_t smem = mm_smem_bytes(p);
-    auto kern = p.group <= 8 ? (gu ? expert_mma_kernel<true, 1> : expert_mma_kernel<false, 1>)
-                             : (gu ? expert_mma_kernel<true, 2> : expert_mma_kernel<false, 2>);
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(kMmThreads), smem,
-                 stream, true, p);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
+  cudaError_t e = cudaMemsetAsync(h->rt.cnt, 0, sizeof(int) * nid, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->rt.inv, 0xFF, sizeof(int) * (size_t)T * kS, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+  const int n8 = T * h->H / 8;
+  e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb,
+             n8, h->x16, h->status);
+  if (e == cudaSuccess)
+    e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
+               stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
+  if (e == cudaSuccess)
+    e = launch(h, PH_BUCKET, bucket_fill_kernel, dim3(nid), dim3(256), 0, stream, true, idx, T,
+               h->k, h->E, h->S, h->rt);
+  if (e != cudaSuccess) return cuda_status(e);
+  const strata_status st = run_tc_experts(h, T, table, stream);
+  if (st != STRATA_OK) return st;
   dim3 cgrid((h->H / 4 + 127) / 128, T);
   e = launch(h, PH_COMBINE, combine_kernel, cgrid, dim3(128), 0, stream, true, h->y, idx, w,
              h->rt.inv, table, T, h->H, h->k, h->S, h->E, static_cast<__nv_bfloat16 *>(out));
@@ -368,31 +316,22 @@ SmallRouteParams small_params(strata_moe *h, const void *x, int T, float *logits
   p.H = h->H;
   p.E = h->E;
   p.k = h->k;
-  p.S = h->S;
   p.logits = logits;
   p.idx = idx;
   p.w = w;
-  p.rt = h->rt;
-  p.x16 = h->x16;
   p.counter = h->counter;
-  p.status = h->status;
   p.mode = h->mode;
   return p;
 }
 
-// Router + top-k (+ bucketing and activation pack when `bucket`).
+// Router + top-k.
 strata_status run_router(strata_moe *h, const void *x, int T, float *logits, int32_t *idx,
-                         float *w, cudaStream_t stream, bool bucket) {
+                         float *w, cudaStream_t stream) {
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
   cudaError_t e;
   if (T <= kSmallT) {
     const SmallRouteParams p = small_params(h, x, T, logits, idx, w);
-    if (bucket)
-      e = launch(h, PH_ROUTER, route_small_kernel<true, true>, dim3(h->E), dim3(256), 0, stream,
-                 false, p);
-    else
-      e = launch(h, PH_ROUTER, route_small_kernel<true, false>, dim3(h->E), dim3(256), 0, stream,
-                 false, p);
+    e = launch(h, PH_ROUTER, route_small_kernel, dim3(h->E), dim3(256), 0, stream, false, p);
     return cuda_status(e);
   }
   e = launch(h, PH_ROUTER, router_gemm_kernel, dim3((T + 127) / 128, (h->E + 63) / 64), dim3(256), 0,
@@ -400,6 +339,83 @@ strata_status run_router(strata_moe *h, const void *x, int T, float *logits, int
   if (e == cudaSuccess)
     e = launch(h, PH_TOPK, topk_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, true, logits, T,
                h->E, h->k, h->mode, idx, w);
+  return cuda_status(e);
+}
+
+// The whole small-batch layer in one cooperative launch (decode_fused.cu).
+// idx_in/w_in: the routing, or null to compute it.
+strata_status run_fused(strata_moe *h, const void *x, int T, const int32_t *idx_in,
+                        const float *w_in, void *out, cudaStream_t stream) {
+  FusedParams p;
+  std::memset(&p, 0, sizeof p);
+  p.table = make_table(h);
+  p.x = static_cast<const __nv_bfloat16 *>(x);
+  p.W = h->router_W;
+  p.bias = h->router_b;
+  p.mode = h->mode;
+  p.idx_in = idx_in;
+  p.w_in = w_in;
+  p.T = T;
+  p.H = h->H;
+  p.I = h->I;
+  p.E = h->E;
+  p.k = h->k;
+  p.S = h->S;
+  p.guq = h->layout.guq;
+  p.gus = h->layout.gus;
+  p.dq = h->layout.dq;
+  p.ds = h->layout.ds;
+  p.group = T <= 8 ? 8 : kMmMaxGroup;
+  p.wait_ns = h->wait_ns;
+  // ring stages of 512 K elements (4 KB of packed weights + 512 B of scales
+  // per copy pair), as many per warp as fit beside the tables
+  p.kc = 512;
+  p.stage_bytes = (int)align_up((size_t)p.kc * 9, 128);
+  const size_t tables = fused_table_bytes(T, h->k, h->S);
+  const size_t bars = (size_t)kFusedWarps * kMmMaxStages * sizeof(uint64_t);
+  const size_t avail = 232448 - tables - bars;
+  p.stages = (int)std::min<size_t>(kMmMaxStages, avail / ((size_t)kFusedWarps * p.stage_bytes));
+  if (p.stages < 2) return STRATA_ERR_UNSUPPORTED;
+  p.smem_tables = (size_t)kFusedWarps * p.stages * p.stage_bytes + bars;
+  const size_t smem = p.smem_tables + tables;
+  p.logits = h->logits;
+  p.idx = h->idx;
+  p.w = h->w;
+  p.x16 = h->x16;
+  p.h16 = h->h16;
+  p.y = h->y;
+  p.partial = h->partial;
+  p.bar = h->counters;
+  p.cut_cnt = h->counters + 4;
+  p.tile_cnt = h->counters + 4 + 2 * kFusedWarps * h->num_sms;
+  p.status = h->status;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  auto kern = p.group <= 8 ? decode_fused_kernel<1> : decode_fused_kernel<2>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_status(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(h->num_sms);
+  cfg.blockDim = dim3(32 * kFusedWarps);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  // every CTA must be resident at once: the phases meet at grid barriers
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  EventPair ev{PH_FUSED, nullptr, nullptr};
+  if (h->profiling) {
+    ev.a = take_event(h);
+    ev.b = take_event(h);
+    cudaEventRecord(ev.a, stream);
+  }
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (h->profiling) {
+    cudaEventRecord(ev.b, stream);
+    h->events.push_back(ev);
+  }
   return cuda_status(e);
 }
 
@@ -565,7 +581,7 @@ strata_status strata_moe_route(strata_moe *h, const void *x_bf16, int n_tokens, 
   st = grow_workspace(h, n_tokens);
   if (st != STRATA_OK) return st;
   return run_router(h, x_bf16, n_tokens, logits_out ? logits_out : h->logits, idx_out, w_out,
-                    stream, false);
+                    stream);
 }
 
 strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens, void *out_bf16,
@@ -579,10 +595,10 @@ strata_status strata_moe_forward(strata_moe *h, const void *x_bf16, int n_tokens
   if (!out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 15)) return STRATA_ERR_INVALID_ARG;
   st = grow_workspace(h, n_tokens);
   if (st != STRATA_OK) return st;
-  const bool small = n_tokens <= kSmallT;
-  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream, small);
+  if (n_tokens <= kSmallT) return run_fused(h, x_bf16, n_tokens, nullptr, nullptr, out_bf16, stream);
+  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream);
   if (st != STRATA_OK) return st;
-  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream, small);
+  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream);
 }
 
 strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n_tokens,
@@ -597,15 +613,8 @@ strata_status strata_moe_forward_routed(strata_moe *h, const void *x_bf16, int n
     return STRATA_ERR_INVALID_ARG;
   st = grow_workspace(h, n_tokens);
   if (st != STRATA_OK) return st;
-  const bool small = n_tokens <= kSmallT;
-  if (small) {
-    const SmallRouteParams p = small_params(h, x_bf16, n_tokens, nullptr, const_cast<int32_t *>(idx),
-                                            nullptr);
-    cudaError_t e = launch(h, PH_BUCKET, route_small_kernel<false, true>, dim3(1), dim3(256), 0,
-                           stream, false, p);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
-  return run_experts(h, x_bf16, n_tokens, idx, w, out_bf16, stream, small);
+  if (n_tokens <= kSmallT) return run_fused(h, x_bf16, n_tokens, idx, w, out_bf16, stream);
+  return run_experts(h, x_bf16, n_tokens, idx, w, out_bf16, stream);
 }
 
 strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream) {
@@ -626,6 +635,12 @@ strata_status strata_moe_get_status(strata_moe *h, strata_stream_t stream) {
 }
 
 int strata_moe_last_device_bits(const strata_moe *h) { return h ? h->last_bits : 0; }
+
+strata_status strata_moe_set_wait_limit(strata_moe *h, unsigned long long ns) {
+  if (!h) return STRATA_ERR_INVALID_ARG;
+  h->wait_ns = ns;
+  return STRATA_OK;
+}
 
 strata_status strata_moe_profile(strata_moe *h, int enable) {
   if (!h) return STRATA_ERR_INVALID_ARG;
@@ -697,11 +712,11 @@ strata_status noalloc_scratch_on(int device, unsigned char **out) {
   return STRATA_OK;
 }
 
-// Byte offsets in the array for T tokens: the routing kernel's block counter
-// (the only thing that must be zero when a call starts), then the regions of
-// the small-batch workspace.
+// Byte offsets in the array for T tokens: the regions of the small-batch
+// workspace (the counters are the only ones that must be zero when a call
+// starts).
 struct NoAllocLayout {
-  size_t counter, logits, idx, w, meta, ptok, pj, inv, x16, h16, y, counters, partial, total;
+  size_t logits, idx, w, meta, ptok, pj, inv, x16, h16, y, counters, partial, total;
 };
 
 NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
@@ -714,7 +729,6 @@ NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
     return o;
   };
   NoAllocLayout L;
-  L.counter = take(sizeof(int));
   L.logits = take(sizeof(float) * T * h->E);
   L.idx = take(sizeof(int32_t) * T * h->k);
   L.w = take(sizeof(float) * T * h->k);
@@ -725,8 +739,8 @@ NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
   L.x16 = take(sizeof(__half) * T * h->H);
   L.h16 = take(sizeof(__half) * P * h->I);
   L.y = take(sizeof(float) * P * h->H);
-  L.counters = take(sizeof(int) * kMmWarps * h->num_sms);
-  L.partial = take(sizeof(float) * kMmWarps * h->num_sms * kMmSlotFloats);
+  L.counters = take(fused_counter_bytes(h));
+  L.partial = take(fused_partial_bytes(h));
   L.total = off;
   return L;
 }
@@ -740,7 +754,7 @@ class NoAllocWorkspace {
  public:
   NoAllocWorkspace(strata_moe *h, unsigned char *base, const NoAllocLayout &L)
       : h_(h), logits_(h->logits), idx_(h->idx), w_(h->w), meta_(h->meta), rt_(h->rt),
-        x16_(h->x16), h16_(h->h16), y_(h->y), xp_(h->xp), counter_(h->counter),
+        x16_(h->x16), h16_(h->h16), y_(h->y), xp_(h->xp),
         partial_(h->partial), counters_(h->counters),
         profiling_(h->profiling) {
     const int nid = h->E + h->S;
@@ -759,7 +773,6 @@ class NoAllocWorkspace {
     h->h16 = reinterpret_cast<__half *>(base + L.h16);
     h->y = reinterpret_cast<float *>(base + L.y);
     h->xp = nullptr;
-    h->counter = reinterpret_cast<int *>(base + L.counter);
     h->counters = reinterpret_cast<int *>(base + L.counters);
     h->partial = reinterpret_cast<float *>(base + L.partial);
     h->profiling = false;
@@ -774,7 +787,6 @@ class NoAllocWorkspace {
     h_->h16 = h16_;
     h_->y = y_;
     h_->xp = xp_;
-    h_->counter = counter_;
     h_->partial = partial_;
     h_->counters = counters_;
     h_->profiling = profiling_;
@@ -792,7 +804,6 @@ class NoAllocWorkspace {
   __half *x16_, *h16_;
   float *y_;
   __half *xp_;
-  int *counter_;
   float *partial_;
   int *counters_;
   bool profiling_;
@@ -819,16 +830,11 @@ extern "C" strata_status strata_moe_forward_noalloc(strata_moe *h, const void *x
   unsigned char *base = nullptr;
   st = noalloc_scratch_on(device, &base);
   if (st != STRATA_OK) return st;
-  // The routing kernel's block counter and the decode kernels' arrival
-  // counters must start at zero (a call that timed out may have left them
-  // otherwise).  Everything else is written before it is read.
-  cudaError_t e = cudaMemsetAsync(base + L.counter, 0, sizeof(int), stream);
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(base + L.counters, 0,
-                        sizeof(int) * kMmWarps * h->num_sms, stream);
+  // The decode kernel's barrier, cut-item and tile counters must start at
+  // zero (a call that timed out may have left them otherwise).  Everything
+  // else is written before it is read.
+  cudaError_t e = cudaMemsetAsync(base + L.counters, 0, fused_counter_bytes(h), stream);
   if (e != cudaSuccess) return cuda_status(e);
   NoAllocWorkspace ws(h, base, L);
-  st = run_router(h, x_bf16, n_tokens, h->logits, h->idx, h->w, stream, true);
-  if (st != STRATA_OK) return st;
-  return run_experts(h, x_bf16, n_tokens, h->idx, h->w, out_bf16, stream, true);
+  return run_fused(h, x_bf16, n_tokens, nullptr, nullptr, out_bf16, stream);
 }
