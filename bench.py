@@ -569,6 +569,70 @@ def measure(wl, steps, warmup, world, clocks, peaks, flush_l2, seed, config_name
     return rec
 
 
+CHUNKS = (1024, 2048, 4096)
+
+
+def measure_chunked(cfg, T, seed, steps, flush_l2, clocks):
+    """Chunked prefill through an arena with half the experts' slots
+    (strata_arena_prefill): per chunk size, the device time of whole prompts
+    (routing, the host read of the routing, per-chunk expert copies from
+    pinned host memory, expert passes and combines), copied bytes and groups."""
+    import torch
+
+    from quantized_routed_expert_04_b200 import binding
+    E, S = cfg.n_experts, cfg.n_shared
+    blobs = synth.make_all_blobs(cfg, seed)
+    W, b = synth.make_router(cfg, seed)
+    W_dev, b_dev = torch.from_numpy(W).cuda(), torch.from_numpy(b).cuda()
+    shared = torch.from_numpy(blobs[E:]).cuda()
+    pool = torch.from_numpy(np.ascontiguousarray(blobs[:E]).reshape(-1)).pin_memory()
+    B_e = synth.expert_bytes(cfg.hidden, cfg.inter)
+    arena_mem = torch.empty(cfg.n_slots * B_e, dtype=torch.uint8, device="cuda")
+    x = torch.from_numpy(synth.make_x(cfg, T, seed).view(np.int16)).cuda().view(torch.bfloat16)
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    copy_stream = torch.cuda.Stream()
+    recs = []
+    for chunk in CHUNKS:
+        layer = binding.StrataMoE(cfg.hidden, cfg.inter, E, cfg.top_k, S, cfg.n_slots)
+        layer.set_router(W_dev, b_dev)
+        for i in range(S):
+            layer.bind_shared(i, shared[i])
+        layer.reserve(T)
+        arena = binding.Arena(layer, pool, arena_mem)
+        arena.prefill(x, chunk, out, copy_stream=copy_stream)      # warm-up
+        torch.cuda.synchronize()
+        tot = {"ms": 0.0, "bytes": 0, "misses": 0, "hits": 0, "passes": 0, "chunks": 0}
+        c0 = clocks.mark()
+        for i in range(steps):
+            flush_l2(i)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            st = arena.prefill(x, chunk, out, copy_stream=copy_stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot["ms"] += e0.elapsed_time(e1)
+            for key in ("bytes", "misses", "hits", "passes", "chunks"):
+                tot[key] += st[key]
+        st, bits = layer.status()
+        if int(st) != 0:
+            raise RuntimeError("chunked prefill status %s bits %d" % (st, bits))
+        ms = tot["ms"] / steps
+        recs.append({"chunk_tokens": chunk, "tokens": T, "n_slots": cfg.n_slots,
+                     "ms_per_step": ms, "value": T / (ms / 1000.0), "unit": UNIT,
+                     "copy_bytes_per_step": tot["bytes"] / steps,
+                     "expert_copies_per_step": tot["misses"] / steps,
+                     "resident_hits_per_step": tot["hits"] / steps,
+                     "expert_groups_per_step": tot["passes"] / steps,
+                     "chunks_per_step": tot["chunks"] / steps,
+                     "clocks": clocks.window(c0, clocks.mark())})
+        arena.close()
+        layer.close()
+    return {"workload": cfg.description, "note": "device time of a whole prompt per chunk size, "
+            "copies included (the arena starts each timed prompt with what the previous one "
+            "left)", "records": recs}
+
+
 def main(argv=None):
     args = parse(argv)
     if args.impl == "reference":
@@ -610,7 +674,7 @@ def main(argv=None):
         wl.close()
         del wl
         torch.cuda.empty_cache()
-        subs = []
+        subs, chunked = [], None
         if args.subrecords:
             for name, t in SUBRECORDS:
                 c = synth.CONFIGS[name]
@@ -622,6 +686,9 @@ def main(argv=None):
                 w.close()
                 del w
                 torch.cuda.empty_cache()
+            chunked = measure_chunked(synth.CONFIGS["prefill_paged"], HEADLINE[1], args.seed,
+                                      3, flush_l2, clocks)
+            torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
@@ -647,6 +714,7 @@ def main(argv=None):
                            "host memory" % (cfg.n_slots, cfg.n_experts)
         if subs:
             line["decode"] = subs
+            line["chunked_prefill"] = chunked
             s0 = clocks.mark()
             line["clocks_whole_run"] = clocks.window(0, s0)
         print(json.dumps(line))

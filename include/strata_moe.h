@@ -284,6 +284,35 @@ strata_status strata_arena_copy_ms(strata_arena *a, float *ms);
 /* Slot holding expert_id, -1 if it is not resident, -2 if out of range. */
 int strata_arena_slot_of(const strata_arena *a, int expert_id);
 
+/* Prefill through the arena in chunks, for a layer whose experts do not all
+ * fit its slots ("Strata on a Mac", "Unsloth's UD-Q4/Q5/Q6_K_XL on the M5
+ * Max": prompts stream in chunks of 4096 tokens, and every chunk makes one
+ * pass over the experts that are not in the arena; "Switches": the chunk size
+ * is a setting).  Every token is routed once; then, chunk by chunk of
+ * chunk_tokens tokens, the chunk's distinct experts -- those already
+ * resident first -- are made resident in groups of at most n_slots
+ * (strata_arena_ensure, LRU), each group's share of the chunk's expert work
+ * runs on the tensor cores, and the chunk's output is combined.  Larger
+ * chunks re-read fewer experts; each chunk needs one group per n_slots of its
+ * distinct experts.  x_bf16 and out_bf16: device bf16 [n_tokens][hidden].
+ * The result equals strata_moe_forward's on the same tokens bit for bit when
+ * n_tokens > 64 (every chunk, of any size, takes the tensor-core path that
+ * the forward takes for more than 64 tokens).  Synchronises `stream` once
+ * (to read the routing on the host); may grow the layer's workspace and a
+ * pinned host buffer of the arena.  stats (may be NULL): chunks, groups run,
+ * experts found resident, copied, and bytes copied.  Errors: INVALID_ARG, OOM,
+ * CUDA, and those of strata_arena_ensure; device errors as for forward. */
+typedef struct {
+  int chunks;   /* chunks of the prompt */
+  int passes;   /* expert groups run over all chunks */
+  int hits;     /* experts already resident when their group ran */
+  int misses;   /* experts copied in */
+  size_t bytes; /* bytes copied host -> device */
+} strata_prefill_stats;
+strata_status strata_arena_prefill(strata_arena *a, const void *x_bf16, int n_tokens,
+                                   int chunk_tokens, void *out_bf16, strata_stream_t stream,
+                                   strata_stream_t copy_stream, strata_prefill_stats *stats);
+
 /* Size of the fixed device scratch of strata_moe_forward_noalloc, and the
  * most tokens one call of it takes. */
 #define STRATA_NOALLOC_SCRATCH_BYTES (16u << 20)

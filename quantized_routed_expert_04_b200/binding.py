@@ -37,6 +37,11 @@ class ArenaStats(ctypes.Structure):
     _fields_ = [("hits", ctypes.c_int), ("misses", ctypes.c_int), ("bytes", ctypes.c_size_t)]
 
 
+class PrefillStats(ctypes.Structure):
+    _fields_ = [("chunks", ctypes.c_int), ("passes", ctypes.c_int), ("hits", ctypes.c_int),
+                ("misses", ctypes.c_int), ("bytes", ctypes.c_size_t)]
+
+
 class StrataError(RuntimeError):
     def __init__(self, status, where=""):
         self.status = Status(status)
@@ -76,6 +81,7 @@ def load_library():
             "strata_arena_ensure": (I, [P, P, I, P, P, ctypes.POINTER(ArenaStats)]),
             "strata_arena_copy_ms": (I, [P, ctypes.POINTER(ctypes.c_float)]),
             "strata_arena_slot_of": (I, [P, I]),
+            "strata_arena_prefill": (I, [P, P, I, I, P, P, P, ctypes.POINTER(PrefillStats)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -243,6 +249,16 @@ def strata_arena_slot_of(a, expert_id):
     return int(_load().strata_arena_slot_of(a, expert_id))
 
 
+def strata_arena_prefill(a, x, n_tokens, chunk_tokens, out, stream=None, copy_stream=None):
+    """Chunked prefill through the arena; returns its stats as a dict."""
+    st = PrefillStats()
+    _check(_load().strata_arena_prefill(a, _addr(x), n_tokens, chunk_tokens, _addr(out),
+                                        _stream(stream), _stream(copy_stream), ctypes.byref(st)),
+           "strata_arena_prefill")
+    return {"chunks": st.chunks, "passes": st.passes, "hits": st.hits, "misses": st.misses,
+            "bytes": int(st.bytes)}
+
+
 class Arena:
     """Owning wrapper of an expert arena over a StrataMoE layer."""
 
@@ -258,6 +274,9 @@ class Arena:
 
     def slot_of(self, expert_id):
         return strata_arena_slot_of(self.a, expert_id)
+
+    def prefill(self, x, chunk_tokens, out, stream=None, copy_stream=None):
+        return strata_arena_prefill(self.a, x, x.shape[0], chunk_tokens, out, stream, copy_stream)
 
     def close(self):
         if self.a:

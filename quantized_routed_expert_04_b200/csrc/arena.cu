@@ -39,6 +39,8 @@ struct strata_arena {
   uint64_t tick = 0;
   std::vector<char> wanted;        // scratch, per expert
   std::vector<int> ids;            // scratch: distinct requested ids
+  int32_t *idx_host = nullptr;     // pinned: routing of a chunked prefill
+  size_t idx_host_count = 0;
   cudaEvent_t ready = nullptr, copy_start = nullptr, copy_end = nullptr;
   bool copies_recorded = false;
 };
@@ -90,6 +92,7 @@ strata_status strata_arena_create(strata_moe *layer, const void *host_pool, void
 
 void strata_arena_destroy(strata_arena *a) {
   if (!a) return;
+  if (a->idx_host) cudaFreeHost(a->idx_host);
   if (a->ready) cudaEventDestroy(a->ready);
   if (a->copy_start) cudaEventDestroy(a->copy_start);
   if (a->copy_end) cudaEventDestroy(a->copy_end);
@@ -187,6 +190,87 @@ strata_status strata_arena_copy_ms(strata_arena *a, float *ms) {
 int strata_arena_slot_of(const strata_arena *a, int expert_id) {
   if (!a || expert_id < 0 || expert_id >= a->E) return -2;
   return a->slot_of[expert_id];
+}
+
+strata_status strata_arena_prefill(strata_arena *a, const void *x_bf16, int n_tokens,
+                                   int chunk_tokens, void *out_bf16, strata_stream_t stream,
+                                   strata_stream_t copy_stream, strata_prefill_stats *stats) {
+  if (!a || n_tokens < 0 || chunk_tokens < 1) return STRATA_ERR_INVALID_ARG;
+  if (stats) *stats = strata_prefill_stats{0, 0, 0, 0, 0};
+  if (n_tokens == 0) return STRATA_OK;
+  if (!x_bf16 || !out_bf16 || (reinterpret_cast<uintptr_t>(x_bf16) & 15) ||
+      (reinterpret_cast<uintptr_t>(out_bf16) & 15))
+    return STRATA_ERR_INVALID_ARG;
+  int H, I, E, n_slots, device;
+  strata_handle_shape(a->layer, &H, &I, &E, &n_slots, &device);
+  const int k = strata_handle_top_k(a->layer);
+  // 1. every token's routing, read back to the host
+  const int32_t *idx_dev = nullptr;
+  const float *w_dev = nullptr;
+  strata_status st = strata_layer_route_all(a->layer, x_bf16, n_tokens, stream, &idx_dev, &w_dev);
+  if (st != STRATA_OK) return st;
+  const size_t n_idx = (size_t)n_tokens * k;
+  if (a->idx_host_count < n_idx) {
+    if (a->idx_host) cudaFreeHost(a->idx_host);
+    a->idx_host = nullptr;
+    a->idx_host_count = 0;
+    cudaError_t e = cudaMallocHost(&a->idx_host, n_idx * sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_err(e);
+    a->idx_host_count = n_idx;
+  }
+  cudaError_t e = cudaMemcpyAsync(a->idx_host, idx_dev, n_idx * sizeof(int32_t),
+                                  cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_err(e);
+  // 2. chunks: the chunk's experts, those already resident first, in groups
+  // that fit the slots; one arena request and one tensor-core pass per group
+  std::vector<unsigned char> in_pass(E, 0);
+  std::vector<int> order, group;
+  const char *xb = static_cast<const char *>(x_bf16);
+  char *ob = static_cast<char *>(out_bf16);
+  for (int t0 = 0; t0 < n_tokens; t0 += chunk_tokens) {
+    const int Tc = std::min(chunk_tokens, n_tokens - t0);
+    const int32_t *ci = a->idx_host + (size_t)t0 * k;
+    order.clear();
+    for (int q = 0; q < Tc * k; ++q) {
+      const int ex = ci[q];
+      if (ex < 0 || ex >= E) return STRATA_ERR_DEVICE_STATUS;
+      if (!in_pass[ex]) {
+        in_pass[ex] = 1;
+        order.push_back(ex);
+      }
+    }
+    for (int ex : order) in_pass[ex] = 0;
+    std::stable_sort(order.begin(), order.end(), [&](int p, int q) {
+      const bool rp = a->slot_of[p] >= 0, rq = a->slot_of[q] >= 0;
+      return rp != rq ? rp : p < q;
+    });
+    st = strata_layer_chunk_prepare(a->layer, xb + (size_t)t0 * H * 2, Tc, idx_dev + (size_t)t0 * k,
+                                    stream);
+    if (st != STRATA_OK) return st;
+    for (size_t g0 = 0; g0 < order.size() || g0 == 0; g0 += n_slots) {
+      group.assign(order.begin() + g0, order.begin() + std::min(order.size(), g0 + n_slots));
+      strata_arena_stats as{0, 0, 0};
+      st = strata_arena_ensure(a, group.data(), (int)group.size(), stream, copy_stream, &as);
+      if (st != STRATA_OK) return st;
+      for (int ex : group) in_pass[ex] = 1;
+      st = strata_layer_chunk_pass(a->layer, Tc, in_pass.data(), g0 == 0, stream);
+      for (int ex : group) in_pass[ex] = 0;
+      if (st != STRATA_OK) return st;
+      if (stats) {
+        stats->passes += 1;
+        stats->hits += as.hits;
+        stats->misses += as.misses;
+        stats->bytes += as.bytes;
+      }
+      if (order.empty()) break;
+    }
+    st = strata_layer_chunk_finish(a->layer, Tc, idx_dev + (size_t)t0 * k, w_dev + (size_t)t0 * k,
+                                   ob + (size_t)t0 * H * 2, stream);
+    if (st != STRATA_OK) return st;
+    if (stats) stats->chunks += 1;
+  }
+  return STRATA_OK;
 }
 
 }  // extern "C"

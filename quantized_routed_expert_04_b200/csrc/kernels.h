@@ -39,8 +39,8 @@ struct SmallRouteParams {
 __global__ void route_small_kernel(SmallRouteParams p);
 
 __global__ void combine_kernel(const float *y, const int32_t *idx, const float *w,
-                               const int *inv, ExpertTable table, int T, int H, int k, int S,
-                               int E, __nv_bfloat16 *out);
+                               const int *inv, ExpertTable table, int check_bound, int T, int H,
+                               int k, int S, int E, __nv_bfloat16 *out);
 
 // ---- the whole small-batch layer in one persistent launch (decode_fused.cu)
 //
@@ -91,6 +91,7 @@ struct TcParams {
   __half *h_out;
   float *y_out;
   int *status;
+  int quiet_unbound;  // 1: experts without a blob are left to another pass, not reported
 };
 }  // namespace strata
 #include <cuda.h>

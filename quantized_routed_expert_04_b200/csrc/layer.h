@@ -71,3 +71,21 @@ struct strata_moe;
 // the public calls): hidden, inter, routed experts, arena slots, device.
 void strata_handle_shape(const strata_moe *h, int *hidden, int *inter, int *n_experts,
                          int *n_slots, int *device);
+int strata_handle_top_k(const strata_moe *h);
+
+// Prefill in chunks over an arena with fewer slots than experts (called by
+// the arena): route every token once (idx/w stay in the layer's workspace),
+// then per chunk of Tc tokens: pack + bucket + gather, one tensor-core pass
+// per group of experts that fit the slots (in_pass[e] marks the group; the
+// shared experts run with the first group), and the combine.  Each pair's
+// result does not depend on the pass that computes it, so the output equals
+// the all-resident forward's.  Chunks always take the tensor-core path.
+#include "strata_moe.h"
+strata_status strata_layer_route_all(strata_moe *h, const void *x, int T, cudaStream_t stream,
+                                     const int32_t **idx, const float **w);
+strata_status strata_layer_chunk_prepare(strata_moe *h, const void *x, int Tc, const int32_t *idx,
+                                         cudaStream_t stream);
+strata_status strata_layer_chunk_pass(strata_moe *h, int Tc, const unsigned char *in_pass,
+                                      bool shared, cudaStream_t stream);
+strata_status strata_layer_chunk_finish(strata_moe *h, int Tc, const int32_t *idx, const float *w,
+                                        void *out, cudaStream_t stream);

@@ -139,13 +139,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   grid_dependency_wait();
 
-  // active experts and tiles per expert (prefix), in shared memory
+  // active experts and tiles per expert (prefix), in shared memory; an
+  // active expert without a blob gets no tiles (and is reported, unless the
+  // call runs one expert pass of several)
   const int n_active = *p.rt.n_active;
   for (int a = threadIdx.x; a < n_active; a += blockDim.x) {
     const int id = p.rt.active[a];
     t_blob[a] = p.table.ptr[id];
     t_off[a] = p.rt.off[id];
     t_cnt[a] = p.rt.cnt[id];
+    if (!t_blob[a] && !p.quiet_unbound && blockIdx.x == 0) set_status(p.status, STATUS_NOT_BOUND);
   }
   tc_fence_before();
   __syncthreads();
@@ -155,7 +158,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int carry = 0;
     for (int a0 = 0; a0 < n_active; a0 += 32) {
       const int a = a0 + lane;
-      const int v = a < n_active ? ((t_cnt[a] + kTcN - 1) / kTcN) * p.row_tiles : 0;
+      const int v = a < n_active && t_blob[a] ? ((t_cnt[a] + kTcN - 1) / kTcN) * p.row_tiles : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -183,15 +186,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     un.blob = t_blob[a];
     return un;
   };
-  // unbound experts: skipped by every role, flagged once
-  auto next_unit = [&](int u, int &a) -> int {
-    for (; u < n_units; u += gridDim.x) {
-      while (unit_base[a + 1] <= u) ++a;
-      if (t_blob[a]) return u;
-      if (threadIdx.x == 0) set_status(p.status, STATUS_NOT_BOUND);
-    }
-    return n_units;
-  };
+  // tiles are interleaved over the CTAs (every tile belongs to a bound expert)
+  auto next_unit = [&](int u, int &) -> int { return min(u, n_units); };
 
   if (warp == 0) {
     // -------------------------------------------------------- activation producer

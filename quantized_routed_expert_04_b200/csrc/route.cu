@@ -246,12 +246,12 @@ __global__ void __launch_bounds__(256) bucket_fill_kernel(const int32_t *__restr
 
 // ---------------------------------------------------------------- combine
 // out[t][r] = bf16( sum_j w[t][j] * y[inv[t][j]][r] + sum_s y[inv[t][k+s]][r] )
-// in fp32, in that order.  A token with an unbound or invalid expert gets a
-// zero row.  Each thread handles 4 consecutive r.
+// in fp32, in that order.  A token with an invalid expert (or, with
+// check_bound, an unbound one) gets a zero row.  Each thread handles 4 consecutive r.
 __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ idx,
                                const float *__restrict__ w, const int *__restrict__ inv,
-                               ExpertTable table, int T, int H, int k, int S, int E,
-                               __nv_bfloat16 *__restrict__ out) {
+                               ExpertTable table, int check_bound, int T, int H, int k, int S,
+                               int E, __nv_bfloat16 *__restrict__ out) {
   grid_dependency_wait();
   const int t = blockIdx.y;
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
@@ -260,7 +260,8 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
   bool ok = true;
   for (int j = 0; j < k; ++j) {
     const int e = idx[(size_t)t * k + j];
-    if (e < 0 || e >= E || !table.ptr[e] || inv[(size_t)t * kS + j] < 0) ok = false;
+    if (e < 0 || e >= E || (check_bound && !table.ptr[e]) || inv[(size_t)t * kS + j] < 0)
+      ok = false;
   }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (ok) {

@@ -232,16 +232,23 @@ bool encode_rows_map(CUtensorMap *m, const __half *base, int K, int rows, int bo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Gather + the two tensor-core passes (large batches).
-strata_status run_tc_experts(strata_moe *h, int T, const ExpertTable &table, cudaStream_t stream) {
+// Activations gathered in sorted pair order (large batches).
+strata_status run_gather(strata_moe *h, int T, cudaStream_t stream) {
   const int P = T * (h->k + h->S);
-  cudaError_t e;
   const int per_row = h->H / 8;
   const long long work = (long long)P * per_row;
   const int gblocks = (int)std::min<long long>((work + 255) / 256, 8LL * h->num_sms);
-  e = launch(h, PH_GATHER, gather_rows_kernel, dim3(gblocks), dim3(256), 0, stream, true, h->x16,
-             h->rt.pair_tok, h->rt.off + (h->E + h->S), h->H, P, h->xp);
-  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch(h, PH_GATHER, gather_rows_kernel, dim3(gblocks), dim3(256), 0, stream,
+                            true, h->x16, h->rt.pair_tok, h->rt.off + (h->E + h->S), h->H, P,
+                            h->xp));
+}
+
+// The two tensor-core passes over the experts that `table` binds.  quiet: the
+// routed experts without a blob belong to another pass of the same batch.
+strata_status run_tc_passes(strata_moe *h, int T, const ExpertTable &table, bool quiet,
+                            cudaStream_t stream) {
+  const int P = T * (h->k + h->S);
+  cudaError_t e;
   const size_t smem = tc_smem_bytes();
   for (int pass = 0; pass < 2; ++pass) {
     const bool gu = pass == 0;
@@ -257,6 +264,7 @@ strata_status run_tc_experts(strata_moe *h, int T, const ExpertTable &table, cud
     p.h_out = h->h16;
     p.y_out = h->y;
     p.status = h->status;
+    p.quiet_unbound = quiet ? 1 : 0;
     CUtensorMap m64, m256;
     if (!encode_rows_map(&m64, gu ? h->xp : h->h16, p.K, P, 64) ||
         !encode_rows_map(&m256, gu ? h->xp : h->h16, p.K, P, 256))
@@ -277,11 +285,9 @@ strata_status check_common(strata_moe *h, const void *x, int T, cudaStream_t) {
   return STRATA_OK;
 }
 
-// Large batches (T > 64): bucketing + the tensor-core expert passes + combine,
-// given idx/w in device memory.
-strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *idx, const float *w,
-                          void *out, cudaStream_t stream) {
-  const ExpertTable table = make_table(h);
+// Activation pack + bucketing of a large batch, given idx in device memory.
+strata_status run_prepare(strata_moe *h, const void *x, int T, const int32_t *idx,
+                          cudaStream_t stream) {
   const int kS = h->k + h->S;
   const int nid = h->E + h->S;
   cudaError_t e = cudaMemsetAsync(h->rt.cnt, 0, sizeof(int) * nid, stream);
@@ -297,13 +303,28 @@ strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *id
   if (e == cudaSuccess)
     e = launch(h, PH_BUCKET, bucket_fill_kernel, dim3(nid), dim3(256), 0, stream, true, idx, T,
                h->k, h->E, h->S, h->rt);
-  if (e != cudaSuccess) return cuda_status(e);
-  const strata_status st = run_tc_experts(h, T, table, stream);
-  if (st != STRATA_OK) return st;
-  dim3 cgrid((h->H / 4 + 127) / 128, T);
-  e = launch(h, PH_COMBINE, combine_kernel, cgrid, dim3(128), 0, stream, true, h->y, idx, w,
-             h->rt.inv, table, T, h->H, h->k, h->S, h->E, static_cast<__nv_bfloat16 *>(out));
   return cuda_status(e);
+}
+
+strata_status run_combine(strata_moe *h, int T, const int32_t *idx, const float *w,
+                          const ExpertTable &table, bool check_bound, void *out,
+                          cudaStream_t stream) {
+  dim3 cgrid((h->H / 4 + 127) / 128, T);
+  return cuda_status(launch(h, PH_COMBINE, combine_kernel, cgrid, dim3(128), 0, stream, true,
+                            h->y, idx, w, h->rt.inv, table, check_bound ? 1 : 0, T, h->H, h->k,
+                            h->S, h->E, static_cast<__nv_bfloat16 *>(out)));
+}
+
+// Large batches (T > 64): bucketing + the tensor-core expert passes + combine,
+// given idx/w in device memory.
+strata_status run_experts(strata_moe *h, const void *x, int T, const int32_t *idx, const float *w,
+                          void *out, cudaStream_t stream) {
+  const ExpertTable table = make_table(h);
+  strata_status st = run_prepare(h, x, T, idx, stream);
+  if (st == STRATA_OK) st = run_gather(h, T, stream);
+  if (st == STRATA_OK) st = run_tc_passes(h, T, table, false, stream);
+  if (st == STRATA_OK) st = run_combine(h, T, idx, w, table, true, out, stream);
+  return st;
 }
 
 SmallRouteParams small_params(strata_moe *h, const void *x, int T, float *logits, int32_t *idx,
@@ -557,6 +578,44 @@ void strata_handle_shape(const strata_moe *h, int *hidden, int *inter, int *n_ex
   *n_experts = h->E;
   *n_slots = h->n_slots;
   *device = h->device;
+}
+
+int strata_handle_top_k(const strata_moe *h) { return h->k; }
+
+strata_status strata_layer_route_all(strata_moe *h, const void *x, int T, cudaStream_t stream,
+                                     const int32_t **idx, const float **w) {
+  if (!h || !x || T <= 0 || !h->router_W) return STRATA_ERR_INVALID_ARG;
+  for (int i = 0; i < h->S; ++i)
+    if (!h->shared_ptr[i]) return STRATA_ERR_INVALID_ARG;
+  // the chunks take the tensor-core path, whose gathered activations exist
+  // only in a workspace for more than kSmallT tokens
+  strata_status st = grow_workspace(h, std::max(T, kSmallT + 1));
+  if (st == STRATA_OK) st = run_router(h, x, T, h->logits, h->idx, h->w, stream);
+  *idx = h->idx;
+  *w = h->w;
+  return st;
+}
+
+strata_status strata_layer_chunk_prepare(strata_moe *h, const void *x, int Tc, const int32_t *idx,
+                                         cudaStream_t stream) {
+  strata_status st = run_prepare(h, x, Tc, idx, stream);
+  if (st == STRATA_OK) st = run_gather(h, Tc, stream);
+  return st;
+}
+
+strata_status strata_layer_chunk_pass(strata_moe *h, int Tc, const unsigned char *in_pass,
+                                      bool shared, cudaStream_t stream) {
+  ExpertTable t = make_table(h);
+  for (int e = 0; e < h->E; ++e)
+    if (!in_pass[e]) t.ptr[e] = nullptr;
+  if (!shared)
+    for (int i = 0; i < h->S; ++i) t.ptr[h->E + i] = nullptr;
+  return run_tc_passes(h, Tc, t, true, stream);
+}
+
+strata_status strata_layer_chunk_finish(strata_moe *h, int Tc, const int32_t *idx, const float *w,
+                                        void *out, cudaStream_t stream) {
+  return run_combine(h, Tc, idx, w, make_table(h), false, out, stream);
 }
 
 extern "C" {

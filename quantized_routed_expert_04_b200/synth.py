@@ -100,6 +100,13 @@ CONFIGS = {
         "sigmoid", 4096, 1024, 256, 10, 0, 256, (1, 4), routing="sigmoid", routed_scale=2.5,
         description="sigmoid-routed decode: hidden 4096, inter 1024, 256 experts top-10, "
                     "correction bias ~N(0, 0.05^2), routed scale 2.5"),
+    # the prefill layer over an arena of half its experts, filled chunk by
+    # chunk (chunked prefill with a partial arena)
+    "prefill_paged": LayerConfig(
+        "prefill_paged", 4096, 2048, 256, 8, 1, 128, (8192,), bias="zipf", zipf_s=0.8,
+        zipf_beta=1.0,
+        description="prefill through a 128-slot arena: hidden 4096, inter 2048, 256 experts "
+                    "top-8 + 1 shared, 8192 tokens, Zipf(0.8) router bias"),
     # the prefill layer's shapes with 32 experts and 2048 tokens: small enough
     # (about 0.5 GB of blobs) for profiler captures and quick parity runs
     "prefill_small": LayerConfig(
