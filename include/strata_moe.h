@@ -112,6 +112,27 @@ void strata_moe_destroy(strata_moe *h);
 /* Size in bytes of one expert blob (the format above) for hidden x inter. */
 size_t strata_moe_expert_bytes(int hidden, int inter);
 
+/* Weight formats of the expert blobs of a layer.
+ * STRATA_FORMAT_INT4 (default): the format described at the top of this file.
+ * STRATA_FORMAT_NVFP4 (ro99/strata README, model table: NVFP4 routed experts,
+ *   E2M1 weights with E4M3 scales per 16 and an fp32 per-tensor global scale,
+ *   run with 16-bit activations): the same sections, tiles and nibble places,
+ *   holding 4-bit E2M1 codes (sign, 2-bit exponent with bias 1, 1-bit
+ *   mantissa: 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives) instead of
+ *   integers; the scale sections hold, per tile row and K group of 128, eight
+ *   E4M3 bytes instead of four fp16 values (byte i scales elements
+ *   16i..16i+15 of the group); and one more 256-byte-aligned section holds
+ *   three fp32 global scales (gate, up, down).  The weight is
+ *   (code value * E4M3 scale) * global scale.  The kernels apply the first
+ *   product exactly in f16 and the global scale once per dot product.
+ * strata_moe_expert_bytes_fmt: blob size in a format (0 for bad arguments).
+ * strata_moe_set_format: the format of the layer's blobs; only while no slot
+ *   and no shared expert is bound (else INVALID_ARG; also for an unknown
+ *   format).  Arenas created afterwards copy blobs of this format's size. */
+enum { STRATA_FORMAT_INT4 = 0, STRATA_FORMAT_NVFP4 = 1 };
+size_t strata_moe_expert_bytes_fmt(int hidden, int inter, int fmt);
+strata_status strata_moe_set_format(strata_moe *h, int fmt);
+
 /* Router weights: W_dev fp32 [n_experts][hidden] row-major (device), bias_dev
  * fp32 [n_experts] (device) or NULL for none.  Pointers must be 16-byte
  * aligned.  Errors: INVALID_ARG. */
@@ -175,9 +196,9 @@ strata_status strata_moe_route(strata_moe *h, const void *x_bf16, int n_tokens, 
  * Range: the kernels feed the tensor cores f16 operands, so activations and
  * the SwiGLU output h must stay below 65520 in magnitude (larger values round
  * to an f16 infinity), and with more than 64 tokens (the tensor-core path,
- * which dequantises each weight to f16(q * scale)) every fp16 scale of a
- * routed or shared expert must be below 8192 in magnitude (8 * 8192 would
- * overflow).  A value beyond these limits is detected on the device and
+ * which dequantises each int4 weight to f16(q * scale)) every fp16 scale of a
+ * routed or shared int4 expert must be below 8192 in magnitude (8 * 8192
+ * would overflow; NVFP4 weights before the global scale are at most 2688).  A value beyond these limits is detected on the device and
  * reported as STRATA_ERR_RANGE by strata_moe_get_status (the affected outputs
  * are then not meaningful); with up to 64 tokens scales of any finite fp16
  * value are applied exactly in fp32.

@@ -60,6 +60,8 @@ def load_library():
             "strata_moe_create": (I, [I, I, I, I, I, I, ctypes.POINTER(P)]),
             "strata_moe_destroy": (None, [P]),
             "strata_moe_expert_bytes": (Z, [I, I]),
+            "strata_moe_expert_bytes_fmt": (Z, [I, I, I]),
+            "strata_moe_set_format": (I, [P, I]),
             "strata_moe_set_router": (I, [P, P, P]),
             "strata_moe_bind_shared": (I, [P, I, P]),
             "strata_moe_set_routing": (I, [P, I, P, ctypes.c_float]),
@@ -129,6 +131,17 @@ def strata_moe_destroy(h):
 
 def strata_moe_expert_bytes(hidden, inter):
     return int(_load().strata_moe_expert_bytes(hidden, inter))
+
+
+FORMAT_INT4, FORMAT_NVFP4 = 0, 1
+
+
+def strata_moe_expert_bytes_fmt(hidden, inter, fmt):
+    return int(_load().strata_moe_expert_bytes_fmt(hidden, inter, fmt))
+
+
+def strata_moe_set_format(h, fmt):
+    _check(_load().strata_moe_set_format(h, int(fmt)), "strata_moe_set_format")
 
 
 def strata_moe_set_router(h, W, bias=None):
@@ -311,6 +324,9 @@ class StrataMoE:
 
     def set_router(self, W, bias=None):
         strata_moe_set_router(self.h, W, bias)
+
+    def set_format(self, fmt):
+        strata_moe_set_format(self.h, fmt)
 
     def set_routing(self, mode, corr=None, routed_scale=1.0):
         strata_moe_set_routing(self.h, mode, corr, routed_scale)

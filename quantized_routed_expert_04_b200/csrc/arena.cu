@@ -70,7 +70,7 @@ strata_status strata_arena_create(strata_moe *layer, const void *host_pool, void
   a->layer = layer;
   a->pool = static_cast<const uint8_t *>(host_pool);
   a->arena = static_cast<uint8_t *>(arena_dev);
-  a->blob_bytes = strata_moe_expert_bytes(H, I);
+  a->blob_bytes = strata_handle_blob_bytes(layer);
   a->E = E;
   a->n_slots = n_slots;
   a->slot_of.assign(E, -1);

@@ -17,10 +17,12 @@ __device__ __forceinline__ void set_status(int *status, int bit) {
   if (status) atomicOr(status, bit);
 }
 
-// Eight bf16 activations -> eight f16 stored in the order 0,4,1,5,2,6,3,7
-// (the order in which int4x8_to_f16 produces weight pairs, so that one
-// 16-byte load gives a thread its four mma B-fragment registers).  Sets
-// `overflow` if a finite or infinite input rounds to an f16 infinity.
+// Eight bf16 activations -> eight f16, in the order in which the format's
+// weight conversion produces weight pairs (so that one 16-byte load gives a
+// thread its four mma B-fragment registers): 0,4,1,5,2,6,3,7 for int4
+// (int4x8_to_f16), 0..7 for NVFP4 (e2m1x8_to_f16).  Sets `overflow` if an
+// input rounds to an f16 infinity.
+template <int FMT>
 __device__ __forceinline__ uint4 pack8_bf16_to_f16(uint4 raw, bool &overflow) {
   const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&raw);
   const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
@@ -30,11 +32,48 @@ __device__ __forceinline__ uint4 pack8_bf16_to_f16(uint4 raw, bool &overflow) {
   overflow = m >= kF16Overflow;
   uint4 o;
   __half2 h;
-  h = __floats2half2_rn(f0.x, f2.x); o.x = *reinterpret_cast<uint32_t *>(&h);
-  h = __floats2half2_rn(f0.y, f2.y); o.y = *reinterpret_cast<uint32_t *>(&h);
-  h = __floats2half2_rn(f1.x, f3.x); o.z = *reinterpret_cast<uint32_t *>(&h);
-  h = __floats2half2_rn(f1.y, f3.y); o.w = *reinterpret_cast<uint32_t *>(&h);
+  if (FMT == kFmtInt4) {
+    h = __floats2half2_rn(f0.x, f2.x); o.x = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2half2_rn(f0.y, f2.y); o.y = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2half2_rn(f1.x, f3.x); o.z = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2half2_rn(f1.y, f3.y); o.w = *reinterpret_cast<uint32_t *>(&h);
+  } else {
+    h = __floats2half2_rn(f0.x, f0.y); o.x = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2half2_rn(f1.x, f1.y); o.y = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2half2_rn(f2.x, f2.y); o.z = *reinterpret_cast<uint32_t *>(&h);
+    h = __floats2half2_rn(f3.x, f3.y); o.w = *reinterpret_cast<uint32_t *>(&h);
+  }
   return o;
+}
+
+// Position of element i (of a row of packed 16-bit activations or SwiGLU
+// outputs) in the format's pair order (see pack8_bf16_to_f16).
+template <int FMT>
+__device__ __forceinline__ int packed_pos(int i) {
+  return FMT == kFmtInt4 ? (i & ~7) | (((i & 3) << 1) | ((i >> 2) & 1)) : i;
+}
+
+// Eight E2M1 codes in one 32-bit word (code e in bits 4e..4e+3) -> four
+// f16x2 registers holding their exact values: out[j] = (code 2j, code 2j+1),
+// low half first (the conversion instruction of sm_100a, one per byte).
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t out[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(w));
+}
+
+// One E4M3 byte (the low byte of `byte`) -> f16x2 holding its exact value
+// twice.
+__device__ __forceinline__ uint32_t e4m3_to_f16x2_dup(uint32_t byte) {
+  const uint16_t v = (uint16_t)((byte & 0xFFu) * 0x101u);
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(v));
+  return d;
 }
 
 // ---------------------------------------------------------------- addresses

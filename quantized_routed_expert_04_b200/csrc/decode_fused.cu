@@ -38,9 +38,12 @@
 // ring of shared-memory stages filled by bulk async copies; the ring runs on
 // from the G share into the D share, so the down weights are in flight while
 // the grid waits at the barrier between the phases.  The int4 words go from
-// shared memory into mma.m16n8k16 A fragments (int4x8_to_f16, exact), two
-// MMAs per quant block, fp32 block-scale FMAs: the weights are applied
-// exactly, the activations are f16.
+// shared memory into mma.m16n8k16 A fragments.  int4: int4x8_to_f16 (exact
+// integers), two MMAs per quant block, fp32 block-scale FMAs.  NVFP4: each
+// code times its E4M3 group scale in f16 (exact: at most six significant
+// bits, at most 2688 in magnitude), MMAs chained over the whole piece, and
+// the fp32 global scale once at the end.  Either way the weights are applied
+// exactly; the activations are f16.
 // An item cut by share boundaries is finished by the last of its pieces to
 // arrive: every piece stores its partial sums, counts itself on the item's
 // counter, and the piece that completes the count adds all pieces' sums in
@@ -289,7 +292,7 @@ __device__ void combine_tile(const FusedParams &p, const Tables &tb, int tau, in
 // One phase's compute: this warp's pieces in order, consuming the ring
 // stages that issue_next filled.  Returns false if a wait gave up (the ring
 // is drained first).
-template <bool kGateUp, int NT>
+template <bool kGateUp, int NT, int FMT>
 __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInfo *ph, int phi,
                           Ring &rg, Cursor &cur, int wg, int lane, int gpc, int kc) {
   const PhaseInfo &P = ph[phi];
@@ -313,15 +316,31 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
     }
   };
   bool any_big = false;
+  // NVFP4: the global scales (gate, up, down) of an item's expert multiply
+  // its sums once at the end
+  auto globals = [&](const Item &it, float &s_lo, float &s_hi) {
+    if (FMT == kFmtNvfp4) {
+      const float *gs = reinterpret_cast<const float *>(it.blob + p.glob);
+      s_lo = kGateUp ? gs[0] : gs[2];
+      s_hi = kGateUp ? gs[1] : gs[2];
+    } else {
+      s_lo = s_hi = 1.0f;
+    }
+  };
   // Output of one (pair n, row g / g + 8) element pair of an item.
   auto emit = [&](const Item &it, int n, float lo, float hi) {
     const size_t prow = (size_t)(it.pi0 + n);
+    if (FMT == kFmtNvfp4) {
+      float s_lo, s_hi;
+      globals(it, s_lo, s_hi);
+      lo *= s_lo;
+      hi *= s_hi;
+    }
     if (kGateUp) {
       // lo: gate row i, hi: up row i, i = 8 tau + g; stored like the packed
-      // activations (groups of 8 in the order 0,4,1,5,2,6,3,7)
+      // activations (the format's pair order)
       const float h = lo / (1.0f + expf(-lo)) * hi;
-      const int ii = it.tau * 8 + g;
-      const int pos = (ii & ~7) | (((ii & 3) << 1) | ((ii >> 2) & 1));
+      const int pos = packed_pos<FMT>(it.tau * 8 + g);
       any_big |= fabsf(h) >= kF16Overflow;
       p.h16[prow * p.I + pos] = __float2half_rn(h);
     } else {
@@ -383,6 +402,14 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
     float2 acc[NT][2];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = make_float2(0.0f, 0.0f);
+    // NVFP4: two chained MMA accumulators per n-tile (even and odd blocks)
+    float acc4[NT][2][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc4[n][h][i] = 0.0f;
 
     for (int cg = pc.g0; cg < pc.g1; ++rg.used) {
       const int slot = (int)(rg.used % rg.stages);
@@ -415,41 +442,69 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
         const uint32_t wr0[4] = {w0.x, w0.y, w0.z, w0.w};
         const uint32_t wr1[4] = {w1.x, w1.y, w1.z, w1.w};
         uint32_t f0[4][4], f1[4][4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          int4x8_to_f16(wr0[b], f0[b]);
-          int4x8_to_f16(wr1[b], f1[b]);
-        }
         float sc0[4], sc1[4];
-        {
+        if (FMT == kFmtInt4) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            int4x8_to_f16(wr0[b], f0[b]);
+            int4x8_to_f16(wr1[b], f1[b]);
+          }
           float2 f;
           f = __half22float2(bits_h2(s0.x)); sc0[0] = f.x; sc0[1] = f.y;
           f = __half22float2(bits_h2(s0.y)); sc0[2] = f.x; sc0[3] = f.y;
           f = __half22float2(bits_h2(s1.x)); sc1[0] = f.x; sc1[1] = f.y;
           f = __half22float2(bits_h2(s1.y)); sc1[2] = f.x; sc1[3] = f.y;
+        } else {
+          // word cq of block b holds elements 32 b + 8 cq .. + 7: scale group
+          // 2 b + cq / 2 (byte of the row's eight); code x scale is exact in f16
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int sel = 2 * b + (cq >> 1);
+            const uint32_t b0 = (sel < 4 ? s0.x : s0.y) >> (8 * (sel & 3));
+            const uint32_t b1 = (sel < 4 ? s1.x : s1.y) >> (8 * (sel & 3));
+            const __half2 z0 = bits_h2(e4m3_to_f16x2_dup(b0));
+            const __half2 z1 = bits_h2(e4m3_to_f16x2_dup(b1));
+            e2m1x8_to_f16(wr0[b], f0[b]);
+            e2m1x8_to_f16(wr1[b], f1[b]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              f0[b][i] = h2_bits(__hmul2(bits_h2(f0[b][i]), z0));
+              f1[b][i] = h2_bits(__hmul2(bits_h2(f1[b][i]), z1));
+            }
+          }
         }
         auto mma_group = [&](const uint4 (&bv)[NT][4]) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             if (NT == 1 || nt < ntn) {
-              float d[4][4];
-              const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+              if (FMT == kFmtInt4) {
+                float d[4][4];
+                const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                const uint32_t a0[4] = {f0[b][0], f1[b][0], f0[b][1], f1[b][1]};
-                mma_16816(d[b], a0, bv[nt][b].x, bv[nt][b].y, zero);
-              }
+                for (int b = 0; b < 4; ++b) {
+                  const uint32_t a0[4] = {f0[b][0], f1[b][0], f0[b][1], f1[b][1]};
+                  mma_16816(d[b], a0, bv[nt][b].x, bv[nt][b].y, zero);
+                }
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                const uint32_t a1[4] = {f0[b][2], f1[b][2], f0[b][3], f1[b][3]};
-                mma_16816(d[b], a1, bv[nt][b].z, bv[nt][b].w, d[b]);
-              }
+                for (int b = 0; b < 4; ++b) {
+                  const uint32_t a1[4] = {f0[b][2], f1[b][2], f0[b][3], f1[b][3]};
+                  mma_16816(d[b], a1, bv[nt][b].z, bv[nt][b].w, d[b]);
+                }
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                acc[nt][0] = __ffma2_rn(make_float2(sc0[b], sc0[b]),
-                                        make_float2(d[b][0], d[b][1]), acc[nt][0]);
-                acc[nt][1] = __ffma2_rn(make_float2(sc1[b], sc1[b]),
-                                        make_float2(d[b][2], d[b][3]), acc[nt][1]);
+                for (int b = 0; b < 4; ++b) {
+                  acc[nt][0] = __ffma2_rn(make_float2(sc0[b], sc0[b]),
+                                          make_float2(d[b][0], d[b][1]), acc[nt][0]);
+                  acc[nt][1] = __ffma2_rn(make_float2(sc1[b], sc1[b]),
+                                          make_float2(d[b][2], d[b][3]), acc[nt][1]);
+                }
+              } else {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  const uint32_t a0[4] = {f0[b][0], f1[b][0], f0[b][1], f1[b][1]};
+                  const uint32_t a1[4] = {f0[b][2], f1[b][2], f0[b][3], f1[b][3]};
+                  mma_16816(acc4[nt][b & 1], a0, bv[nt][b].x, bv[nt][b].y, acc4[nt][b & 1]);
+                  mma_16816(acc4[nt][b & 1], a1, bv[nt][b].z, bv[nt][b].w, acc4[nt][b & 1]);
+                }
               }
             }
           }
@@ -464,6 +519,13 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       issue_next(cur, rg, tb, ph, p.group, gpc, kc, lane);
     }
     if (!ok) break;
+    if (FMT == kFmtNvfp4) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        acc[nt][0] = make_float2(acc4[nt][0][0] + acc4[nt][1][0], acc4[nt][0][1] + acc4[nt][1][1]);
+        acc[nt][1] = make_float2(acc4[nt][0][2] + acc4[nt][1][2], acc4[nt][0][3] + acc4[nt][1][3]);
+      }
+    }
 
     // ---- epilogue
     if (pc.g0 == 0 && pc.g1 == G) {
@@ -553,7 +615,7 @@ size_t fused_table_bytes(int T, int k, int S) {
   return (b + 127) / 128 * 128 + 128;
 }
 
-template <int NT>
+template <int NT, int FMT>
 __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -601,7 +663,8 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     bool over = false;
     for (int i = blockIdx.x * blockDim.x + tid; i < n8; i += gridDim.x * blockDim.x) {
       bool o;
-      const uint4 v = pack8_bf16_to_f16(*reinterpret_cast<const uint4 *>(p.x + (size_t)i * 8), o);
+      const uint4 v =
+          pack8_bf16_to_f16<FMT>(*reinterpret_cast<const uint4 *>(p.x + (size_t)i * 8), o);
       over |= o;
       *reinterpret_cast<uint4 *>(p.x16 + (size_t)i * 8) = v;
     }
@@ -816,11 +879,11 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     cur.have = piece_at(tb, ph[0], cur.x, cur.a, cur.pc);
     if (cur.have) cur.cg = cur.pc.g0;
     for (int s = 0; s < rg.stages; ++s) issue_next(cur, rg, tb, ph, p.group, gpc, p.kc, lane);
-    if (!run_phase<true, NT>(p, tb, ph, 0, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
+    if (!run_phase<true, NT, FMT>(p, tb, ph, 0, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
   }
   live = grid_sync(p.bar + 2, abort_flag, p.status, p.wait_ns) && live;
   if (live) {
-    if (!run_phase<false, NT>(p, tb, ph, 1, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
+    if (!run_phase<false, NT, FMT>(p, tb, ph, 1, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
     // no combine happens if no expert item ran at all: every token is then
     // one with an unbound expert, and its output row is zero
     if (blockIdx.x == 0 && tb.misc[1] == 0)
@@ -843,7 +906,9 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   }
 }
 
-template __global__ void decode_fused_kernel<1>(FusedParams);
-template __global__ void decode_fused_kernel<2>(FusedParams);
+template __global__ void decode_fused_kernel<1, kFmtInt4>(FusedParams);
+template __global__ void decode_fused_kernel<2, kFmtInt4>(FusedParams);
+template __global__ void decode_fused_kernel<1, kFmtNvfp4>(FusedParams);
+template __global__ void decode_fused_kernel<2, kFmtNvfp4>(FusedParams);
 
 }  // namespace strata

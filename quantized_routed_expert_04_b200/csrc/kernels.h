@@ -20,7 +20,8 @@ struct RouteMode {
 };
 __global__ void topk_kernel(const float *logits, int T, int E, int k, RouteMode mode,
                             int32_t *idx, float *w);
-__global__ void pack_x_kernel(const __nv_bfloat16 *x, int n8, __half *x16, int *status);
+__global__ void pack_x_kernel(const __nv_bfloat16 *x, int n8, __half *x16, int fmt,
+                              int *status);
 __global__ void bucket_count_kernel(const int32_t *idx, int T, int k, int E, int *cnt,
                                     int *status);
 __global__ void bucket_fill_kernel(const int32_t *idx, int T, int k, int E, int S, Routing rt);
@@ -59,6 +60,7 @@ struct FusedParams {
   const float *w_in;
   int T, H, I, E, k, S;
   size_t guq, gus, dq, ds;  // blob sections
+  size_t glob;              // NVFP4: offset of the three fp32 global scales (gate, up, down)
   int kc;                   // K elements per ring stage (multiple of 128)
   int stages, stage_bytes;  // per-warp ring
   int group;                // pairs per item: 8 or 16
@@ -76,7 +78,7 @@ struct FusedParams {
   int *status;
   __nv_bfloat16 *out;       // [T][H]
 };
-template <int NT>   // NT: 8-pair MMA tiles per item (1 or 2)
+template <int NT, int FMT>   // NT: 8-pair MMA tiles per item (1 or 2); FMT: weight format
 __global__ void decode_fused_kernel(FusedParams p);
 size_t fused_table_bytes(int T, int k, int S);
 
@@ -92,11 +94,12 @@ struct TcParams {
   float *y_out;
   int *status;
   int quiet_unbound;  // 1: experts without a blob are left to another pass, not reported
+  size_t glob_off;    // NVFP4: offset of the three fp32 global scales in a blob
 };
 }  // namespace strata
 #include <cuda.h>
 namespace strata {
-template <bool kGateUp>
+template <bool kGateUp, int FMT>
 __global__ void expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b64,
                                  const __grid_constant__ CUtensorMap tmap_b256);
 __global__ void gather_rows_kernel(const __half *x16, const int *pair_tok, const int *n_pairs_dev,

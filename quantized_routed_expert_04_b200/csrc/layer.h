@@ -27,13 +27,19 @@ enum : int {
 // (65504 is the largest finite f16; half-way to the next power step rounds up).
 constexpr float kF16Overflow = 65520.0f;
 
-// Byte offsets of the four sections of an expert blob: gate+up weights,
-// down weights, gate+up scales, down scales (see include/strata_moe.h).
+// Weight formats of an expert blob (the values of STRATA_FORMAT_*): 4-bit
+// integers with fp16 scales per 32, or NVFP4 (E2M1 codes, E4M3 scales per
+// 16, fp32 global scales).
+enum : int { kFmtInt4 = 0, kFmtNvfp4 = 1 };
+
+// Byte offsets of the sections of an expert blob: gate+up weights, down
+// weights, gate+up scales, down scales, and for NVFP4 the three fp32 global
+// scales (see include/strata_moe.h).
 struct BlobLayout {
-  size_t guq, dq, gus, ds, total;
+  size_t guq, dq, gus, ds, glob, total;
 };
 
-inline BlobLayout blob_layout(int H, int I) {
+inline BlobLayout blob_layout(int H, int I, int fmt = 0) {
   auto up = [](size_t v) { return (v + 255) / 256 * 256; };
   BlobLayout L;
   size_t off = 0;
@@ -41,6 +47,8 @@ inline BlobLayout blob_layout(int H, int I) {
   L.dq = off;  off = up(off + (size_t)H * I / 2);
   L.gus = off; off = up(off + (size_t)I * H / 8);
   L.ds = off;  off = up(off + (size_t)H * I / 16);
+  L.glob = off;
+  if (fmt == kFmtNvfp4) off = up(off + 3 * sizeof(float));
   L.total = off;
   return L;
 }
@@ -72,6 +80,7 @@ struct strata_moe;
 void strata_handle_shape(const strata_moe *h, int *hidden, int *inter, int *n_experts,
                          int *n_slots, int *device);
 int strata_handle_top_k(const strata_moe *h);
+size_t strata_handle_blob_bytes(const strata_moe *h);  // bytes of one blob in the layer's format
 
 // Prefill in chunks over an arena with fewer slots than experts (called by
 // the arena): route every token once (idx/w stay in the layer's workspace),

@@ -27,7 +27,10 @@
 //               commits to the stage barriers and, at the end of a tile, to
 //               the accumulator;
 //   warps 2-9   dequant: int4 -> exact f16 integers -> times the fp16 scale
-//               (one f16 rounding) -> the K-major 128-byte-swizzled A layout;
+//               (one f16 rounding), or NVFP4 E2M1 codes times their E4M3
+//               group scale (exact in f16; the fp32 global scale multiplies
+//               the accumulator in the epilogue) -> the K-major
+//               128-byte-swizzled A layout;
 //   warps 10-13 epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
 //               transposed through shared memory, stored.
 // Both operands are staged one 64-wide swizzle atom at a time in a ring of
@@ -96,7 +99,7 @@ size_t tc_smem_bytes() { return kTcSmem; }
 int tc_threads() { return kTcThreads; }
 static_assert(kTcSmem <= 232448, "shared memory budget");
 
-template <bool kGateUp>
+template <bool kGateUp, int FMT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b64,
                      const __grid_constant__ CUtensorMap tmap_b256) {
@@ -325,22 +328,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 pq + j * (kPkGroups * 1024) + gi * 1024 + tr * 64 + w * 16 + atom * 8);
             const uint32_t sv = *reinterpret_cast<const uint32_t *>(
                 psc + j * (kPkGroups * 128) + gi * 128 + tr * 8 + atom * 4);
-            // |scale| >= 8192 (or not finite): q * scale can overflow f16
-            big_scale |= __vcmpgeu2(sv & 0x7FFF7FFFu, 0x70007000u) != 0u;
             const uint32_t words[2] = {qv.x, qv.y};
-            const __half2 sc[2] = {__half2half2(__low2half(bits_h2(sv))),
-                                   __half2half2(__high2half(bits_h2(sv)))};
+            if (FMT == kFmtInt4) {
+              // |scale| >= 8192 (or not finite): q * scale can overflow f16
+              big_scale |= __vcmpgeu2(sv & 0x7FFF7FFFu, 0x70007000u) != 0u;
+              const __half2 sc[2] = {__half2half2(__low2half(bits_h2(sv))),
+                                     __half2half2(__high2half(bits_h2(sv)))};
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-              uint32_t f[4];
-              int4x8_to_f16(words[b], f);
-              uint4 o;
-              o.x = h2_bits(__hmul2(bits_h2(f[0]), sc[b]));
-              o.y = h2_bits(__hmul2(bits_h2(f[1]), sc[b]));
-              o.z = h2_bits(__hmul2(bits_h2(f[2]), sc[b]));
-              o.w = h2_bits(__hmul2(bits_h2(f[3]), sc[b]));
-              const int chunk = (b * 4 + w) ^ (r & 7);
-              *reinterpret_cast<uint4 *>(ad + r * 128 + chunk * 16) = o;
+              for (int b = 0; b < 2; ++b) {
+                uint32_t f[4];
+                int4x8_to_f16(words[b], f);
+                uint4 o;
+                o.x = h2_bits(__hmul2(bits_h2(f[0]), sc[b]));
+                o.y = h2_bits(__hmul2(bits_h2(f[1]), sc[b]));
+                o.z = h2_bits(__hmul2(bits_h2(f[2]), sc[b]));
+                o.w = h2_bits(__hmul2(bits_h2(f[3]), sc[b]));
+                const int chunk = (b * 4 + w) ^ (r & 7);
+                *reinterpret_cast<uint4 *>(ad + r * 128 + chunk * 16) = o;
+              }
+            } else {
+              // NVFP4: word w of block 2 atom + b is scale group 4 atom + 2 b
+              // + w / 2 (byte 2 b + w / 2 of the four loaded); code x E4M3
+              // scale is exact in f16
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                const __half2 z = bits_h2(e4m3_to_f16x2_dup(sv >> (8 * (2 * b + (w >> 1)))));
+                uint32_t f[4];
+                e2m1x8_to_f16(words[b], f);
+                uint4 o;
+                o.x = h2_bits(__hmul2(bits_h2(f[0]), z));
+                o.y = h2_bits(__hmul2(bits_h2(f[1]), z));
+                o.z = h2_bits(__hmul2(bits_h2(f[2]), z));
+                o.w = h2_bits(__hmul2(bits_h2(f[3]), z));
+                const int chunk = (b * 4 + w) ^ (r & 7);
+                *reinterpret_cast<uint4 *>(ad + r * 128 + chunk * 16) = o;
+              }
             }
           }
           fence_async_smem();
@@ -371,14 +393,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int buf = (int)(t_cnt_local & 1u);
       if (!wwait(&acc_full[buf], (t_cnt_local >> 1) & 1u, p.status)) { ok = false; break; }
       tc_fence_after();
+      // NVFP4: this lane's row's global scale (gate, up or down)
+      float gsc = 1.0f;
+      if (FMT == kFmtNvfp4) {
+        const float *gs = reinterpret_cast<const float *>(un.blob + p.glob_off);
+        gsc = kGateUp ? gs[(lane & 15) < 8 ? 0 : 1] : gs[2];
+      }
       for (int col0 = 0; col0 < un.n; col0 += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * qd) << 16) + buf * kAccCols + col0, v);
+        if (FMT == kFmtNvfp4) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] *= gsc;
+        }
         if (kGateUp) {
           // lane L: blob tile 2 qd + L / 16, tile row L % 16 (gate if < 8)
           __half *hs = reinterpret_cast<__half *>(stage);  // [32 pairs][16]
           const bool gate = (lane & 15) < 8;
-          const int pos16 = 8 * (lane >> 4) + (((lane & 3) << 1) | ((lane >> 2) & 1));
+          const int pos16 = 8 * (lane >> 4) + packed_pos<FMT>(lane & 7);
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             const float up = __shfl_xor_sync(0xffffffffu, v[t], 8);
@@ -440,10 +472,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template __global__ void expert_tc_kernel<true>(TcParams, const __grid_constant__ CUtensorMap,
-                                               const __grid_constant__ CUtensorMap);
-template __global__ void expert_tc_kernel<false>(TcParams, const __grid_constant__ CUtensorMap,
-                                                const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<true, kFmtInt4>(TcParams,
+                                                         const __grid_constant__ CUtensorMap,
+                                                         const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<false, kFmtInt4>(TcParams,
+                                                          const __grid_constant__ CUtensorMap,
+                                                          const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<true, kFmtNvfp4>(TcParams,
+                                                          const __grid_constant__ CUtensorMap,
+                                                          const __grid_constant__ CUtensorMap);
+template __global__ void expert_tc_kernel<false, kFmtNvfp4>(TcParams,
+                                                           const __grid_constant__ CUtensorMap,
+                                                           const __grid_constant__ CUtensorMap);
 
 // x_perm[pair] = x16[token of pair], 16 bytes per thread.
 __global__ void gather_rows_kernel(const __half *__restrict__ x16, const int *__restrict__ pair_tok,

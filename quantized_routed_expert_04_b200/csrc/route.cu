@@ -134,15 +134,17 @@ __global__ void topk_kernel(const float *__restrict__ logits, int T, int E, int 
 }
 
 // ---------------------------------------------------------------- activation pack
-// x bf16 -> f16 (pack8_bf16_to_f16: groups of 8 in the order 0,4,1,5,2,6,3,7);
-// an activation beyond the f16 range sets STATUS_RANGE.
+// x bf16 -> f16 in the weight format's pair order (pack8_bf16_to_f16); an
+// activation beyond the f16 range sets STATUS_RANGE.
 __global__ void pack_x_kernel(const __nv_bfloat16 *__restrict__ x, int n8,
-                              __half *__restrict__ x16, int *status) {
+                              __half *__restrict__ x16, int fmt, int *status) {
   grid_dependency_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   bool over;
-  const uint4 o = pack8_bf16_to_f16(*reinterpret_cast<const uint4 *>(x + (size_t)i * 8), over);
+  const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)i * 8);
+  const uint4 o = fmt == kFmtInt4 ? pack8_bf16_to_f16<kFmtInt4>(raw, over)
+                                  : pack8_bf16_to_f16<kFmtNvfp4>(raw, over);
   if (over) set_status(status, STATUS_RANGE);
   *reinterpret_cast<uint4 *>(x16 + (size_t)i * 8) = o;
 }

@@ -36,6 +36,7 @@ struct EventPair {
 struct strata_moe {
   int H, I, E, k, S, n_slots;
   int device = 0, num_sms = 0;
+  int fmt = kFmtInt4;       // weight format of every blob of the layer
   BlobLayout layout{};
 
   std::vector<int> slot_expert;            // per slot: expert id or -1
@@ -265,11 +266,14 @@ strata_status run_tc_passes(strata_moe *h, int T, const ExpertTable &table, bool
     p.y_out = h->y;
     p.status = h->status;
     p.quiet_unbound = quiet ? 1 : 0;
+    p.glob_off = h->layout.glob;
     CUtensorMap m64, m256;
     if (!encode_rows_map(&m64, gu ? h->xp : h->h16, p.K, P, 64) ||
         !encode_rows_map(&m256, gu ? h->xp : h->h16, p.K, P, 256))
       return STRATA_ERR_CUDA;
-    auto kern = gu ? expert_tc_kernel<true> : expert_tc_kernel<false>;
+    auto kern = h->fmt == kFmtInt4
+                    ? (gu ? expert_tc_kernel<true, kFmtInt4> : expert_tc_kernel<false, kFmtInt4>)
+                    : (gu ? expert_tc_kernel<true, kFmtNvfp4> : expert_tc_kernel<false, kFmtNvfp4>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
       e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(tc_threads()), smem,
@@ -296,7 +300,7 @@ strata_status run_prepare(strata_moe *h, const void *x, int T, const int32_t *id
   const auto *xb = static_cast<const __nv_bfloat16 *>(x);
   const int n8 = T * h->H / 8;
   e = launch(h, PH_PACK, pack_x_kernel, dim3((n8 + 255) / 256), dim3(256), 0, stream, false, xb,
-             n8, h->x16, h->status);
+             n8, h->x16, h->fmt, h->status);
   if (e == cudaSuccess)
     e = launch(h, PH_BUCKET, bucket_count_kernel, dim3((T * h->k + 255) / 256), dim3(256), 0,
                stream, true, idx, T, h->k, h->E, h->rt.cnt, h->status);
@@ -411,7 +415,11 @@ strata_status run_fused(strata_moe *h, const void *x, int T, const int32_t *idx_
   p.tile_cnt = h->counters + 4 + 2 * kFusedWarps * h->num_sms;
   p.status = h->status;
   p.out = static_cast<__nv_bfloat16 *>(out);
-  auto kern = p.group <= 8 ? decode_fused_kernel<1> : decode_fused_kernel<2>;
+  p.glob = h->layout.glob;
+  auto kern = h->fmt == kFmtInt4
+                  ? (p.group <= 8 ? decode_fused_kernel<1, kFmtInt4> : decode_fused_kernel<2, kFmtInt4>)
+                  : (p.group <= 8 ? decode_fused_kernel<1, kFmtNvfp4>
+                                  : decode_fused_kernel<2, kFmtNvfp4>);
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_status(e);
@@ -464,8 +472,24 @@ const char *strata_status_str(strata_status s) {
 }
 
 size_t strata_moe_expert_bytes(int hidden, int inter) {
+  return strata_moe_expert_bytes_fmt(hidden, inter, STRATA_FORMAT_INT4);
+}
+
+size_t strata_moe_expert_bytes_fmt(int hidden, int inter, int fmt) {
   if (hidden <= 0 || inter <= 0 || hidden % 128 || inter % 128) return 0;
-  return blob_layout(hidden, inter).total;
+  if (fmt != STRATA_FORMAT_INT4 && fmt != STRATA_FORMAT_NVFP4) return 0;
+  return blob_layout(hidden, inter, fmt).total;
+}
+
+strata_status strata_moe_set_format(strata_moe *h, int fmt) {
+  if (!h || (fmt != STRATA_FORMAT_INT4 && fmt != STRATA_FORMAT_NVFP4)) return STRATA_ERR_INVALID_ARG;
+  for (int s = 0; s < h->n_slots; ++s)
+    if (h->slot_expert[s] >= 0) return STRATA_ERR_INVALID_ARG;
+  for (int i = 0; i < h->S; ++i)
+    if (h->shared_ptr[i]) return STRATA_ERR_INVALID_ARG;
+  h->fmt = fmt;
+  h->layout = blob_layout(h->H, h->I, fmt);
+  return STRATA_OK;
 }
 
 strata_status strata_moe_create(int hidden, int inter, int n_experts, int top_k, int n_shared,
@@ -581,6 +605,8 @@ void strata_handle_shape(const strata_moe *h, int *hidden, int *inter, int *n_ex
 }
 
 int strata_handle_top_k(const strata_moe *h) { return h->k; }
+
+size_t strata_handle_blob_bytes(const strata_moe *h) { return h->layout.total; }
 
 strata_status strata_layer_route_all(strata_moe *h, const void *x, int T, cudaStream_t stream,
                                      const int32_t **idx, const float **w) {

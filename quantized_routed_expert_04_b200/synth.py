@@ -366,6 +366,15 @@ def make_all_blobs(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
     return out
 
 
+def make_all_blobs_nvfp4(cfg: LayerConfig, seed: int = 0) -> np.ndarray:
+    """All E + S NVFP4 blobs as one u8 array [E+S][expert_bytes(..., "nvfp4")]."""
+    nb = expert_bytes(cfg.hidden, cfg.inter, "nvfp4")
+    out = np.empty((cfg.n_experts + cfg.n_shared, nb), np.uint8)
+    for e in range(cfg.n_experts + cfg.n_shared):
+        out[e] = make_expert_blob_nvfp4(cfg, e, seed)
+    return out
+
+
 def make_slot_permutation(cfg: LayerConfig, seed: int = 0, index: int = 0) -> np.ndarray:
     """Seeded permutation: slot s holds expert perm[s] (all experts bound)."""
     return _rng(seed, _STREAM_SLOTS, index).permutation(cfg.n_experts).astype(np.int32)

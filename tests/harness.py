@@ -28,14 +28,18 @@ def assert_within_tolerance(out_bf16_bits, ref, what=""):
 class GpuLayer:
     """A layer handle with all blobs resident on the device."""
 
-    def __init__(self, cfg, seed=0, blobs=None, bind="all", perm_index=0):
+    def __init__(self, cfg, seed=0, blobs=None, bind="all", perm_index=0, fmt="int4"):
         import torch
 
         from quantized_routed_expert_04_b200 import binding
         self.torch = torch
         self.cfg = cfg
         self.seed = seed
-        self.blobs = synth.make_all_blobs(cfg, seed) if blobs is None else blobs
+        self.fmt = fmt
+        if blobs is None:
+            blobs = synth.make_all_blobs(cfg, seed) if fmt == "int4" else \
+                synth.make_all_blobs_nvfp4(cfg, seed)
+        self.blobs = blobs
         self.dev_blobs = torch.from_numpy(self.blobs).cuda()
         W, b = synth.make_router(cfg, seed)
         self.W, self.b = W, b
@@ -44,6 +48,8 @@ class GpuLayer:
         self.layer = binding.StrataMoE(cfg.hidden, cfg.inter, cfg.n_experts, cfg.top_k,
                                        cfg.n_shared, cfg.n_slots)
         self.layer.set_router(self.W_dev, self.b_dev)
+        if fmt != "int4":
+            self.layer.set_format(binding.FORMAT_NVFP4)
         for i in range(cfg.n_shared):
             self.layer.bind_shared(i, self.blob_ptr(cfg.n_experts + i))
         self.slot_expert = np.full(cfg.n_slots, -1, np.int32)
@@ -108,7 +114,8 @@ class GpuLayer:
         self.layer.close()
 
 
-def oracle_reference_parallel(cfg, blobs, W, b, x_bits, idx=None, w=None, n_threads=None):
+def oracle_reference_parallel(cfg, blobs, W, b, x_bits, idx=None, w=None, n_threads=None,
+                              fmt="int4"):
     """oracle_reference split over token chunks run in threads (the oracle's
     C calls release the interpreter lock, so the chunks run in parallel on
     the host cores).  Each token's output depends only on that token, so the
@@ -128,14 +135,14 @@ def oracle_reference_parallel(cfg, blobs, W, b, x_bits, idx=None, w=None, n_thre
         lo, hi = bounds[i], bounds[i + 1]
         if hi > lo:
             out[lo:hi] = oracle_reference(cfg, blobs, W, b, x_bits[lo:hi], idx[lo:hi],
-                                          w[lo:hi])[0]
+                                          w[lo:hi], fmt=fmt)[0]
 
     with concurrent.futures.ThreadPoolExecutor(max_workers=n) as ex:
         list(ex.map(run, range(n)))
     return out, idx, w
 
 
-def oracle_reference(cfg, blobs, W, b, x_bits, idx=None, w=None):
+def oracle_reference(cfg, blobs, W, b, x_bits, idx=None, w=None, fmt="int4"):
     """Oracle output (fp32 [T][H]) with every expert bound; routing computed
     by the oracle unless idx/w are given.  Returns (out, idx, w)."""
     import oracle
@@ -146,6 +153,6 @@ def oracle_reference(cfg, blobs, W, b, x_bits, idx=None, w=None):
     if idx is None:
         _, idx, w = oracle.route(x_bits, W, b, cfg.top_k)
     st, out = oracle.forward_routed(x_bits, cfg.hidden, cfg.inter, E, cfg.top_k, se, sb, shared,
-                                    idx, w)
+                                    idx, w, fmt=fmt)
     assert st == oracle.OK
     return out, idx, w
