@@ -417,7 +417,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (gate) {
               const float gv = v[t];
               const float hv = gv / (1.0f + expf(-gv)) * up;
-              big_h |= fabsf(hv) >= kF16Overflow;
+              // (columns past the tile's pairs hold stale accumulators)
+              big_h |= col0 + t < un.n && fabsf(hv) >= kF16Overflow;
               hs[t * 16 + pos16] = __float2half_rn(hv);
             }
           }
