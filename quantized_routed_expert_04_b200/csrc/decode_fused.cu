@@ -21,13 +21,14 @@
 // no other CTA waits on it.
 //
 // Phases:
-//  R  every CTA packs a slice of x to f16 (range-checked); CTA c computes the
-//     logits of experts c, c + grid, ... for all tokens (12 warps split H,
-//     per-warp double sums added in warp order).  Barrier.
-//  K  top-k: for up to 12 tokens every CTA selects all tokens itself (one
-//     warp per token, the same inputs and code, so the same result
-//     everywhere); for more tokens CTA c selects token c and a second
-//     barrier publishes the choices.
+//  R  every CTA packs a slice of x to f16 (range-checked); the router's
+//     dot products are cut into units (expert, range of H) spread over every
+//     CTA, each storing double partial sums.  Barrier.
+//  K  logits = the units' partial sums added in a fixed order + bias, one
+//     rounding to fp32; top-k: for up to 12 tokens every CTA selects all
+//     tokens itself (one warp per token, the same inputs and code, so the
+//     same result everywhere); for more tokens CTA c selects token c and a
+//     second barrier publishes the choices.
 //  B  every CTA buckets the (token, j) pairs in shared memory: counts,
 //     offsets, the active experts, and a stable order by (expert, token), so
 //     the layout is a pure function of the routing.
@@ -62,6 +63,7 @@ namespace {
 constexpr int kFW = kFusedWarps;
 
 struct Tables {
+  const uint8_t **ptr;   // per expert id: the slot table (null: not bound)
   const uint8_t **blob;  // per active expert (null: not bound)
   int *aoff, *acnt;      // per active expert: first sorted pair, pair count
   int *gbase;            // per active expert: first pair group (prefix), [n_active + 1]
@@ -119,11 +121,9 @@ __device__ __forceinline__ int ld_acquire(const int *ptr) {
   return v;
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Ring-stage wait of one warp (lane 0 polls, with the given limit).
+// Ring-stage wait of one warp (lane 0 polls, with the given limit); once the
+// phase is complete every lane observes it itself (acquiring the stage's
+// bytes).
 __device__ __forceinline__ bool warp_wait_limit(uint64_t *bar, uint32_t parity, int *status,
                                                 unsigned long long limit_ns) {
   int ok = 1;
@@ -131,7 +131,7 @@ __device__ __forceinline__ bool warp_wait_limit(uint64_t *bar, uint32_t parity, 
     if (!mbar_try_wait(bar, parity)) {
       const uint64_t t0 = global_timer_ns();
       while (true) {
-        if (mbar_try_wait_sleep(bar, parity)) break;
+        if (mbar_try_wait(bar, parity)) break;
         if (global_timer_ns() - t0 > limit_ns) {
           set_status(status, STATUS_TIMEOUT);
           ok = 0;
@@ -140,7 +140,9 @@ __device__ __forceinline__ bool warp_wait_limit(uint64_t *bar, uint32_t parity, 
       }
     }
   }
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) (void)mbar_try_wait(bar, parity);
+  return ok != 0;
 }
 
 // Grid barrier: every thread of every CTA calls it the same number of times.
@@ -152,8 +154,7 @@ __device__ bool grid_sync(int *ctr, volatile int *abort_flag, int *status,
                           unsigned long long limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1);
+    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
     if (!*abort_flag) {
       const uint64_t t0 = global_timer_ns();
       unsigned ns = 32;
@@ -164,10 +165,9 @@ __device__ bool grid_sync(int *ctr, volatile int *abort_flag, int *status,
           break;
         }
         __nanosleep(ns);
-        if (ns < 128) ns <<= 1;
+        if (ns < 64) ns <<= 1;
       }
     }
-    __threadfence();
   }
   __syncthreads();
   return !*abort_flag;
@@ -210,9 +210,21 @@ __device__ __forceinline__ Item item_of(const Tables &tb, const PhaseInfo &ph, i
   return it;
 }
 
+// 16-byte asynchronous global -> shared copy (L2 only), and the arrival on a
+// stage barrier once all of this thread's earlier such copies have landed.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 // Issue the copies of the next stage: up to gpc K groups of the current piece
-// (packed weights and scales of 16 rows), one bulk copy each, completion in
-// transaction bytes on the stage's barrier.
+// (packed weights and scales of 16 rows, ng KB + ng x 128 B), as 16-byte
+// asynchronous copies spread over the warp's 32 lanes; each lane then arrives
+// on the stage's barrier when its copies have landed (32 arrivals per phase).
 __device__ __forceinline__ void issue_next(Cursor &c, Ring &rg, const Tables &tb,
                                            const PhaseInfo *ph, int group, int gpc, int kc,
                                            int lane) {
@@ -229,12 +241,13 @@ __device__ __forceinline__ void issue_next(Cursor &c, Ring &rg, const Tables &tb
   const int slot = (int)(rg.issued % rg.stages);
   uint8_t *dst = rg.base + slot * rg.stage_bytes;
   const int ng = min(gpc, c.pc.g1 - c.cg);
-  if (lane == 0) {
+  {
     const size_t g0 = (size_t)it.tau * P.groups + (size_t)c.cg;
-    mbar_arrive_expect_tx(&rg.full[slot], (uint32_t)ng * (1024u + 128u));
-    bulk_g2s(dst, it.blob + P.q_off + g0 * 1024, (uint32_t)ng * 1024u, &rg.full[slot]);
-    bulk_g2s(dst + (size_t)kc * 8, it.blob + P.s_off + g0 * 128, (uint32_t)ng * 128u,
-             &rg.full[slot]);
+    const uint8_t *qsrc = it.blob + P.q_off + g0 * 1024;
+    const uint8_t *ssrc = it.blob + P.s_off + g0 * 128;
+    for (int ch = lane; ch < ng * 64; ch += 32) cp_async16(dst + ch * 16, qsrc + ch * 16);
+    if (lane < ng * 8) cp_async16(dst + (size_t)kc * 8 + lane * 16, ssrc + lane * 16);
+    cp_async_arrive(&rg.full[slot]);
   }
   ++rg.issued;
   c.cg += ng;
@@ -514,7 +527,6 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       }
       cg += ng;
       // the stage's bytes are in registers now: refill it
-      fence_proxy_async_smem();
       __syncwarp();
       issue_next(cur, rg, tb, ph, p.group, gpc, kc, lane);
     }
@@ -603,7 +615,7 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
 size_t fused_table_bytes(int T, int k, int S) {
   const size_t P = (size_t)T * (k + S);
   size_t b = 0;
-  b += kMaxIds * sizeof(void *);            // blob
+  b += 2 * kMaxIds * sizeof(void *);        // ptr, blob
   b += 2 * kMaxIds * sizeof(int);           // aoff, acnt
   b += (kMaxIds + 2) * sizeof(int);         // gbase
   b += kMaxIds * sizeof(int);               // cnt
@@ -634,6 +646,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   Tables tb;
   {
     uint8_t *q = smem + p.smem_tables;
+    tb.ptr = reinterpret_cast<const uint8_t **>(q); q += kMaxIds * sizeof(void *);
     tb.blob = reinterpret_cast<const uint8_t **>(q); q += kMaxIds * sizeof(void *);
     tb.aoff = reinterpret_cast<int *>(q); q += kMaxIds * sizeof(int);
     tb.acnt = reinterpret_cast<int *>(q); q += kMaxIds * sizeof(int);
@@ -649,8 +662,10 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     tb.bad = reinterpret_cast<int *>(q);
   }
   volatile int *abort_flag = tb.misc + 2;
+  // the slot table, read with per-lane indices below, into shared memory
+  for (int i = tid; i < nid; i += blockDim.x) tb.ptr[i] = p.table.ptr[i];
   if (lane == 0)
-    for (int s = 0; s < p.stages; ++s) mbar_init(&rg.full[s], 1);
+    for (int s = 0; s < p.stages; ++s) mbar_init(&rg.full[s], 32);
   if (tid == 0) {
     *abort_flag = 0;
     fence_mbar_init();
@@ -671,16 +686,25 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     if (over) set_status(p.status, STATUS_RANGE);
   }
   const bool routed_given = p.idx_in != nullptr;
+  // Router: unit = (expert e, split sp), sp covering a range of the H/128
+  // chunks; splits = grid / E (at least 1) so that small E still uses every
+  // CTA.  A unit's 12 warps take its chunks round-robin, each lane 4
+  // consecutive elements; per token a lane's products are summed in double
+  // in chunk order, the 32 lanes reduced by one transpose-reduction, the
+  // warps added in warp order, and the unit's partial sum stored.
+  const int splits = max(1, (int)gridDim.x / E);
   if (!routed_given) {
-    const int chunks = H / 128;
-    for (int e = blockIdx.x; e < E; e += gridDim.x) {
+    const int C = H / 128;
+    for (int u = blockIdx.x; u < E * splits; u += gridDim.x) {
+      const int e = u / splits, sp = u - (u / splits) * splits;
+      const int c0 = sp * C / splits, c1 = (sp + 1) * C / splits;
       const float *wr = p.W + (size_t)e * H;
       for (int t0 = 0; t0 < T; t0 += 8) {
         const int nt = min(8, T - t0);
         double acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-        for (int c = warp; c < chunks; c += kFW) {
+        for (int c = c0 + warp; c < c1; c += kFW) {
           const int h = c * 128 + lane * 4;
           const float4 wv = *reinterpret_cast<const float4 *>(wr + h);
 #pragma unroll
@@ -696,18 +720,37 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
             }
           }
         }
+        // transpose-reduction: 8 values per lane -> lane l holds the sum for
+        // token 4 (l >> 4 & 1) + 2 (l >> 3 & 1) + (l >> 2 & 1)
+        {
+          const bool hi16 = lane & 16, hi8 = lane & 8, hi4 = lane & 4;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < 4; ++i) {
+            const double send = hi16 ? acc[i] : acc[i + 4];
+            const double keep = hi16 ? acc[i + 4] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+          }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-        if (lane == 0)
-          for (int i = 0; i < nt; ++i) tb.part[warp * 8 + i] = acc[i];
+          for (int i = 0; i < 2; ++i) {
+            const double send = hi8 ? acc[i] : acc[i + 2];
+            const double keep = hi8 ? acc[i + 2] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+          }
+          {
+            const double send = hi4 ? acc[0] : acc[1];
+            const double keep = hi4 ? acc[1] : acc[0];
+            acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+          }
+          acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+          acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+          const int tok = (hi16 ? 4 : 0) + (hi8 ? 2 : 0) + (hi4 ? 1 : 0);
+          if ((lane & 3) == 0) tb.part[warp * 8 + tok] = acc[0];
+        }
         __syncthreads();
         if (tid < nt) {
           double v = tb.part[tid];
           for (int w = 1; w < kFW; ++w) v += tb.part[w * 8 + tid];
-          if (p.bias) v += (double)p.bias[e];
-          p.logits[(size_t)(t0 + tid) * E + e] = (float)v;
+          p.rpart[((size_t)e * splits + sp) * T + t0 + tid] = v;
         }
         __syncthreads();
       }
@@ -715,28 +758,48 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   }
   bool live = grid_sync(p.bar + 0, abort_flag, p.status, p.wait_ns);
 
-  // ---- phase K: top-k
+  // ---- phase K: logits (the units' partial sums added in split order, plus
+  // the bias, rounded once to fp32) and top-k, from shared memory (the ring
+  // space, unused until the weight copies start)
+  float *s_logit = reinterpret_cast<float *>(smem);
   const bool redundant = T <= kFW;
+  auto logit_of = [&](int t, int e) -> float {
+    double v = __ldcg(p.rpart + ((size_t)e * splits) * T + t);
+    for (int sp = 1; sp < splits; ++sp) v += __ldcg(p.rpart + ((size_t)e * splits + sp) * T + t);
+    if (p.bias) v += (double)p.bias[e];
+    return (float)v;
+  };
+  auto topk_row = [&](const float *row, int &e, float &wt) {
+    if (E <= 64) select_topk_warp_t<2, true>(row, E, k, p.mode, lane, e, wt);
+    else select_topk_warp_t<kMaxExperts / 32, true>(row, E, k, p.mode, lane, e, wt);
+  };
   if (live && !routed_given) {
     if (redundant) {
+      for (int q = tid; q < T * E; q += blockDim.x) s_logit[q] = logit_of(q / E, q - (q / E) * E);
+      __syncthreads();
       if (warp < T) {
         int e;
         float wt;
-        select_topk_warp(p.logits + (size_t)warp * E, E, k, p.mode, lane, e, wt);
+        topk_row(s_logit + warp * E, e, wt);
         if (lane < k) {
           tb.idx[warp * k + lane] = e;
           tb.w[warp * k + lane] = wt;
         }
       }
-    } else if (warp == 0) {
+    } else {
       for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        int e;
-        float wt;
-        select_topk_warp(p.logits + (size_t)t * E, E, k, p.mode, lane, e, wt);
-        if (lane < k) {
-          p.idx[(size_t)t * k + lane] = e;
-          p.w[(size_t)t * k + lane] = wt;
+        for (int e = tid; e < E; e += blockDim.x) s_logit[e] = logit_of(t, e);
+        __syncthreads();
+        if (warp == 0) {
+          int e;
+          float wt;
+          topk_row(s_logit, e, wt);
+          if (lane < k) {
+            p.idx[(size_t)t * k + lane] = e;
+            p.w[(size_t)t * k + lane] = wt;
+          }
         }
+        __syncthreads();
       }
     }
   }
@@ -765,7 +828,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
       const int e = tb.idx[q];
       if (e >= 0 && e < E) {
         atomicAdd(&tb.cnt[e], 1);
-        if (!p.table.ptr[e]) tb.bad[q / k] = 1;
+        if (!tb.ptr[e]) tb.bad[q / k] = 1;
       } else {
         tb.bad[q / k] = 1;
         if (blockIdx.x == 0) set_status(p.status, STATUS_BAD_ROUTING);
@@ -780,7 +843,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
         const int c = i < nid ? tb.cnt[i] : 0;
         const int f = c > 0;
         const int ng = (c + p.group - 1) / p.group;
-        const uint8_t *bp = i < nid ? p.table.ptr[i] : nullptr;
+        const uint8_t *bp = i < nid ? tb.ptr[i] : nullptr;
         int inc = c, finc = f, ginc = ng, binc = bp ? ng : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

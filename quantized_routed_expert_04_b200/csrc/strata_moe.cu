@@ -60,6 +60,7 @@ struct strata_moe {
   __half *h16 = nullptr;
   float *y = nullptr;
   __half *xp = nullptr;     // activations gathered in sorted pair order (large batches)
+  double *rpart = nullptr;  // decode kernel: router partial sums
   float *partial = nullptr; // decode kernel: partial sums of items cut between warps
   int *counters = nullptr;  // decode kernel: barrier, cut-item and tile counters (zero between launches)
   size_t counters_bytes = 0;
@@ -160,6 +161,7 @@ strata_status grow_workspace(strata_moe *h, int T) {
   const size_t o_h16 = take(sizeof(__half) * P * h->I);
   const size_t o_y = take(sizeof(float) * P * h->H);
   const size_t o_xp = cap > kSmallT ? take(sizeof(__half) * P * h->H) : 0;
+  const size_t o_rpart = take(sizeof(double) * std::max(h->E, h->num_sms) * (size_t)cap);
   const size_t o_partial = take(fused_partial_bytes(h));
   const size_t o_counters = take(fused_counter_bytes(h));
   void *mem = nullptr;
@@ -188,6 +190,7 @@ strata_status grow_workspace(strata_moe *h, int T) {
   h->h16 = reinterpret_cast<__half *>(b + o_h16);
   h->y = reinterpret_cast<float *>(b + o_y);
   h->xp = cap > kSmallT ? reinterpret_cast<__half *>(b + o_xp) : nullptr;
+  h->rpart = reinterpret_cast<double *>(b + o_rpart);
   h->partial = reinterpret_cast<float *>(b + o_partial);
   h->counters = reinterpret_cast<int *>(b + o_counters);
   h->counters_bytes = fused_counter_bytes(h);
@@ -403,7 +406,7 @@ strata_status run_fused(strata_moe *h, const void *x, int T, const int32_t *idx_
   if (p.stages < 2) return STRATA_ERR_UNSUPPORTED;
   p.smem_tables = (size_t)kFusedWarps * p.stages * p.stage_bytes + bars;
   const size_t smem = p.smem_tables + tables;
-  p.logits = h->logits;
+  p.rpart = h->rpart;
   p.idx = h->idx;
   p.w = h->w;
   p.x16 = h->x16;
@@ -801,7 +804,7 @@ strata_status noalloc_scratch_on(int device, unsigned char **out) {
 // workspace (the counters are the only ones that must be zero when a call
 // starts).
 struct NoAllocLayout {
-  size_t logits, idx, w, meta, ptok, pj, inv, x16, h16, y, counters, partial, total;
+  size_t logits, idx, w, meta, ptok, pj, inv, x16, h16, y, rpart, counters, partial, total;
 };
 
 NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
@@ -824,6 +827,7 @@ NoAllocLayout noalloc_layout(const strata_moe *h, int T) {
   L.x16 = take(sizeof(__half) * T * h->H);
   L.h16 = take(sizeof(__half) * P * h->I);
   L.y = take(sizeof(float) * P * h->H);
+  L.rpart = take(sizeof(double) * std::max(h->E, h->num_sms) * (size_t)T);
   L.counters = take(fused_counter_bytes(h));
   L.partial = take(fused_partial_bytes(h));
   L.total = off;
@@ -840,7 +844,7 @@ class NoAllocWorkspace {
   NoAllocWorkspace(strata_moe *h, unsigned char *base, const NoAllocLayout &L)
       : h_(h), logits_(h->logits), idx_(h->idx), w_(h->w), meta_(h->meta), rt_(h->rt),
         x16_(h->x16), h16_(h->h16), y_(h->y), xp_(h->xp),
-        partial_(h->partial), counters_(h->counters),
+        rpart_(h->rpart), partial_(h->partial), counters_(h->counters),
         profiling_(h->profiling) {
     const int nid = h->E + h->S;
     h->logits = reinterpret_cast<float *>(base + L.logits);
@@ -859,6 +863,7 @@ class NoAllocWorkspace {
     h->y = reinterpret_cast<float *>(base + L.y);
     h->xp = nullptr;
     h->counters = reinterpret_cast<int *>(base + L.counters);
+    h->rpart = reinterpret_cast<double *>(base + L.rpart);
     h->partial = reinterpret_cast<float *>(base + L.partial);
     h->profiling = false;
   }
@@ -872,6 +877,7 @@ class NoAllocWorkspace {
     h_->h16 = h16_;
     h_->y = y_;
     h_->xp = xp_;
+    h_->rpart = rpart_;
     h_->partial = partial_;
     h_->counters = counters_;
     h_->profiling = profiling_;
@@ -889,6 +895,7 @@ class NoAllocWorkspace {
   __half *x16_, *h16_;
   float *y_;
   __half *xp_;
+  double *rpart_;
   float *partial_;
   int *counters_;
   bool profiling_;

@@ -14,14 +14,17 @@ namespace strata {
 // 1 / (1 + exp(-l)) in double rounded to fp32, key = score + correction,
 // weights = score_j / (sum of the selected scores in selection order) *
 // routed scale.  Lane j (< k) returns selection j in sel_e / sel_w.
-__device__ __forceinline__ void select_topk_warp(const float *__restrict__ logit_row, int E, int k,
-                                 const RouteMode &mode, int lane, int &sel_e, float &sel_w) {
-  constexpr int kPer = kMaxExperts / 32;
+// kPer: experts per lane (E <= 32 kPer); kShared: the row is in shared
+// memory (else global memory written by other CTAs, read from L2).
+template <int kPer, bool kShared>
+__device__ __forceinline__ void select_topk_warp_t(const float *__restrict__ logit_row, int E,
+                                                   int k, const RouteMode &mode, int lane,
+                                                   int &sel_e, float &sel_w) {
   float key[kPer], val[kPer];   // val: logit (softmax) or score (sigmoid)
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
-    const float l = e < E ? __ldcg(logit_row + e) : -INFINITY;
+    const float l = e < E ? (kShared ? logit_row[e] : __ldcg(logit_row + e)) : -INFINITY;
     if (mode.sigmoid && e < E) {
       val[i] = (float)(1.0 / (1.0 + exp(-(double)l)));
       key[i] = mode.corr ? __fadd_rn(val[i], mode.corr[e]) : val[i];
@@ -73,6 +76,12 @@ __device__ __forceinline__ void select_topk_warp(const float *__restrict__ logit
   }
   sel_e = my_e;
   sel_w = mode.sigmoid ? __fmul_rn(__fdiv_rn(my_v, z), mode.scale) : expf(my_v - v0) / z;
+}
+
+__device__ __forceinline__ void select_topk_warp(const float *__restrict__ logit_row, int E, int k,
+                                                 const RouteMode &mode, int lane, int &sel_e,
+                                                 float &sel_w) {
+  select_topk_warp_t<kMaxExperts / 32, false>(logit_row, E, k, mode, lane, sel_e, sel_w);
 }
 
 }  // namespace strata
