@@ -379,20 +379,14 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
     }
   };
 
-  uint4 bb0[NT][4], bb1[NT][4];
+  uint4 bb[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) bb0[nt][b] = bb1[nt][b] = make_uint4(0u, 0u, 0u, 0u);
-  int pb = 0;
+    for (int b = 0; b < 4; ++b) bb[nt][b] = make_uint4(0u, 0u, 0u, 0u);
   int a = 0;
   Piece pc;
   bool have = piece_at(tb, P, P.x_lo, a, pc);
-  if (have) {
-    const Item it0 = item_of(tb, P, p.group, pc.item, a);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) load_b(bb0[nt], act_row(it0, nt), pc.g0 * 128);
-  }
   bool ok = true;
   while (have && ok) {
     const Item it = item_of(tb, P, p.group, pc.item, a);
@@ -401,17 +395,9 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
     int a_nx = a;
     Piece pc_nx;
     const bool have_nx = piece_at(tb, P, x + (pc.g1 - pc.g0), a_nx, pc_nx);
-    const __half *row_cur[NT], *row_nx[NT];
+    const __half *row_cur[NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      row_cur[nt] = act_row(it, nt);
-      row_nx[nt] = nullptr;
-    }
-    if (have_nx) {
-      const Item it_nx = item_of(tb, P, p.group, pc_nx.item, a_nx);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) row_nx[nt] = act_row(it_nx, nt);
-    }
+    for (int nt = 0; nt < NT; ++nt) row_cur[nt] = act_row(it, nt);
     float2 acc[NT][2];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = make_float2(0.0f, 0.0f);
@@ -433,21 +419,12 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       const uint8_t *stq = rg.base + slot * rg.stage_bytes;
       const uint8_t *sts = stq + (size_t)kc * 8;
       const int ng = min(gpc, pc.g1 - cg);
-#pragma unroll 4
+#pragma unroll 2
       for (int j = 0; j < ng; ++j) {
-        {
-          const int G_next = cg + j + 1;
-          const bool same = G_next < pc.g1;
-          if (same || have_nx) {
-            const int k0 = (same ? G_next : pc_nx.g0) * 128;
+        // this group's activation fragments (L1-resident rows), loaded ahead
+        // of the weight conversion that hides their latency
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const __half *r = same ? row_cur[nt] : row_nx[nt];
-              if (pb == 0) load_b(bb1[nt], r, k0);
-              else load_b(bb0[nt], r, k0);
-            }
-          }
-        }
+        for (int nt = 0; nt < NT; ++nt) load_b(bb[nt], row_cur[nt], (cg + j) * 128);
         const uint4 w0 = *reinterpret_cast<const uint4 *>(stq + j * 1024 + g * 64 + cq * 16);
         const uint4 w1 = *reinterpret_cast<const uint4 *>(stq + j * 1024 + (g + 8) * 64 + cq * 16);
         const uint2 s0 = *reinterpret_cast<const uint2 *>(sts + j * 128 + g * 8);
@@ -522,8 +499,7 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
             }
           }
         };
-        if (pb == 0) mma_group(bb0); else mma_group(bb1);
-        pb ^= 1;
+        mma_group(bb);
       }
       cg += ng;
       // the stage's bytes are in registers now: refill it

@@ -7,42 +7,46 @@
 //   gate/up pass:  h = silu(Wg x) * (Wu x)  -> h16 [P][I] (f16)
 //   down pass:     y = Wd h                -> y   [P][H] (fp32)
 //
-// Tile = (expert, chunk of <= 256 of its pairs, 128 weight rows).  For
+// Unit = (expert, block of <= 512 of its pairs, 128 weight rows).  For
 // gate/up the 128 rows are 8 blob tiles, i.e. 64 gate rows and the same 64 up
 // rows interleaved by 8 (TMEM lane l holds gate if l % 16 < 8, else up; its
 // partner is lane l ^ 8, in the same warp).  For down they are 128
-// consecutive rows of Wd.
+// consecutive rows of Wd.  A unit's pairs form one or two chunks of <= 256
+// (one MMA N each); every dequantised weight atom feeds both chunks, so an
+// expert with many pairs pays the dequantisation once per 512 pairs.
 //
-// Warp roles (one CTA per SM, persistent; tiles interleaved over CTAs):
+// Warp roles (one CTA per SM, persistent; units interleaved over CTAs):
 //   warp 0      activation producer: per 64 K elements (one swizzle atom)
-//               the activation rows (f16, 128-byte swizzle; x_perm or h16)
-//               in one 256-row TMA box, or in up to three 64-row boxes for
-//               shorter tiles;
-//   last warp   weight producer: per four K groups (of 128) one bulk copy per
-//               blob tile of packed weights and one of scales (its own warp,
-//               so the weight ring runs ahead of the activations);
+//               and chunk, the activation rows (f16, 128-byte swizzle; x_perm
+//               or h16) in one 256-row TMA box, or in up to three 64-row
+//               boxes for shorter chunks;
+//   last warp   weight producer: per two K groups (of 128) one bulk copy per
+//               blob tile of packed weights and one of scales;
 //   warp 1      MMA: allocates all 512 TMEM columns (two 256-column
-//               accumulator buffers), and one thread issues 4 tcgen05.mma
-//               (M=128, N=pairs rounded up to 16, K=16) per atom, then
-//               commits to the stage barriers and, at the end of a tile, to
-//               the accumulator;
+//               accumulators), and one thread issues 4 tcgen05.mma (M=128,
+//               N=chunk pairs rounded up to 16, K=16) per atom and chunk,
+//               commits to the operand stages and, at the end of a unit, to
+//               the accumulators it used;
 //   warps 2-9   dequant: int4 -> exact f16 integers -> times the fp16 scale
 //               (one f16 rounding), or NVFP4 E2M1 codes times their E4M3
 //               group scale (exact in f16; the fp32 global scale multiplies
 //               the accumulator in the epilogue) -> the K-major
 //               128-byte-swizzled A layout;
-//   warps 10-13 epilogue: tcgen05.ld, SwiGLU (gate/up) or plain (down),
-//               transposed through shared memory, stored.
-// Both operands are staged one 64-wide swizzle atom at a time in a ring of
-// three stages with one "full" barrier (dequant arrivals + activation bytes)
-// and one "empty" barrier (MMA commit) per stage; packed weights sit in two
-// stages of four K groups.  The copy engine's per-operation cost, not bytes,
-// limits this kernel when the copies are small, so both producers move few,
-// large pieces.
-// N = 256 matters: one M=128 MMA costs about the same issue time at N = 128
-// as at N = 256, so the wide tile nearly doubles tensor throughput.
+//   warps 10-17 epilogue: two warps per TMEM lane quarter, each taking
+//               alternate 32-column blocks: tcgen05.ld, SwiGLU (gate/up; the
+//               gate lane and its up partner each compute every other
+//               column) or plain (down), transposed through shared memory,
+//               stored.
+// The A operand (16 KB per atom) and the B operand (32 KB per atom and
+// chunk) have rings of their own (three and four stages) with one "full" and
+// one "empty" mbarrier per stage.  A unit of two chunks uses both
+// accumulators; a unit of one chunk uses the next one in turn, so the
+// epilogue of a unit overlaps the MMAs of the next.  The copy engine's
+// per-operation cost, not bytes, limits this kernel when copies are small,
+// so both producers move few, large pieces.
 // Every wait is bounded; on a timeout the status word is set and the roles
-// wind down (the allocating warp still frees the tensor memory).
+// wind down (the producers let their issued copies land; the allocating warp
+// still frees the tensor memory).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -52,17 +56,20 @@ namespace strata {
 
 namespace {
 
-constexpr int kTcM = 128;          // weight rows per tile
-constexpr int kTcN = 256;          // pairs per tile (max MMA N used)
-constexpr int kPkStages = 2;       // packed-weight stages (four K groups each)
-constexpr int kPkGroups = 4;
-constexpr int kStages = 3;         // operand stages: one 64-wide atom of A and of B each
+constexpr int kTcM = 128;          // weight rows per unit
+constexpr int kTcN = 256;          // pairs per chunk (max MMA N used)
+constexpr int kUnitPairs = 2 * kTcN;
+constexpr int kPkStages = 2;       // packed-weight stages
+constexpr int kPkGroups = 2;       // K groups (of 128) per packed stage
+constexpr int kAStages = 3;        // A ring: one 64-wide dequantised atom each
+constexpr int kBStages = 4;        // B ring: one 64-wide activation atom of one chunk each
 constexpr int kDqWarps = 8;
 constexpr int kDqRows = kTcM / kDqWarps;    // weight rows per dequant warp
 static_assert(kDqRows % 8 == 0, "dequant warps cover whole 8-row groups");
-constexpr int kPkWarp = 2 + kDqWarps + 4;   // the last warp
+constexpr int kEpiWarps = 8;                // two per TMEM lane quarter
+constexpr int kPkWarp = 2 + kDqWarps + kEpiWarps;   // the last warp
 constexpr int kTcThreads = 32 * (kPkWarp + 1);
-constexpr int kAccCols = 256;      // TMEM columns per accumulator buffer
+constexpr int kAccCols = 256;      // TMEM columns per accumulator
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kAStageBytes = kTcM * 128;               // one 64-wide atom
@@ -70,14 +77,14 @@ constexpr int kBStageBytes = kTcN * 128;
 constexpr int kPkQBytes = 8 * kPkGroups * 1024;        // 8 blob tiles
 constexpr int kPkSBytes = 8 * kPkGroups * 128;
 constexpr int kPkStageBytes = kPkQBytes + kPkSBytes;
-constexpr int kEpiBytes = 4 * 1024;                    // per epilogue warp: 1 KB
+constexpr int kEpiBytes = kEpiWarps * 1024;            // per epilogue warp: 1 KB
 
 constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kStages * kAStageBytes;
-constexpr int kOffPk = kOffB + kStages * kBStageBytes;
+constexpr int kOffB = kOffA + kAStages * kAStageBytes;
+constexpr int kOffPk = kOffB + kBStages * kBStageBytes;
 constexpr int kOffEpi = kOffPk + kPkStages * kPkStageBytes;
 constexpr int kOffBar = kOffEpi + kEpiBytes;
-constexpr int kNumBars = 2 * kPkStages + 2 * kStages + 4;
+constexpr int kNumBars = 2 * kPkStages + 2 * kAStages + 2 * kBStages + 4;
 constexpr int kOffTab = kOffBar + kNumBars * 8 + 16;   // + TMEM address slot
 constexpr int kTabBytes = kMaxIds * 8 + (3 * kMaxIds + 1) * 4;
 constexpr int kTcSmem = kOffTab + kTabBytes + 1024;    // + alignment slack
@@ -91,6 +98,42 @@ __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *statu
 struct Unit {
   const uint8_t *blob;
   int pi0, n, rt;
+  __device__ __forceinline__ int chunks() const { return n > kTcN ? 2 : 1; }
+  __device__ __forceinline__ int chunk_n(int c) const { return c == 0 ? min(n, kTcN) : n - kTcN; }
+};
+
+// A ring position (stage and phase parity), advanced in the same order by
+// the roles that share the ring.
+struct RingPos {
+  uint32_t st = 0, ph = 0;
+  __device__ __forceinline__ void next(uint32_t stages) {
+    if (++st == stages) {
+      st = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
+// Accumulator use: a two-chunk unit uses accumulators 0 and 1; a one-chunk
+// unit uses the one after the last it used.  Both the MMA thread and the
+// epilogue walk the units in the same order, so they agree on every
+// accumulator's use count (and so on the barrier phases).
+struct AccTrack {
+  uint32_t uses[2] = {0u, 0u};
+  int next_single = 0;
+  __device__ __forceinline__ int buf_of(int nchunks, int c) const {
+    return nchunks == 2 ? c : next_single;
+  }
+  __device__ __forceinline__ void done_unit(int nchunks) {
+    if (nchunks == 2) {
+      uses[0]++;
+      uses[1]++;
+      next_single = 0;
+    } else {
+      uses[next_single]++;
+      next_single ^= 1;
+    }
+  }
 };
 
 }  // namespace
@@ -108,10 +151,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint64_t *pk_full = bars, *pk_empty = pk_full + kPkStages;
-  // full[s]: the dequant warps' arrivals plus the activation TMA bytes;
-  // empty[s]: the MMAs that read stage s have completed
-  uint64_t *full = pk_empty + kPkStages, *empty = full + kStages;
-  uint64_t *acc_full = empty + kStages, *acc_empty = acc_full + 2;
+  // fullA[s]: the dequant warps' arrivals; fullB[s]: the activation TMA bytes;
+  // emptyA/emptyB[s]: the MMAs that read stage s have completed
+  uint64_t *fullA = pk_empty + kPkStages, *emptyA = fullA + kAStages;
+  uint64_t *fullB = emptyA + kAStages, *emptyB = fullB + kBStages;
+  uint64_t *acc_full = emptyB + kBStages, *acc_empty = acc_full + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
   const uint8_t **t_blob = reinterpret_cast<const uint8_t **>(smem + kOffTab);
   int *t_off = reinterpret_cast<int *>(t_blob + kMaxIds);
@@ -124,13 +168,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&pk_full[s], 1);
       mbar_init(&pk_empty[s], kDqWarps);
     }
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], kDqWarps + 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&fullA[s], kDqWarps);
+      mbar_init(&emptyA[s], 1);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&fullB[s], 1);
+      mbar_init(&emptyB[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);
+      mbar_init(&acc_empty[s], kEpiWarps);
     }
     fence_mbar_init();
     prefetch_tmap(&tmap_b64);
@@ -142,8 +190,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   grid_dependency_wait();
 
-  // active experts and tiles per expert (prefix), in shared memory; an
-  // active expert without a blob gets no tiles (and is reported, unless the
+  // active experts and units per expert (prefix), in shared memory; an
+  // active expert without a blob gets no units (and is reported, unless the
   // call runs one expert pass of several)
   const int n_active = *p.rt.n_active;
   for (int a = threadIdx.x; a < n_active; a += blockDim.x) {
@@ -161,7 +209,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int carry = 0;
     for (int a0 = 0; a0 < n_active; a0 += 32) {
       const int a = a0 + lane;
-      const int v = a < n_active && t_blob[a] ? ((t_cnt[a] + kTcN - 1) / kTcN) * p.row_tiles : 0;
+      const int v = a < n_active && t_blob[a]
+                        ? ((t_cnt[a] + kUnitPairs - 1) / kUnitPairs) * p.row_tiles : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -181,57 +230,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto decode = [&](int u, int &a) -> Unit {
     while (unit_base[a + 1] <= u) ++a;
     const int rem = u - unit_base[a];
-    const int tcn = rem / p.row_tiles;
+    const int ub = rem / p.row_tiles;
     Unit un;
-    un.rt = rem - tcn * p.row_tiles;
-    un.pi0 = t_off[a] + tcn * kTcN;
-    un.n = min(kTcN, t_cnt[a] - tcn * kTcN);
+    un.rt = rem - ub * p.row_tiles;
+    un.pi0 = t_off[a] + ub * kUnitPairs;
+    un.n = min(kUnitPairs, t_cnt[a] - ub * kUnitPairs);
     un.blob = t_blob[a];
     return un;
   };
-  // tiles are interleaved over the CTAs (every tile belongs to a bound expert)
-  auto next_unit = [&](int u, int &) -> int { return min(u, n_units); };
 
   if (warp == 0) {
     // -------------------------------------------------------- activation producer
-    uint32_t issued = 0, st = 0, ph = 0;
+    uint32_t issued = 0;
+    RingPos rb;
     bool ok = true;
     int a = 0;
-    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit un = decode(u, a);
-      const bool wide = un.n > 192;           // one 256-row box, else 64-row boxes
-      const int nb = wide ? 1 : (un.n + 63) / 64;
-      const uint32_t tx = wide ? 32768u : nb * 8192u;
+      const int nc = un.chunks();
       for (int at = 0; at < 2 * G && ok; ++at) {
-        if (!wwait(&empty[st], ph ^ 1u, p.status)) { ok = false; break; }
-        uint8_t *dst = smem + kOffB + st * kBStageBytes;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[st], tx);
-          if (wide)
-            tma_load_2d(dst, &tmap_b256, at * 64, un.pi0, &full[st]);
-          else
-            for (int rb = 0; rb < nb; ++rb)
-              tma_load_2d(dst + rb * 8192, &tmap_b64, at * 64, un.pi0 + rb * 64, &full[st]);
-        }
-        __syncwarp();
-        ++issued;
-        if (++st == kStages) {
-          st = 0;
-          ph ^= 1u;
+        for (int c = 0; c < nc; ++c) {
+          if (!wwait(&emptyB[rb.st], rb.ph ^ 1u, p.status)) { ok = false; break; }
+          const int cn = un.chunk_n(c), row0 = un.pi0 + c * kTcN;
+          const bool wide = cn > 192;            // one 256-row box, else 64-row boxes
+          const int nb = wide ? 1 : (cn + 63) / 64;
+          const uint32_t tx = wide ? 32768u : nb * 8192u;
+          uint8_t *dst = smem + kOffB + rb.st * kBStageBytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&fullB[rb.st], tx);
+            if (wide)
+              tma_load_2d(dst, &tmap_b256, at * 64, row0, &fullB[rb.st]);
+            else
+              for (int q = 0; q < nb; ++q)
+                tma_load_2d(dst + q * 8192, &tmap_b64, at * 64, row0 + q * 64, &fullB[rb.st]);
+          }
+          __syncwarp();
+          ++issued;
+          rb.next(kBStages);
         }
       }
     }
     if (!ok) {
       // let issued copies land before the CTA exits (bounded waits)
-      for (uint32_t m = issued > kStages ? issued - kStages : 0; m < issued; ++m)
-        (void)wwait(&full[m % kStages], (m / kStages) & 1u, p.status);
+      for (uint32_t m = issued > kBStages ? issued - kBStages : 0; m < issued; ++m)
+        (void)wwait(&fullB[m % kBStages], (m / kBStages) & 1u, p.status);
     }
   } else if (warp == kPkWarp) {
     // -------------------------------------------------------- weight producer
     uint32_t pk_cnt = 0;
     bool ok = true;
     int a = 0;
-    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit un = decode(u, a);
       for (int g = 0; g < G && ok; g += kPkGroups) {
         const int s = (int)(pk_cnt % kPkStages);
@@ -258,44 +307,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issue
-    // One thread does it all: per atom one wait, four MMAs, one commit, so
-    // the tensor pipe's queue never runs dry behind warp-level overheads.
+    // One thread does it all: per atom one wait for A, per chunk one wait for
+    // B, four MMAs and one commit, so the tensor pipe's queue never runs dry
+    // behind warp-level overheads.
     if (lane == 0) {
-      uint32_t st = 0, ph = 0, t_cnt_local = 0;
+      RingPos ra, rb;
+      AccTrack acc;
       bool ok = true;
       int a = 0;
-      for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const Unit un = decode(u, a);
-        const int N = (un.n + 15) & ~15;
-        const uint32_t idesc = umma_idesc_f16(kTcM, N);
-        const int buf = (int)(t_cnt_local & 1u);
-        if (!mbar_wait(&acc_empty[buf], ((t_cnt_local >> 1) & 1u) ^ 1u, p.status)) {
-          ok = false;
-          break;
+        const int nc = un.chunks();
+        uint32_t idesc[2], d_tmem[2];
+        int bufs[2];
+        for (int c = 0; c < nc; ++c) {
+          bufs[c] = acc.buf_of(nc, c);
+          idesc[c] = umma_idesc_f16(kTcM, (un.chunk_n(c) + 15) & ~15);
+          d_tmem[c] = tmem_base + bufs[c] * kAccCols;
         }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * kAccCols;
-        for (int at = 0; at < 2 * G; ++at) {
-          if (!mbar_wait(&full[st], ph, p.status)) {
-            ok = false;
-            break;
-          }
+        for (int at = 0; at < 2 * G && ok; ++at) {
+          if (!mbar_wait(&fullA[ra.st], ra.ph, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + kOffA + st * kAStageBytes);
-          const uint32_t b_addr = smem_u32(smem + kOffB + st * kBStageBytes);
+          const uint32_t a_addr = smem_u32(smem + kOffA + ra.st * kAStageBytes);
+          for (int c = 0; c < nc; ++c) {
+            if (at == 0) {
+              // the accumulator must have been drained by the epilogue
+              const int b = bufs[c];
+              if (!mbar_wait(&acc_empty[b], (acc.uses[b] & 1u) ^ 1u, p.status)) { ok = false; break; }
+              tc_fence_after();
+            }
+            if (!mbar_wait(&fullB[rb.st], rb.ph, p.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t b_addr = smem_u32(smem + kOffB + rb.st * kBStageBytes);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            umma_f16(d_tmem, umma_desc_sw128(a_addr + j * 32), umma_desc_sw128(b_addr + j * 32),
-                     idesc, (at > 0 || j > 0) ? 1u : 0u);
-          umma_commit(&empty[st]);
-          if (++st == kStages) {
-            st = 0;
-            ph ^= 1u;
+            for (int j = 0; j < 4; ++j)
+              umma_f16(d_tmem[c], umma_desc_sw128(a_addr + j * 32),
+                       umma_desc_sw128(b_addr + j * 32), idesc[c], (at > 0 || j > 0) ? 1u : 0u);
+            umma_commit(&emptyB[rb.st]);
+            rb.next(kBStages);
           }
+          if (!ok) break;
+          umma_commit(&emptyA[ra.st]);
+          ra.next(kAStages);
         }
         if (!ok) break;
-        umma_commit(&acc_full[buf]);
-        ++t_cnt_local;
+        for (int c = 0; c < nc; ++c) umma_commit(&acc_full[bufs[c]]);
+        acc.done_unit(nc);
       }
     }
     __syncwarp();
@@ -305,10 +362,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int w = lane & 3;
     const int q = lane >> 2;
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
-    uint32_t pk_cnt = 0, st = 0, ph = 0;
+    uint32_t pk_cnt = 0;
+    RingPos ra;
     bool ok = true, big_scale = false;
-    int a = 0;
-    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       for (int g = 0; g < G && ok; ++g) {
         const int ps = (int)(pk_cnt % kPkStages);
         if (g % kPkGroups == 0)
@@ -317,8 +374,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint8_t *psc = pq + kPkQBytes;
         const int gi = g % kPkGroups;
         for (int atom = 0; atom < 2 && ok; ++atom) {
-          if (!wwait(&empty[st], ph ^ 1u, p.status)) { ok = false; break; }
-          uint8_t *ad = smem + kOffA + st * kAStageBytes;
+          if (!wwait(&emptyA[ra.st], ra.ph ^ 1u, p.status)) { ok = false; break; }
+          uint8_t *ad = smem + kOffA + ra.st * kAStageBytes;
 #pragma unroll
           for (int m = 0; m < kDqRows / 8; ++m) {
             const int r = kDqRows * dw + 8 * m + row_in_8;
@@ -367,11 +424,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&full[st]);
-          if (++st == kStages) {
-            st = 0;
-            ph ^= 1u;
-          }
+          if (lane == 0) mbar_arrive(&fullA[ra.st]);
+          ra.next(kAStages);
         }
         if (!ok) break;
         if (gi == kPkGroups - 1 || g == G - 1) {
@@ -383,84 +437,93 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (__any_sync(0xffffffffu, big_scale) && lane == 0) set_status(p.status, STATUS_RANGE);
   } else if (warp < kPkWarp) {
     // -------------------------------------------------------- epilogue
-    const int qd = warp & 3;  // TMEM lane quarter of this warp
-    float *stage = reinterpret_cast<float *>(smem + kOffEpi + (warp - 2 - kDqWarps) * 1024);
-    uint32_t t_cnt_local = 0;
+    const int ew = warp - 2 - kDqWarps;       // 0 .. kEpiWarps - 1
+    const int qd = warp & 3;                  // TMEM lane quarter of this warp
+    const int cpar = ew >> 2;                 // which alternate 32-column blocks
+    float *stage = reinterpret_cast<float *>(smem + kOffEpi + ew * 1024);
+    AccTrack acc;
     bool ok = true, big_h = false;
     int a = 0;
-    for (int u = next_unit(blockIdx.x, a); u < n_units && ok; u = next_unit(u + gridDim.x, a)) {
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit un = decode(u, a);
-      const int buf = (int)(t_cnt_local & 1u);
-      if (!wwait(&acc_full[buf], (t_cnt_local >> 1) & 1u, p.status)) { ok = false; break; }
-      tc_fence_after();
+      const int nc = un.chunks();
       // NVFP4: this lane's row's global scale (gate, up or down)
       float gsc = 1.0f;
       if (FMT == kFmtNvfp4) {
         const float *gs = reinterpret_cast<const float *>(un.blob + p.glob_off);
         gsc = kGateUp ? gs[(lane & 15) < 8 ? 0 : 1] : gs[2];
       }
-      for (int col0 = 0; col0 < un.n; col0 += 32) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * qd) << 16) + buf * kAccCols + col0, v);
-        if (FMT == kFmtNvfp4) {
+      for (int c = 0; c < nc && ok; ++c) {
+        const int buf = acc.buf_of(nc, c);
+        const int cn = un.chunk_n(c), pi0 = un.pi0 + c * kTcN;
+        if (!wwait(&acc_full[buf], acc.uses[buf] & 1u, p.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int col0 = 32 * cpar; col0 < cn; col0 += 64) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * qd) << 16) + buf * kAccCols + col0, v);
+          if (FMT == kFmtNvfp4) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) v[t] *= gsc;
-        }
-        if (kGateUp) {
-          // lane L: blob tile 2 qd + L / 16, tile row L % 16 (gate if < 8)
-          __half *hs = reinterpret_cast<__half *>(stage);  // [32 pairs][16]
-          const bool gate = (lane & 15) < 8;
-          const int pos16 = 8 * (lane >> 4) + packed_pos<FMT>(lane & 7);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float up = __shfl_xor_sync(0xffffffffu, v[t], 8);
-            if (gate) {
-              const float gv = v[t];
-              const float hv = gv / (1.0f + expf(-gv)) * up;
-              // (columns past the tile's pairs hold stale accumulators)
-              big_h |= col0 + t < un.n && fabsf(hv) >= kF16Overflow;
-              hs[t * 16 + pos16] = __float2half_rn(hv);
-            }
+            for (int t = 0; t < 32; ++t) v[t] *= gsc;
           }
-          __syncwarp();
+          if (kGateUp) {
+            // lane L: blob tile 2 qd + L / 16, tile row L % 16 (gate if < 8);
+            // the gate lane computes the even columns, its up partner (L ^ 8)
+            // the odd ones
+            __half *hs = reinterpret_cast<__half *>(stage);  // [32 pairs][16]
+            const bool is_up = (lane & 15) >= 8;
+            const int pos16 = 8 * (lane >> 4) + packed_pos<FMT>(lane & 7);
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int piece = lane + 32 * k;  // 64 pieces of 16 bytes
-            const int t = piece >> 1, half = piece & 1;
-            if (col0 + t < un.n) {
-              const uint4 val = *reinterpret_cast<const uint4 *>(hs + t * 16 + half * 8);
-              __half *dst = p.h_out + (size_t)(un.pi0 + col0 + t) * p.out_ld +
-                            64 * un.rt + 16 * qd + 8 * half;
-              *reinterpret_cast<uint4 *>(dst) = val;
+            for (int t = 0; t < 32; ++t) {
+              const float pv = __shfl_xor_sync(0xffffffffu, v[t], 8);
+              if ((t & 1) == (is_up ? 1 : 0)) {
+                const float gv = is_up ? pv : v[t];
+                const float uv = is_up ? v[t] : pv;
+                const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                // (columns past the chunk's pairs hold stale accumulators)
+                big_h |= col0 + t < cn && fabsf(hv) >= kF16Overflow;
+                hs[t * 16 + pos16] = __float2half_rn(hv);
+              }
             }
-          }
-          __syncwarp();
-        } else {
-          // 8 pairs at a time through a 1 KB stage: [8 pairs][32 rows] fp32
-#pragma unroll
-          for (int t8 = 0; t8 < 32; t8 += 8) {
-#pragma unroll
-            for (int t = 0; t < 8; ++t) stage[t * 32 + lane] = v[t8 + t];
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
               const int piece = lane + 32 * k;  // 64 pieces of 16 bytes
-              const int t = piece >> 3, seg = piece & 7;
-              if (col0 + t8 + t < un.n) {
-                const float4 val = *reinterpret_cast<const float4 *>(stage + t * 32 + seg * 4);
-                float *dst = p.y_out + (size_t)(un.pi0 + col0 + t8 + t) * p.out_ld + 128 * un.rt +
-                             32 * qd + 4 * seg;
-                *reinterpret_cast<float4 *>(dst) = val;
+              const int t = piece >> 1, half = piece & 1;
+              if (col0 + t < cn) {
+                const uint4 val = *reinterpret_cast<const uint4 *>(hs + t * 16 + half * 8);
+                __half *dst = p.h_out + (size_t)(pi0 + col0 + t) * p.out_ld + 64 * un.rt +
+                              16 * qd + 8 * half;
+                *reinterpret_cast<uint4 *>(dst) = val;
               }
             }
             __syncwarp();
+          } else {
+            // 8 pairs at a time through a 1 KB stage: [8 pairs][32 rows] fp32
+#pragma unroll
+            for (int t8 = 0; t8 < 32; t8 += 8) {
+#pragma unroll
+              for (int t = 0; t < 8; ++t) stage[t * 32 + lane] = v[t8 + t];
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                const int piece = lane + 32 * k;  // 64 pieces of 16 bytes
+                const int t = piece >> 3, seg = piece & 7;
+                if (col0 + t8 + t < cn) {
+                  const float4 val = *reinterpret_cast<const float4 *>(stage + t * 32 + seg * 4);
+                  float *dst = p.y_out + (size_t)(pi0 + col0 + t8 + t) * p.out_ld + 128 * un.rt +
+                               32 * qd + 4 * seg;
+                  *reinterpret_cast<float4 *>(dst) = val;
+                }
+              }
+              __syncwarp();
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      ++t_cnt_local;
+      acc.done_unit(nc);
     }
     if (__any_sync(0xffffffffu, big_h) && lane == 0) set_status(p.status, STATUS_RANGE);
   }
