@@ -32,7 +32,10 @@
 //  B  every CTA buckets the (token, j) pairs in shared memory: counts,
 //     offsets, the active experts, and a stable order by (expert, token), so
 //     the layout is a pure function of the routing.
-//  G  gate/up + SwiGLU -> h16; barrier;  D  down -> y, and the combine.
+//  G  gate/up + SwiGLU -> h16;  D  down -> y, and the combine.  A down
+//     piece starts once every gate/up item of its pair group has counted
+//     itself done (a counter per group, release/acquire), not at a grid
+//     barrier.
 // G and D cut their (item, K group) sequences -- item = (active expert, <= 8
 // or 16 of its pairs, one 16-row weight tile) -- into one equal contiguous
 // share per warp of the grid.  Each warp streams its shares through its own
@@ -302,6 +305,29 @@ __device__ void combine_tile(const FusedParams &p, const Tables &tb, int tau, in
   }
 }
 
+// Bounded wait until *ctr >= target (acquire); false (and STATUS_TIMEOUT) if
+// it gives up.  Lane 0 polls; the whole warp returns the result.
+__device__ __forceinline__ bool warp_wait_count(const int *ctr, int target, int *status,
+                                                unsigned long long limit_ns) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0 && ld_acquire(ctr) < target) {
+    const uint64_t t0 = global_timer_ns();
+    unsigned ns = 32;
+    while (ld_acquire(ctr) < target) {
+      if (global_timer_ns() - t0 > limit_ns) {
+        set_status(status, STATUS_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(ns);
+      if (ns < 256) ns <<= 1;
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 // One phase's compute: this warp's pieces in order, consuming the ring
 // stages that issue_next filled.  Returns false if a wait gave up (the ring
 // is drained first).
@@ -362,6 +388,16 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       p.y[prow * p.H + r0 + 8] = hi;
     }
   };
+  // Gate/up: after an item's h rows are stored, count it on its pair group
+  // (active expert a, group of its pairs); the down pass reads a group's h
+  // rows once all I/8 gate/up items of the group have counted themselves.
+  auto group_done = [&](const Item &it, int a_item) {
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(&p.grp_done[tb.gbase[a_item] + (it.pi0 - tb.aoff[a_item]) / p.group], 1);
+    }
+  };
   // After a down item's rows are stored: count it on its output tile; the
   // item that completes the tile combines it.
   auto tile_done = [&](int tau) {
@@ -388,8 +424,22 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
   Piece pc;
   bool have = piece_at(tb, P, P.x_lo, a, pc);
   bool ok = true;
+  int ready_group = -1;   // down: the last pair group seen complete
   while (have && ok) {
     const Item it = item_of(tb, P, p.group, pc.item, a);
+    int a_item = a;       // the active expert of this piece
+    while (tb.gbase[a_item + 1] * P.tiles <= pc.item) ++a_item;
+    if (!kGateUp) {
+      const int grp = tb.gbase[a_item] + (it.pi0 - tb.aoff[a_item]) / p.group;
+      if (grp != ready_group) {
+        if (!warp_wait_count(p.grp_done + grp, p.I / 8, p.status, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        __threadfence();
+        ready_group = grp;
+      }
+    }
     const int ntn = (it.ntok + 7) >> 3;
     const int x = pc.item * G + pc.g0;   // this piece's place in the sequence
     int a_nx = a;
@@ -419,7 +469,7 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       const uint8_t *stq = rg.base + slot * rg.stage_bytes;
       const uint8_t *sts = stq + (size_t)kc * 8;
       const int ng = min(gpc, pc.g1 - cg);
-#pragma unroll 2
+#pragma unroll(NT == 1 ? 2 : 1)
       for (int j = 0; j < ng; ++j) {
         // this group's activation fragments (L1-resident rows), loaded ahead
         // of the weight conversion that hides their latency
@@ -525,7 +575,8 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
           if (nt < ntn && n < it.ntok)
             emit(it, n, v ? acc[nt][0].y : acc[nt][0].x, v ? acc[nt][1].y : acc[nt][1].x);
         }
-      if (!kGateUp) tile_done(it.tau);
+      if (kGateUp) group_done(it, a_item);
+      else tile_done(it.tau);
     } else {
       // a piece of an item cut by share boundaries: store the partial sums,
       // count the piece; the last piece to arrive adds all of them in warp
@@ -574,7 +625,8 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
           }
         __syncwarp();
         if (lane == 0) *ctr = 0;  // ready for the next launch
-        if (!kGateUp) tile_done(it.tau);
+        if (kGateUp) group_done(it, a_item);
+        else tile_done(it.tau);
       }
     }
     pc = pc_nx;
@@ -920,8 +972,9 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     for (int s = 0; s < rg.stages; ++s) issue_next(cur, rg, tb, ph, p.group, gpc, p.kc, lane);
     if (!run_phase<true, NT, FMT>(p, tb, ph, 0, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
   }
-  live = grid_sync(p.bar + 2, abort_flag, p.status, p.wait_ns) && live;
-  if (live) {
+  // the down pass waits per pair group for the gate/up items it reads (no
+  // grid barrier); a warp that gave up in the gate/up pass does not start it
+  if (live && !*abort_flag) {
     if (!run_phase<false, NT, FMT>(p, tb, ph, 1, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
     // no combine happens if no expert item ran at all: every token is then
     // one with an unbound expert, and its output row is zero
@@ -933,15 +986,19 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   // before the CTA exits
   drain_ring(rg, p.status);
 
-  // ---- exit: the last CTA out resets the barrier counters
+  // ---- exit: the last CTA out resets the barrier and pair-group counters
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    if (atomicAdd(p.bar + 3, 1) == (int)gridDim.x - 1) {
-      p.bar[0] = p.bar[1] = p.bar[2] = 0;
-      __threadfence();
-      p.bar[3] = 0;
-    }
+    tb.misc[3] = atomicAdd(p.bar + 3, 1) == (int)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (tb.misc[3]) {
+    for (int i = tid; i < T * kS; i += blockDim.x) p.grp_done[i] = 0;
+    if (tid == 0) p.bar[0] = p.bar[1] = p.bar[2] = 0;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) p.bar[3] = 0;
   }
 }
 

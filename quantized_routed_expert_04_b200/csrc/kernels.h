@@ -47,7 +47,7 @@ __global__ void combine_kernel(const float *y, const int32_t *idx, const float *
 //
 // One work item = (active expert, group of <= 16 of its pairs, one 16-row
 // weight tile: 8 gate + 8 up rows, or 16 down rows).
-constexpr int kFusedWarps = 12;                     // warps per CTA, each with its own ring
+constexpr int kFusedWarps = 16;                     // warps per CTA, each with its own ring
 constexpr int kMmMaxStages = 8;                     // stages per warp ring
 constexpr int kMmMaxGroup = 16;                     // pairs per item (two n8 MMA tiles)
 constexpr int kMmSlotFloats = kMmMaxGroup * 16;     // partial sums of one piece: pairs x rows
@@ -74,7 +74,8 @@ struct FusedParams {
   float *partial;           // [warps of the grid][2][kMmSlotFloats]
   int *cut_cnt;             // [2][warps of the grid]   } zero between launches
   int *tile_cnt;            // [H/16]                   } (each resets what it
-  int *bar;                 // [4] grid barriers, exit  }  used)
+  int *bar;                 // [4] grid barriers, exit  }  used, or the last CTA
+  int *grp_done;            // [T*(k+S)] gate/up items done per pair group  }  out resets)
   int *status;
   __nv_bfloat16 *out;       // [T][H]
 };

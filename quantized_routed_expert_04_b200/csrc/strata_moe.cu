@@ -135,7 +135,8 @@ size_t fused_partial_bytes(const strata_moe *h) {
   return sizeof(float) * 2 * (size_t)kFusedWarps * h->num_sms * kMmSlotFloats;
 }
 size_t fused_counter_bytes(const strata_moe *h) {
-  return sizeof(int) * (4 + 2 * (size_t)kFusedWarps * h->num_sms + (size_t)h->H / 16);
+  return sizeof(int) * (4 + 2 * (size_t)kFusedWarps * h->num_sms + (size_t)h->H / 16 +
+                        (size_t)kSmallT * (kMaxTopK + kMaxShared));
 }
 
 strata_status grow_workspace(strata_moe *h, int T) {
@@ -416,6 +417,7 @@ strata_status run_fused(strata_moe *h, const void *x, int T, const int32_t *idx_
   p.bar = h->counters;
   p.cut_cnt = h->counters + 4;
   p.tile_cnt = h->counters + 4 + 2 * kFusedWarps * h->num_sms;
+  p.grp_done = p.tile_cnt + h->H / 16;
   p.status = h->status;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.glob = h->layout.glob;
