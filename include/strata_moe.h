@@ -356,10 +356,11 @@ strata_status strata_arena_prefill(strata_arena *a, const void *x_bf16, int n_to
  * device's multiprocessor count, about
  *     4*T*n_experts + 8*T*top_k + 4*(3N + 2) + 12*P + 2*T*hidden
  *       + 2*P*inter + 4*P*hidden + 8*T*max(n_experts, M)
- *       + 4*(4 + 24*M + hidden/16) + 24576*M  bytes
+ *       + 4*(2308 + 32*M + hidden/16) + 65536*M  bytes
  * (each term rounded up to 256; the last three terms are the decode
- * kernel's router partial sums, its barrier, cut-item and tile counters and
- * its two partial-sum slots per warp, 3.7 MB on 148 multiprocessors);
+ * kernel's router partial sums, its barrier, cut-item, tile and pair-group
+ * counters and its two partial-sum slots per warp and phase, 9.7 MB on 148
+ * multiprocessors);
  * a request beyond either limit returns STRATA_ERR_SCRATCH_LIMIT and
  * enqueues nothing.  The current device must be the handle's device
  * (otherwise INVALID_ARG).  The first call on a device looks up the array's

@@ -124,6 +124,20 @@ __device__ __forceinline__ int ld_acquire(const int *ptr) {
   return v;
 }
 
+// Counter increments that publish the writes before them: a release
+// reduction (the warp's other lanes' writes are ordered before it by a warp
+// barrier), or an acquire-release add whose caller also reads what the
+// earlier increments published.
+__device__ __forceinline__ void red_release_add(int *ptr, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ int atom_acq_rel_add(int *ptr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v)
+               : "memory");
+  return old;
+}
+
 // Ring-stage wait of one warp (lane 0 polls, with the given limit); once the
 // phase is complete every lane observes it itself (acquiring the stage's
 // bytes).
@@ -393,22 +407,17 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
   // rows once all I/8 gate/up items of the group have counted themselves.
   auto group_done = [&](const Item &it, int a_item) {
     __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      atomicAdd(&p.grp_done[tb.gbase[a_item] + (it.pi0 - tb.aoff[a_item]) / p.group], 1);
-    }
+    if (lane == 0)
+      red_release_add(&p.grp_done[tb.gbase[a_item] + (it.pi0 - tb.aoff[a_item]) / p.group], 1);
   };
   // After a down item's rows are stored: count it on its output tile; the
   // item that completes the tile combines it.
   auto tile_done = [&](int tau) {
     __syncwarp();
     int last = 0;
-    if (lane == 0) {
-      __threadfence();
-      last = atomicAdd(&p.tile_cnt[tau], 1) == tb.misc[1] - 1;
-    }
+    if (lane == 0) last = atom_acq_rel_add(&p.tile_cnt[tau], 1) == tb.misc[1] - 1;
     if (__shfl_sync(0xffffffffu, last, 0)) {
-      __threadfence();
+      __syncwarp();
       combine_tile(p, tb, tau, lane);
       __syncwarp();
       if (lane == 0) p.tile_cnt[tau] = 0;  // ready for the next launch
@@ -436,7 +445,6 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
           ok = false;
           break;
         }
-        __threadfence();
         ready_group = grp;
       }
     }
@@ -584,7 +592,7 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       const int x_item = pc.item * G;
       const int w_first = share_owner(P, x_item), w_last = share_owner(P, x_item + G - 1);
       const int my_slot = x == P.x_lo ? 0 : 1;
-      float *mine = p.partial + ((size_t)wg * 2 + my_slot) * kMmSlotFloats;
+      float *mine = p.partial + (((size_t)phi * Wtot + wg) * 2 + my_slot) * kMmSlotFloats;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -600,12 +608,9 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       int *ctr = p.cut_cnt + (size_t)phi * Wtot + w_first;
       __syncwarp();
       int last = 0;
-      if (lane == 0) {
-        __threadfence();
-        last = atomicAdd(ctr, 1) == n_pieces - 1;
-      }
+      if (lane == 0) last = atom_acq_rel_add(ctr, 1) == n_pieces - 1;
       if (__shfl_sync(0xffffffffu, last, 0)) {
-        __threadfence();
+        __syncwarp();
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -616,7 +621,7 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
               for (int w = w_first; w <= w_last; ++w) {
                 if (share_cut(P, w + 1) == share_cut(P, w)) continue;  // empty share
                 const int slot = (w == w_first && share_cut(P, w) != x_item) ? 1 : 0;
-                const float *src = p.partial + ((size_t)w * 2 + slot) * kMmSlotFloats;
+                const float *src = p.partial + (((size_t)phi * Wtot + w) * 2 + slot) * kMmSlotFloats;
                 lo += __ldcg(src + n * 16 + g);
                 hi += __ldcg(src + n * 16 + g + 8);
               }

@@ -71,7 +71,7 @@ struct FusedParams {
   float *w;                 // [T][k]
   __half *x16, *h16;        // packed activations [T][H], SwiGLU output [P][I]
   float *y;                 // [P][H]
-  float *partial;           // [warps of the grid][2][kMmSlotFloats]
+  float *partial;           // [phase][warps of the grid][2][kMmSlotFloats]
   int *cut_cnt;             // [2][warps of the grid]   } zero between launches
   int *tile_cnt;            // [H/16]                   } (each resets what it
   int *bar;                 // [4] grid barriers, exit  }  used, or the last CTA

@@ -128,11 +128,13 @@ cudaError_t launch(strata_moe *h, int phase, void (*kern)(Exp...), dim3 grid, di
   return err;
 }
 
-// Decode kernel workspace: two partial-sum slots per warp of the grid; the
-// counters: 4 barrier/exit counters, one cut-item counter per warp and phase,
-// one tile counter per 16 output rows.
+// Decode kernel workspace: two partial-sum slots per warp of the grid and
+// phase (a warp may start its down-projection pieces while the last piece of
+// one of its cut gate/up items has yet to read its slot); the counters: 4
+// barrier/exit counters, one cut-item counter per warp and phase, one tile
+// counter per 16 output rows, one readiness counter per pair group.
 size_t fused_partial_bytes(const strata_moe *h) {
-  return sizeof(float) * 2 * (size_t)kFusedWarps * h->num_sms * kMmSlotFloats;
+  return sizeof(float) * 2 * 2 * (size_t)kFusedWarps * h->num_sms * kMmSlotFloats;
 }
 size_t fused_counter_bytes(const strata_moe *h) {
   return sizeof(int) * (4 + 2 * (size_t)kFusedWarps * h->num_sms + (size_t)h->H / 16 +
