@@ -108,6 +108,7 @@ struct Cursor {  // the copy-issue position, running over the G then the D piece
   int ph, x, a, cg;
   Piece pc;
   bool have;
+  const uint8_t *qsrc, *ssrc;  // the next stage's packed weights and scales
 };
 
 __device__ __forceinline__ uint4 ld_v4(const void *ptr) {
@@ -227,51 +228,51 @@ __device__ __forceinline__ Item item_of(const Tables &tb, const PhaseInfo &ph, i
   return it;
 }
 
-// 16-byte asynchronous global -> shared copy (L2 only), and the arrival on a
-// stage barrier once all of this thread's earlier such copies have landed.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+// Move the cursor to the first piece at or after c.x in phase c.ph (and on
+// into the D share once the G share is done); caches the piece's sources.
+__device__ __forceinline__ void cursor_seek(Cursor &c, const Tables &tb, const PhaseInfo *ph,
+                                            int group) {
+  while (true) {
+    const PhaseInfo &P = ph[c.ph];
+    c.have = piece_at(tb, P, c.x, c.a, c.pc);
+    if (c.have) {
+      const Item it = item_of(tb, P, group, c.pc.item, c.a);
+      const size_t g0 = (size_t)it.tau * P.groups + (size_t)c.pc.g0;
+      c.qsrc = it.blob + P.q_off + g0 * 1024;
+      c.ssrc = it.blob + P.s_off + g0 * 128;
+      c.cg = c.pc.g0;
+      return;
+    }
+    if (c.ph == 1) return;
+    c.ph = 1;
+    c.x = ph[1].x_lo;
+    c.a = 0;
+  }
 }
 
-// Issue the copies of the next stage: up to gpc K groups of the current piece
-// (packed weights and scales of 16 rows, ng KB + ng x 128 B), as 16-byte
-// asynchronous copies spread over the warp's 32 lanes; each lane then arrives
-// on the stage's barrier when its copies have landed (32 arrivals per phase).
+// Issue the next stage: up to gpc K groups of the current piece (packed
+// weights and scales of 16 rows: ng KB and ng x 128 B, each contiguous in the
+// blob) as two bulk asynchronous copies by lane 0, completing on the stage's
+// barrier as transaction bytes.
 __device__ __forceinline__ void issue_next(Cursor &c, Ring &rg, const Tables &tb,
                                            const PhaseInfo *ph, int group, int gpc, int kc,
                                            int lane) {
-  while (!c.have && c.ph < 1) {
-    ++c.ph;
-    c.x = ph[c.ph].x_lo;
-    c.a = 0;
-    c.have = piece_at(tb, ph[c.ph], c.x, c.a, c.pc);
-    if (c.have) c.cg = c.pc.g0;
-  }
   if (!c.have) return;
-  const PhaseInfo &P = ph[c.ph];
-  const Item it = item_of(tb, P, group, c.pc.item, c.a);
   const int slot = (int)(rg.issued % rg.stages);
-  uint8_t *dst = rg.base + slot * rg.stage_bytes;
   const int ng = min(gpc, c.pc.g1 - c.cg);
-  {
-    const size_t g0 = (size_t)it.tau * P.groups + (size_t)c.cg;
-    const uint8_t *qsrc = it.blob + P.q_off + g0 * 1024;
-    const uint8_t *ssrc = it.blob + P.s_off + g0 * 128;
-    for (int ch = lane; ch < ng * 64; ch += 32) cp_async16(dst + ch * 16, qsrc + ch * 16);
-    if (lane < ng * 8) cp_async16(dst + (size_t)kc * 8 + lane * 16, ssrc + lane * 16);
-    cp_async_arrive(&rg.full[slot]);
+  if (lane == 0) {
+    uint8_t *dst = rg.base + slot * rg.stage_bytes;
+    mbar_arrive_expect_tx(&rg.full[slot], (uint32_t)ng * 1152u);
+    bulk_g2s(dst, c.qsrc, (uint32_t)ng * 1024u, &rg.full[slot]);
+    bulk_g2s(dst + (size_t)kc * 8, c.ssrc, (uint32_t)ng * 128u, &rg.full[slot]);
   }
   ++rg.issued;
   c.cg += ng;
+  c.qsrc += (size_t)ng * 1024;
+  c.ssrc += (size_t)ng * 128;
   if (c.cg == c.pc.g1) {
-    c.x = c.pc.item * P.groups + c.pc.g1;   // just past this piece (skipped ones included)
-    c.have = piece_at(tb, P, c.x, c.a, c.pc);
-    if (c.have) c.cg = c.pc.g0;
+    c.x = c.pc.item * ph[c.ph].groups + c.pc.g1;   // just past this piece (skipped ones included)
+    cursor_seek(c, tb, ph, group);
   }
 }
 
@@ -698,7 +699,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   // the slot table, read with per-lane indices below, into shared memory
   for (int i = tid; i < nid; i += blockDim.x) tb.ptr[i] = p.table.ptr[i];
   if (lane == 0)
-    for (int s = 0; s < p.stages; ++s) mbar_init(&rg.full[s], 32);
+    for (int s = 0; s < p.stages; ++s) mbar_init(&rg.full[s], 1);
   if (tid == 0) {
     *abort_flag = 0;
     fence_mbar_init();
@@ -783,7 +784,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
         if (tid < nt) {
           double v = tb.part[tid];
           for (int w = 1; w < kFW; ++w) v += tb.part[w * 8 + tid];
-          p.rpart[((size_t)e * splits + sp) * T + t0 + tid] = v;
+          p.rpart[((size_t)sp * T + t0 + tid) * E + e] = v;
         }
         __syncthreads();
       }
@@ -797,8 +798,8 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   float *s_logit = reinterpret_cast<float *>(smem);
   const bool redundant = T <= kFW;
   auto logit_of = [&](int t, int e) -> float {
-    double v = __ldcg(p.rpart + ((size_t)e * splits) * T + t);
-    for (int sp = 1; sp < splits; ++sp) v += __ldcg(p.rpart + ((size_t)e * splits + sp) * T + t);
+    double v = __ldcg(p.rpart + (size_t)t * E + e);
+    for (int sp = 1; sp < splits; ++sp) v += __ldcg(p.rpart + ((size_t)sp * T + t) * E + e);
     if (p.bias) v += (double)p.bias[e];
     return (float)v;
   };
@@ -869,43 +870,56 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     }
     __syncthreads();
     if (warp == 0) {
-      // offsets by id, the active list and the pair groups per active expert
-      int carry = 0, acarry = 0, gcarry = 0, gbound = 0;
-      for (int i0 = 0; i0 < nid; i0 += 32) {
-        const int i = i0 + lane;
-        const int c = i < nid ? tb.cnt[i] : 0;
-        const int f = c > 0;
+      // offsets by id, the active list and the pair groups per active
+      // expert: each lane scans a contiguous run of ids, one warp scan joins
+      // the runs
+      const int per = (nid + 31) >> 5;
+      const int i0 = min(nid, lane * per), i1 = min(nid, i0 + per);
+      int sc = 0, sf = 0, sg = 0, sb = 0;
+      for (int i = i0; i < i1; ++i) {
+        const int c = tb.cnt[i];
         const int ng = (c + p.group - 1) / p.group;
-        const uint8_t *bp = i < nid ? tb.ptr[i] : nullptr;
-        int inc = c, finc = f, ginc = ng, binc = bp ? ng : 0;
+        sc += c;
+        sf += c > 0;
+        sg += ng;
+        sb += tb.ptr[i] ? ng : 0;
+      }
+      int ec = sc, ef = sf, eg = sg, eb = sb;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v1 = __shfl_up_sync(0xffffffffu, inc, o);
-          const int v2 = __shfl_up_sync(0xffffffffu, finc, o);
-          const int v3 = __shfl_up_sync(0xffffffffu, ginc, o);
-          const int v4 = __shfl_up_sync(0xffffffffu, binc, o);
-          if (lane >= o) {
-            inc += v1;
-            finc += v2;
-            ginc += v3;
-            binc += v4;
-          }
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v1 = __shfl_up_sync(0xffffffffu, ec, o);
+        const int v2 = __shfl_up_sync(0xffffffffu, ef, o);
+        const int v3 = __shfl_up_sync(0xffffffffu, eg, o);
+        const int v4 = __shfl_up_sync(0xffffffffu, eb, o);
+        if (lane >= o) {
+          ec += v1;
+          ef += v2;
+          eg += v3;
+          eb += v4;
         }
-        if (i < nid) {
-          tb.off[i] = carry + inc - c;
-          if (f) {
-            const int a = acarry + finc - 1;
-            tb.blob[a] = bp;
-            tb.aoff[a] = carry + inc - c;
-            tb.acnt[a] = c;
-            tb.gbase[a] = gcarry + ginc - ng;
-            if (!bp && blockIdx.x == 0) set_status(p.status, STATUS_NOT_BOUND);
-          }
+      }
+      const int carry = __shfl_sync(0xffffffffu, ec, 31);
+      const int acarry = __shfl_sync(0xffffffffu, ef, 31);
+      const int gcarry = __shfl_sync(0xffffffffu, eg, 31);
+      const int gbound = __shfl_sync(0xffffffffu, eb, 31);
+      ec -= sc;
+      ef -= sf;
+      eg -= sg;
+      for (int i = i0; i < i1; ++i) {
+        const int c = tb.cnt[i];
+        const int ng = (c + p.group - 1) / p.group;
+        const uint8_t *bp = tb.ptr[i];
+        tb.off[i] = ec;
+        if (c > 0) {
+          tb.blob[ef] = bp;
+          tb.aoff[ef] = ec;
+          tb.acnt[ef] = c;
+          tb.gbase[ef] = eg;
+          if (!bp && blockIdx.x == 0) set_status(p.status, STATUS_NOT_BOUND);
+          ++ef;
         }
-        carry += __shfl_sync(0xffffffffu, inc, 31);
-        acarry += __shfl_sync(0xffffffffu, finc, 31);
-        gcarry += __shfl_sync(0xffffffffu, ginc, 31);
-        gbound += __shfl_sync(0xffffffffu, binc, 31);
+        ec += c;
+        eg += ng;
       }
       if (lane == 0) {
         tb.off[nid] = carry;
@@ -972,8 +986,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
     }
     cur.x = ph[0].x_lo;
     cur.a = 0;
-    cur.have = piece_at(tb, ph[0], cur.x, cur.a, cur.pc);
-    if (cur.have) cur.cg = cur.pc.g0;
+    cursor_seek(cur, tb, ph, p.group);
     for (int s = 0; s < rg.stages; ++s) issue_next(cur, rg, tb, ph, p.group, gpc, p.kc, lane);
     if (!run_phase<true, NT, FMT>(p, tb, ph, 0, rg, cur, wg, lane, gpc, p.kc)) *abort_flag = 1;
   }

@@ -66,7 +66,7 @@ struct FusedParams {
   int group;                // pairs per item: 8 or 16
   unsigned long long wait_ns;  // limit of every wait that depends on other warps or copies
   size_t smem_tables;       // offset of the routing tables in dynamic shared memory
-  double *rpart;            // router partial sums [E][max(1, grid / E)][T]
+  double *rpart;            // router partial sums [max(1, grid / E)][T][E]
   int32_t *idx;             // [T][k] (used when more tokens than warps per CTA)
   float *w;                 // [T][k]
   __half *x16, *h16;        // packed activations [T][H], SwiGLU output [P][I]

@@ -7,9 +7,19 @@
 
 namespace strata {
 
+// Order-preserving map of an fp32 key to an unsigned integer (larger key,
+// larger integer; -0 and +0 equal; NaN below every other key), so that a
+// warp's largest key is one hardware warp reduction.
+__device__ __forceinline__ uint32_t topk_order_key(float f) {
+  if (f != f) return 0u;
+  const uint32_t b = f == 0.0f ? 0u : __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // One warp per token.  Lane l holds experts l, l+32, ...; k rounds of a warp
-// arg-max of the selection key (larger wins, equal keys: lower id wins).
-// Softmax routing: key = logit, weights = exp(l_j - l_0) / sum_j (the
+// arg-max of the selection key (larger wins, equal keys: lower id wins), each
+// round a max-reduction of the keys and a min-reduction of the ids that hold
+// it.  Softmax routing: key = logit, weights = exp(l_j - l_0) / sum_j (the
 // renormalised softmax of the selected experts).  Sigmoid routing: score =
 // 1 / (1 + exp(-l)) in double rounded to fp32, key = score + correction,
 // weights = score_j / (sum of the selected scores in selection order) *
@@ -20,42 +30,37 @@ template <int kPer, bool kShared>
 __device__ __forceinline__ void select_topk_warp_t(const float *__restrict__ logit_row, int E,
                                                    int k, const RouteMode &mode, int lane,
                                                    int &sel_e, float &sel_w) {
-  float key[kPer], val[kPer];   // val: logit (softmax) or score (sigmoid)
+  uint32_t key[kPer];
+  float val[kPer];   // logit (softmax) or score (sigmoid)
+  unsigned taken = 0;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
-    const float l = e < E ? (kShared ? logit_row[e] : __ldcg(logit_row + e)) : -INFINITY;
+    const float l = e < E ? (kShared ? logit_row[e] : __ldcg(logit_row + e)) : 0.0f;
     if (mode.sigmoid && e < E) {
       val[i] = (float)(1.0 / (1.0 + exp(-(double)l)));
-      key[i] = mode.corr ? __fadd_rn(val[i], mode.corr[e]) : val[i];
+      key[i] = topk_order_key(mode.corr ? __fadd_rn(val[i], mode.corr[e]) : val[i]);
     } else {
       val[i] = l;
-      key[i] = l;
+      key[i] = topk_order_key(l);
     }
+    if (e >= E) taken |= 1u << i;
   }
-  unsigned taken = 0;
   float v0 = 0.0f, z = 0.0f, my_v = 0.0f;
   int my_e = 0;
   for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY;
-    int be = 0x7fffffff;
+    // this lane's best untaken key (lowest id among equal keys)
+    uint32_t bk = 0u;
+    int bi = -1;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || key[i] > bk)) {
+    for (int i = 0; i < kPer; ++i)
+      if (!((taken >> i) & 1u) && (bi < 0 || key[i] > bk)) {
         bk = key[i];
-        be = e;
+        bi = i;
       }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (oe != 0x7fffffff && (be == 0x7fffffff || ok > bk || (ok == bk && oe < be))) {
-        bk = ok;
-        be = oe;
-      }
-    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
+    const uint32_t cand = bi >= 0 && bk == m ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+    const int be = (int)__reduce_min_sync(0xffffffffu, cand);
     // the winner's logit or score, from the lane that holds it
     float mine = 0.0f;
 #pragma unroll
