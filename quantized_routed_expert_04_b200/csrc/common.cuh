@@ -144,6 +144,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *s
 }
 
 // ---------------------------------------------------------------- bulk copy
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned source) into L2 ahead
+// of the copies that will read them; no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Plain (non-multicast) bulk copy global -> this CTA's shared memory; the
 // completion is counted on `bar` as transaction bytes.  Both addresses and
 // the size must be multiples of 16 bytes.

@@ -60,6 +60,7 @@ constexpr int kTcM = 128;          // weight rows per unit
 constexpr int kTcN = 256;          // pairs per chunk (max MMA N used)
 constexpr int kUnitPairs = 2 * kTcN;
 constexpr int kPkStages = 2;       // packed-weight stages
+constexpr int kPfUnits = 2;        // units whose weights are prefetched into L2 ahead
 constexpr int kPkGroups = 2;       // K groups (of 128) per packed stage
 constexpr int kAStages = 3;        // A ring: one 64-wide dequantised atom each
 constexpr int kBStages = 4;        // B ring: one 64-wide activation atom of one chunk each
@@ -67,8 +68,8 @@ constexpr int kDqWarps = 8;
 constexpr int kDqRows = kTcM / kDqWarps;    // weight rows per dequant warp
 static_assert(kDqRows % 8 == 0, "dequant warps cover whole 8-row groups");
 constexpr int kEpiWarps = 8;                // two per TMEM lane quarter
-constexpr int kPkWarp = 2 + kDqWarps + kEpiWarps;   // the last warp
-constexpr int kTcThreads = 32 * (kPkWarp + 1);
+constexpr int kTcWarps = 3 + kDqWarps + kEpiWarps;
+constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kAccCols = 256;      // TMEM columns per accumulator
 constexpr uint32_t kTmemCols = 512;
 
@@ -94,6 +95,40 @@ __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *statu
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
+
+// Warp roles.  A warp issues from the scheduler of warp id % 4; the single
+// thread that issues every MMA gets scheduler 1 with only warps that mostly
+// sleep (two epilogue warps, both producers), while the dequant warps, the
+// busiest, share schedulers 0, 2 and 3 with the other epilogue warps.  An
+// epilogue warp may only read its own TMEM lane quarter (warp id % 4).
+enum TcRole : int { kRoleAct, kRoleMma, kRoleDq, kRoleEpi, kRoleWgt };
+struct TcWarp {
+  int role, idx;  // idx: dequant warp 0..7, or epilogue warp 0..7 (= 2 quarter + half)
+};
+__device__ __forceinline__ TcWarp tc_warp(int warp) {
+  switch (warp) {
+    case 1: return {kRoleMma, 0};
+    case 13: return {kRoleWgt, 0};
+    case 17: return {kRoleAct, 0};
+    case 0: return {kRoleDq, 0};
+    case 4: return {kRoleDq, 1};
+    case 8: return {kRoleDq, 2};
+    case 2: return {kRoleDq, 3};
+    case 6: return {kRoleDq, 4};
+    case 10: return {kRoleDq, 5};
+    case 3: return {kRoleDq, 6};
+    case 7: return {kRoleDq, 7};
+    case 12: return {kRoleEpi, 0};
+    case 16: return {kRoleEpi, 1};
+    case 5: return {kRoleEpi, 2};
+    case 9: return {kRoleEpi, 3};
+    case 14: return {kRoleEpi, 4};
+    case 18: return {kRoleEpi, 5};
+    case 11: return {kRoleEpi, 6};
+    default: return {kRoleEpi, 7};  // 15
+  }
+}
+static_assert(kTcWarps == 19 && kDqWarps == 8 && kEpiWarps == 8, "role table");
 
 struct Unit {
   const uint8_t *blob;
@@ -163,6 +198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int *unit_base = t_cnt + kMaxIds;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const TcWarp role = tc_warp(warp);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPkStages; ++s) {
       mbar_init(&pk_full[s], 1);
@@ -239,7 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return un;
   };
 
-  if (warp == 0) {
+  if (role.role == kRoleAct) {
     // -------------------------------------------------------- activation producer
     uint32_t issued = 0;
     RingPos rb;
@@ -275,13 +311,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (uint32_t m = issued > kBStages ? issued - kBStages : 0; m < issued; ++m)
         (void)wwait(&fullB[m % kBStages], (m / kBStages) & 1u, p.status);
     }
-  } else if (warp == kPkWarp) {
+  } else if (role.role == kRoleWgt) {
     // -------------------------------------------------------- weight producer
     uint32_t pk_cnt = 0;
     bool ok = true;
-    int a = 0;
+    int a = 0, a_pf = 0;
+    // the packed weights of a unit stream in from HBM through this small
+    // ring; L2 prefetches of the units ahead hide their latency
+    auto prefetch_unit = [&](int v) {
+      if (v >= n_units || lane >= 8) return;
+      const Unit nx = decode(v, a_pf);
+      const int tile = nx.rt * 8 + lane;
+      bulk_prefetch_l2(nx.blob + p.q_off + (size_t)tile * G * 1024, (uint32_t)G * 1024u);
+      bulk_prefetch_l2(nx.blob + p.s_off + (size_t)tile * G * 128, (uint32_t)G * 128u);
+    };
+    for (int i = 0; i < kPfUnits; ++i) prefetch_unit(blockIdx.x + i * gridDim.x);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit un = decode(u, a);
+      prefetch_unit(u + kPfUnits * gridDim.x);
       for (int g = 0; g < G && ok; g += kPkGroups) {
         const int s = (int)(pk_cnt % kPkStages);
         if (!wwait(&pk_empty[s], ((pk_cnt / kPkStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
@@ -305,7 +352,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (uint32_t m = pk_cnt > kPkStages ? pk_cnt - kPkStages : 0; m < pk_cnt; ++m)
         (void)wwait(&pk_full[m % kPkStages], (m / kPkStages) & 1u, p.status);
     }
-  } else if (warp == 1) {
+  } else if (role.role == kRoleMma) {
     // -------------------------------------------------------- MMA issue
     // One thread does it all: per atom one wait for A, per chunk one wait for
     // B, four MMAs and one commit, so the tensor pipe's queue never runs dry
@@ -315,6 +362,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       AccTrack acc;
       bool ok = true;
       int a = 0;
+      // stage 0's descriptors; a stage adds its offset / 16 to the address
+      // field, a 16-element K step (32 bytes) adds 2
+      const uint64_t a_desc0 = umma_desc_sw128(smem_u32(smem + kOffA));
+      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(smem + kOffB));
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const Unit un = decode(u, a);
         const int nc = un.chunks();
@@ -328,7 +379,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int at = 0; at < 2 * G && ok; ++at) {
           if (!mbar_wait(&fullA[ra.st], ra.ph, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + kOffA + ra.st * kAStageBytes);
+          const uint64_t ad = a_desc0 + (uint64_t)((ra.st * kAStageBytes) >> 4);
           for (int c = 0; c < nc; ++c) {
             if (at == 0) {
               // the accumulator must have been drained by the epilogue
@@ -338,11 +389,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (!mbar_wait(&fullB[rb.st], rb.ph, p.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t b_addr = smem_u32(smem + kOffB + rb.st * kBStageBytes);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              umma_f16(d_tmem[c], umma_desc_sw128(a_addr + j * 32),
-                       umma_desc_sw128(b_addr + j * 32), idesc[c], (at > 0 || j > 0) ? 1u : 0u);
+            const uint64_t bd = b_desc0 + (uint64_t)((rb.st * kBStageBytes) >> 4);
+            umma_f16(d_tmem[c], ad, bd, idesc[c], at > 0 ? 1u : 0u);
+            umma_f16(d_tmem[c], ad + 2, bd + 2, idesc[c], 1u);
+            umma_f16(d_tmem[c], ad + 4, bd + 4, idesc[c], 1u);
+            umma_f16(d_tmem[c], ad + 6, bd + 6, idesc[c], 1u);
             umma_commit(&emptyB[rb.st]);
             rb.next(kBStages);
           }
@@ -356,9 +407,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 2 + kDqWarps) {
+  } else if (role.role == kRoleDq) {
     // -------------------------------------------------------- dequant
-    const int dw = warp - 2;
+    const int dw = role.idx;
     const int w = lane & 3;
     const int q = lane >> 2;
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
@@ -435,11 +486,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     if (__any_sync(0xffffffffu, big_scale) && lane == 0) set_status(p.status, STATUS_RANGE);
-  } else if (warp < kPkWarp) {
+  } else {
     // -------------------------------------------------------- epilogue
-    const int ew = warp - 2 - kDqWarps;       // 0 .. kEpiWarps - 1
+    const int ew = role.idx;                  // 0 .. kEpiWarps - 1
     const int qd = warp & 3;                  // TMEM lane quarter of this warp
-    const int cpar = ew >> 2;                 // which alternate 32-column blocks
+    const int cpar = ew & 1;                  // which alternate 32-column blocks
     float *stage = reinterpret_cast<float *>(smem + kOffEpi + ew * 1024);
     AccTrack acc;
     bool ok = true, big_h = false;
@@ -467,22 +518,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           if (kGateUp) {
             // lane L: blob tile 2 qd + L / 16, tile row L % 16 (gate if < 8);
-            // the gate lane computes the even columns, its up partner (L ^ 8)
-            // the odd ones
+            // of each column pair the gate lane computes the even column and
+            // its up partner (L ^ 8) the odd one: each sends the partner the
+            // value of the partner's column (one shuffle per pair, no branch)
             __half *hs = reinterpret_cast<__half *>(stage);  // [32 pairs][16]
             const bool is_up = (lane & 15) >= 8;
             const int pos16 = 8 * (lane >> 4) + packed_pos<FMT>(lane & 7);
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              const float pv = __shfl_xor_sync(0xffffffffu, v[t], 8);
-              if ((t & 1) == (is_up ? 1 : 0)) {
-                const float gv = is_up ? pv : v[t];
-                const float uv = is_up ? v[t] : pv;
-                const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-                // (columns past the chunk's pairs hold stale accumulators)
-                big_h |= col0 + t < cn && fabsf(hv) >= kF16Overflow;
-                hs[t * 16 + pos16] = __float2half_rn(hv);
-              }
+            for (int t = 0; t < 32; t += 2) {
+              const float mine = is_up ? v[t + 1] : v[t];
+              const float other = __shfl_xor_sync(0xffffffffu, is_up ? v[t] : v[t + 1], 8);
+              const float gv = is_up ? other : mine;
+              const float uv = is_up ? mine : other;
+              const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+              const int c = t + (is_up ? 1 : 0);
+              // (columns past the chunk's pairs hold stale accumulators)
+              big_h |= col0 + c < cn && fabsf(hv) >= kF16Overflow;
+              hs[c * 16 + pos16] = __float2half_rn(hv);
             }
             __syncwarp();
 #pragma unroll
