@@ -85,7 +85,8 @@ struct PhaseInfo {
   int groups;           // K groups of 128 per tile row
   size_t q_off, s_off;  // weight and scale sections
   int x_lo, x_hi;       // this warp's share of the (item, group) sequence
-  int q, r;             // share sizes: the first r warps take q + 1 groups
+  int q, r;             // share sizes: the first r warps take q + 1 stages
+  int unit, total;      // K groups per stage, groups in the phase
 };
 
 struct Piece {
@@ -191,14 +192,17 @@ __device__ bool grid_sync(int *ctr, volatile int *abort_flag, int *status,
   return !*abort_flag;
 }
 
+// Shares are whole ring stages (ph.unit K groups) of the phase's sequence of
+// ph.total groups, so that a piece that starts a share starts a full stage.
 __device__ __forceinline__ int share_cut(const PhaseInfo &ph, int w) {
-  return w * ph.q + min(w, ph.r);
+  return min(ph.total, (w * ph.q + min(w, ph.r)) * ph.unit);
 }
 
 // The warp whose share holds position x.
 __device__ __forceinline__ int share_owner(const PhaseInfo &ph, int x) {
+  const int s = x / ph.unit;
   const int big = ph.r * (ph.q + 1);
-  return x < big ? x / (ph.q + 1) : ph.r + (x - big) / ph.q;
+  return s < big ? s / (ph.q + 1) : ph.r + (s - big) / ph.q;
 }
 
 // First piece of a bound expert at or after x in this warp's share.
@@ -406,10 +410,18 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
   // Gate/up: after an item's h rows are stored, count it on its pair group
   // (active expert a, group of its pairs); the down pass reads a group's h
   // rows once all I/8 gate/up items of the group have counted themselves.
+  // The count is a release, which waits until the stores before it are
+  // performed; it is issued after the next stage's math (or at the end of
+  // the share), when they long are, so that the warp does not stall on it.
+  int pending_grp = -1;
+  auto flush_group = [&]() {
+    if (lane == 0 && pending_grp >= 0) red_release_add(&p.grp_done[pending_grp], 1);
+    pending_grp = -1;
+  };
   auto group_done = [&](const Item &it, int a_item) {
     __syncwarp();
-    if (lane == 0)
-      red_release_add(&p.grp_done[tb.gbase[a_item] + (it.pi0 - tb.aoff[a_item]) / p.group], 1);
+    flush_group();
+    pending_grp = tb.gbase[a_item] + (it.pi0 - tb.aoff[a_item]) / p.group;
   };
   // After a down item's rows are stored: count it on its output tile; the
   // item that completes the tile combines it.
@@ -563,6 +575,7 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
       cg += ng;
       // the stage's bytes are in registers now: refill it
       __syncwarp();
+      if (kGateUp) flush_group();
       issue_next(cur, rg, tb, ph, p.group, gpc, kc, lane);
     }
     if (!ok) break;
@@ -638,6 +651,10 @@ __device__ bool run_phase(const FusedParams &p, const Tables &tb, const PhaseInf
     pc = pc_nx;
     have = have_nx;
     a = a_nx;
+  }
+  if (kGateUp) {
+    __syncwarp();
+    flush_group();
   }
   if (kGateUp && __any_sync(0xffffffffu, any_big) && lane == 0) set_status(p.status, STATUS_RANGE);
   if (!ok) drain_ring(rg, p.status);
@@ -979,8 +996,11 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
       P.q_off = phi == 0 ? p.guq : p.dq;
       P.s_off = phi == 0 ? p.gus : p.ds;
       const int total = n_groups * P.tiles * P.groups;
-      P.q = total / Wtot;
-      P.r = total - P.q * Wtot;
+      const int slots = (total + gpc - 1) / gpc;
+      P.unit = gpc;
+      P.total = total;
+      P.q = slots / Wtot;
+      P.r = slots - P.q * Wtot;
       P.x_lo = share_cut(P, wg);
       P.x_hi = share_cut(P, wg + 1);
     }
