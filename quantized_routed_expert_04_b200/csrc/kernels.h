@@ -101,7 +101,8 @@ struct TcParams {
 #include <cuda.h>
 namespace strata {
 template <bool kGateUp, int FMT>
-__global__ void expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b64,
+__global__ void expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b16,
+                                 const __grid_constant__ CUtensorMap tmap_b64,
                                  const __grid_constant__ CUtensorMap tmap_b256);
 __global__ void gather_rows_kernel(const __half *x16, const int *pair_tok, const int *n_pairs_dev,
                                    int H, int P_cap, __half *xp);

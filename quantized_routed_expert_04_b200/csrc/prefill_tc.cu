@@ -179,7 +179,8 @@ static_assert(kTcSmem <= 232448, "shared memory budget");
 
 template <bool kGateUp, int FMT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b64,
+    expert_tc_kernel(TcParams p, const __grid_constant__ CUtensorMap tmap_b16,
+                     const __grid_constant__ CUtensorMap tmap_b64,
                      const __grid_constant__ CUtensorMap tmap_b256) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&acc_empty[s], kEpiWarps);
     }
     fence_mbar_init();
+    prefetch_tmap(&tmap_b16);
     prefetch_tmap(&tmap_b64);
     prefetch_tmap(&tmap_b256);
   }
@@ -288,17 +290,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < nc; ++c) {
           if (!wwait(&emptyB[rb.st], rb.ph ^ 1u, p.status)) { ok = false; break; }
           const int cn = un.chunk_n(c), row0 = un.pi0 + c * kTcN;
-          const bool wide = cn > 192;            // one 256-row box, else 64-row boxes
-          const int nb = wide ? 1 : (cn + 63) / 64;
-          const uint32_t tx = wide ? 32768u : nb * 8192u;
+          // one 256-row box, else 64-row boxes and 16-row boxes for the rest
+          // (rows land at 128 bytes each whatever the box, so the swizzled
+          // layout is the same)
+          const bool wide = cn > 192;
+          const int n64 = wide ? 0 : cn / 64;
+          const int n16 = wide ? 0 : (cn - 64 * n64 + 15) / 16;
+          const uint32_t tx = wide ? 32768u : n64 * 8192u + n16 * 2048u;
           uint8_t *dst = smem + kOffB + rb.st * kBStageBytes;
           if (lane == 0) {
             mbar_arrive_expect_tx(&fullB[rb.st], tx);
-            if (wide)
+            if (wide) {
               tma_load_2d(dst, &tmap_b256, at * 64, row0, &fullB[rb.st]);
-            else
-              for (int q = 0; q < nb; ++q)
+            } else {
+              for (int q = 0; q < n64; ++q)
                 tma_load_2d(dst + q * 8192, &tmap_b64, at * 64, row0 + q * 64, &fullB[rb.st]);
+              for (int q = 0; q < n16; ++q)
+                tma_load_2d(dst + n64 * 8192 + q * 2048, &tmap_b16, at * 64, row0 + 64 * n64 + 16 * q,
+                            &fullB[rb.st]);
+            }
           }
           __syncwarp();
           ++issued;
@@ -590,14 +600,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 template __global__ void expert_tc_kernel<true, kFmtInt4>(TcParams,
                                                          const __grid_constant__ CUtensorMap,
+                                                         const __grid_constant__ CUtensorMap,
                                                          const __grid_constant__ CUtensorMap);
 template __global__ void expert_tc_kernel<false, kFmtInt4>(TcParams,
+                                                          const __grid_constant__ CUtensorMap,
                                                           const __grid_constant__ CUtensorMap,
                                                           const __grid_constant__ CUtensorMap);
 template __global__ void expert_tc_kernel<true, kFmtNvfp4>(TcParams,
                                                           const __grid_constant__ CUtensorMap,
+                                                          const __grid_constant__ CUtensorMap,
                                                           const __grid_constant__ CUtensorMap);
 template __global__ void expert_tc_kernel<false, kFmtNvfp4>(TcParams,
+                                                           const __grid_constant__ CUtensorMap,
                                                            const __grid_constant__ CUtensorMap,
                                                            const __grid_constant__ CUtensorMap);
 

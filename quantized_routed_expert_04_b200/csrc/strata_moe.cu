@@ -273,8 +273,9 @@ strata_status run_tc_passes(strata_moe *h, int T, const ExpertTable &table, bool
     p.status = h->status;
     p.quiet_unbound = quiet ? 1 : 0;
     p.glob_off = h->layout.glob;
-    CUtensorMap m64, m256;
-    if (!encode_rows_map(&m64, gu ? h->xp : h->h16, p.K, P, 64) ||
+    CUtensorMap m16, m64, m256;
+    if (!encode_rows_map(&m16, gu ? h->xp : h->h16, p.K, P, 16) ||
+        !encode_rows_map(&m64, gu ? h->xp : h->h16, p.K, P, 64) ||
         !encode_rows_map(&m256, gu ? h->xp : h->h16, p.K, P, 256))
       return STRATA_ERR_CUDA;
     auto kern = h->fmt == kFmtInt4
@@ -283,7 +284,7 @@ strata_status run_tc_passes(strata_moe *h, int T, const ExpertTable &table, bool
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
       e = launch(h, gu ? PH_GATEUP : PH_DOWN, kern, dim3(h->num_sms), dim3(tc_threads()), smem,
-                 stream, true, p, m64, m256);
+                 stream, true, p, m16, m64, m256);
     if (e != cudaSuccess) return cuda_status(e);
   }
   return STRATA_OK;
