@@ -13,19 +13,19 @@
 // microseconds to stream, while each extra launch costs a few microseconds of
 // launch, prologue and tail.  Here the grid is one CTA per multiprocessor,
 // all resident at once (cooperative launch), and the phases are separated by
-// grid barriers: device counters, each CTA's writes released by a fence
-// before its increment and acquired after it (the relaxed-only hand-off of
-// the fused Metal router in "Strata on a Mac", "Switches", is the failure
-// this ordering avoids).  Every wait is bounded; a wait that gives up sets
-// STATUS_TIMEOUT and the CTA winds down, still passing every barrier so that
-// no other CTA waits on it.
+// grid barriers: device counters, each CTA's writes released by a release
+// reduction on the counter and acquired by the waiter's acquire loads (the
+// relaxed-only hand-off of the fused Metal router in "Strata on a Mac",
+// "Switches", is the failure this ordering avoids).  Every wait is bounded;
+// a wait that gives up sets STATUS_TIMEOUT and the CTA winds down, still
+// passing every barrier so that no other CTA waits on it.
 //
 // Phases:
 //  R  every CTA packs a slice of x to f16 (range-checked); the router's
 //     dot products are cut into units (expert, range of H) spread over every
 //     CTA, each storing double partial sums.  Barrier.
 //  K  logits = the units' partial sums added in a fixed order + bias, one
-//     rounding to fp32; top-k: for up to 12 tokens every CTA selects all
+//     rounding to fp32; top-k: for up to 16 tokens every CTA selects all
 //     tokens itself (one warp per token, the same inputs and code, so the
 //     same result everywhere); for more tokens CTA c selects token c and a
 //     second barrier publishes the choices.
@@ -38,11 +38,13 @@
 //     barrier.
 // G and D cut their (item, K group) sequences -- item = (active expert, <= 8
 // or 16 of its pairs, one 16-row weight tile) -- into one equal contiguous
-// share per warp of the grid.  Each warp streams its shares through its own
-// ring of shared-memory stages filled by bulk async copies; the ring runs on
-// from the G share into the D share, so the down weights are in flight while
-// the grid waits at the barrier between the phases.  The int4 words go from
-// shared memory into mma.m16n8k16 A fragments.  int4: int4x8_to_f16 (exact
+// share per warp of the grid, cut at whole ring stages.  Each warp streams
+// its shares through its own ring of shared-memory stages filled by bulk
+// async copies (lane 0: packed weights and scales, completing as transaction
+// bytes on the stage's mbarrier); the ring runs on from the G share into the
+// D share, so the first down weights are in flight while the warp waits for
+// its first pair group.  The int4 words go from shared memory into
+// mma.m16n8k16 A fragments.  int4: int4x8_to_f16 (exact
 // integers), two MMAs per quant block, fp32 block-scale FMAs.  NVFP4: each
 // code times its E4M3 group scale in f16 (exact: at most six significant
 // bits, at most 2688 in magnitude), MMAs chained over the whole piece, and
@@ -739,7 +741,7 @@ __global__ void __launch_bounds__(kFW * 32, 1) decode_fused_kernel(FusedParams p
   const bool routed_given = p.idx_in != nullptr;
   // Router: unit = (expert e, split sp), sp covering a range of the H/128
   // chunks; splits = grid / E (at least 1) so that small E still uses every
-  // CTA.  A unit's 12 warps take its chunks round-robin, each lane 4
+  // CTA.  A unit's warps (the CTA's) take its chunks round-robin, each lane 4
   // consecutive elements; per token a lane's products are summed in double
   // in chunk order, the 32 lanes reduced by one transpose-reduction, the
   // warps added in warp order, and the unit's partial sum stored.
