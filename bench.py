@@ -61,7 +61,7 @@ NOMINAL_HBM_GBS = 8000.0   # the HBM figure the targets are stated against
 def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=HEADLINE[0], choices=sorted(synth.CONFIGS))
@@ -69,7 +69,7 @@ def parse(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-subrecords", action="store_true",
                     help="only the headline workload (profiler runs)")
-    ap.add_argument("--sub-steps", type=int, default=200, help="timed steps per sub-record")
+    ap.add_argument("--sub-steps", type=int, default=1000, help="timed steps per sub-record")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args(argv)
     if a.tokens is None:
