@@ -21,10 +21,12 @@
 //               activation rows (f16, 128-byte swizzle; x_perm or h16) in one
 //               256-row TMA box, or in 64-row and 16-row boxes for shorter
 //               chunks;
-//   MMA: allocates all 512 TMEM columns (two 256-column accumulators), and
-//               one thread issues 4 tcgen05.mma (M=128, N=chunk pairs rounded
-//               up to 16, K=16) per atom and chunk, commits to the operand
-//               stages and, at the end of a unit, to the accumulators it used;
+//   MMA (two warps): the first allocates all 512 TMEM columns (two
+//               256-column accumulators); one thread of each issues the
+//               tcgen05.mma (M=128, N=chunk pairs rounded up to 16, K=16; 4
+//               per atom and chunk) of the chunks that use its accumulator,
+//               commits to the operand stages and, at the end of a unit, to
+//               its accumulator;
 //   8 dequant warps: load their rows' packed weights and scales straight
 //               from global memory (one K group ahead; dequant warp 0 brings
 //               the weights of the units ahead into L2 by bulk prefetches),
@@ -37,8 +39,6 @@
 //               32-column blocks: tcgen05.ld, SwiGLU (gate/up; the gate lane
 //               and its up partner each compute one column of every pair) or
 //               plain (down), transposed through shared memory, stored;
-//   one more warp has no role (it kept a ring of packed weights in shared
-//               memory, which now goes to the activation ring).
 // The A operand (16 KB per atom) and the B operand (32 KB per atom and
 // chunk) have rings of their own (three and five stages) with one "full" and
 // one "empty" mbarrier per stage: the kernel is bound by the hand-offs
@@ -92,19 +92,19 @@ __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *statu
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// Warp roles.  A warp issues from the scheduler of warp id % 4; the single
-// thread that issues every MMA gets scheduler 1 with only warps that mostly
-// sleep (two epilogue warps, the producer, the warp with no role), while the dequant warps, the
+// Warp roles.  A warp issues from the scheduler of warp id % 4; the two
+// MMA-issuing warps get scheduler 1 with only warps that mostly sleep (two
+// epilogue warps and the activation producer), while the dequant warps, the
 // busiest, share schedulers 0, 2 and 3 with the other epilogue warps.  An
 // epilogue warp may only read its own TMEM lane quarter (warp id % 4).
-enum TcRole : int { kRoleAct, kRoleMma, kRoleDq, kRoleEpi, kRoleIdle };
+enum TcRole : int { kRoleAct, kRoleMma, kRoleDq, kRoleEpi };
 struct TcWarp {
-  int role, idx;  // idx: dequant warp 0..7, or epilogue warp 0..7 (= 2 quarter + half)
+  int role, idx;  // idx: MMA warp 0..1, dequant warp 0..7, or epilogue warp 0..7
 };
 __device__ __forceinline__ TcWarp tc_warp(int warp) {
   switch (warp) {
     case 1: return {kRoleMma, 0};
-    case 13: return {kRoleIdle, 0};
+    case 13: return {kRoleMma, 1};
     case 17: return {kRoleAct, 0};
     case 0: return {kRoleDq, 0};
     case 4: return {kRoleDq, 1};
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAStages; ++s) {
       mbar_init(&fullA[s], kDqWarps);
-      mbar_init(&emptyA[s], 1);
+      mbar_init(&emptyA[s], 2);   // one arrival per MMA-issuing thread
     }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&fullB[s], 1);
@@ -312,14 +312,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (uint32_t m = issued > kBStages ? issued - kBStages : 0; m < issued; ++m)
         (void)wwait(&fullB[m % kBStages], (m / kBStages) & 1u, p.status);
     }
-  } else if (role.role == kRoleIdle) {
-    // -------------------------------------------------------- (no role)
   } else if (role.role == kRoleMma) {
     // -------------------------------------------------------- MMA issue
-    // One thread does it all: per atom one wait for A, per chunk one wait for
-    // B, four MMAs and one commit, so the tensor pipe's queue never runs dry
-    // behind warp-level overheads.
+    // Two issuing threads (role index 0 and 1), each owning one accumulator:
+    // the chunk that uses accumulator i is issued by thread i (both chunks of
+    // a two-chunk unit at once; a one-chunk unit by the owner of the
+    // accumulator it takes in turn).  Per atom each waits for A, the owner of
+    // a chunk for its B stage, issues four MMAs and commits the B stage; both
+    // then release the A stage (its empty barrier counts two arrivals: a
+    // commit from a thread that issued MMAs, a plain arrival from one that
+    // did not).  Both walk every unit and atom, so their ring positions and
+    // accumulator use counts agree with the producers' and the epilogue's.
     if (lane == 0) {
+      const int me = role.idx;
       RingPos ra, rb;
       AccTrack acc;
       bool ok = true;
@@ -328,43 +333,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // field, a 16-element K step (32 bytes) adds 2
       const uint64_t a_desc0 = umma_desc_sw128(smem_u32(smem + kOffA));
       const uint64_t b_desc0 = umma_desc_sw128(smem_u32(smem + kOffB));
+      const uint32_t d_tmem = tmem_base + me * kAccCols;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const Unit un = decode(u, a);
         const int nc = un.chunks();
-        uint32_t idesc[2], d_tmem[2];
-        int bufs[2];
-        for (int c = 0; c < nc; ++c) {
-          bufs[c] = acc.buf_of(nc, c);
-          idesc[c] = umma_idesc_f16(kTcM, (un.chunk_n(c) + 15) & ~15);
-          d_tmem[c] = tmem_base + bufs[c] * kAccCols;
-        }
+        int mine = -1;   // the chunk this thread issues, if any
+        for (int c = 0; c < nc; ++c)
+          if (acc.buf_of(nc, c) == me) mine = c;
+        const uint32_t idesc = mine >= 0 ? umma_idesc_f16(kTcM, (un.chunk_n(mine) + 15) & ~15) : 0u;
         for (int at = 0; at < 2 * G && ok; ++at) {
           if (!mbar_wait(&fullA[ra.st], ra.ph, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = a_desc0 + (uint64_t)((ra.st * kAStageBytes) >> 4);
           for (int c = 0; c < nc; ++c) {
-            if (at == 0) {
-              // the accumulator must have been drained by the epilogue
-              const int b = bufs[c];
-              if (!mbar_wait(&acc_empty[b], (acc.uses[b] & 1u) ^ 1u, p.status)) { ok = false; break; }
+            if (c == mine) {
+              if (at == 0) {
+                // the accumulator must have been drained by the epilogue
+                if (!mbar_wait(&acc_empty[me], (acc.uses[me] & 1u) ^ 1u, p.status)) { ok = false; break; }
+                tc_fence_after();
+              }
+              if (!mbar_wait(&fullB[rb.st], rb.ph, p.status)) { ok = false; break; }
               tc_fence_after();
+              const uint64_t bd = b_desc0 + (uint64_t)((rb.st * kBStageBytes) >> 4);
+              umma_f16(d_tmem, ad, bd, idesc, at > 0 ? 1u : 0u);
+              umma_f16(d_tmem, ad + 2, bd + 2, idesc, 1u);
+              umma_f16(d_tmem, ad + 4, bd + 4, idesc, 1u);
+              umma_f16(d_tmem, ad + 6, bd + 6, idesc, 1u);
+              umma_commit(&emptyB[rb.st]);
             }
-            if (!mbar_wait(&fullB[rb.st], rb.ph, p.status)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t bd = b_desc0 + (uint64_t)((rb.st * kBStageBytes) >> 4);
-            umma_f16(d_tmem[c], ad, bd, idesc[c], at > 0 ? 1u : 0u);
-            umma_f16(d_tmem[c], ad + 2, bd + 2, idesc[c], 1u);
-            umma_f16(d_tmem[c], ad + 4, bd + 4, idesc[c], 1u);
-            umma_f16(d_tmem[c], ad + 6, bd + 6, idesc[c], 1u);
-            umma_commit(&emptyB[rb.st]);
             rb.next(kBStages);
           }
           if (!ok) break;
-          umma_commit(&emptyA[ra.st]);
+          if (mine >= 0) umma_commit(&emptyA[ra.st]);
+          else mbar_arrive(&emptyA[ra.st]);
           ra.next(kAStages);
         }
         if (!ok) break;
-        for (int c = 0; c < nc; ++c) umma_commit(&acc_full[bufs[c]]);
+        if (mine >= 0) umma_commit(&acc_full[me]);
         acc.done_unit(nc);
       }
     }
