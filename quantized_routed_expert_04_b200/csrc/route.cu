@@ -29,10 +29,12 @@ namespace strata {
 // fp32 at the end; the order of the fp64 additions differs from a plain
 // ascending loop, which moves a logit by at most about 1e-11 relative before
 // that rounding.  8 warps as 4 (tokens) x 2 (experts), each 32 x 32 = 4 x 4
-// tiles of 8 x 8; K staged 16 at a time in shared memory as doubles, the
-// next K slice prefetched into registers during the MMAs.
+// tiles of 8 x 8; K staged 16 at a time in shared memory (as fp32, exact for
+// both operands, widened to fp64 when the fragments are read), two stages so
+// that one barrier per slice suffices, the next slice prefetched into
+// registers during the MMAs.
 constexpr int kRT = 128, kRE = 64, kRK = 16;
-constexpr int kRXL = kRT + 8, kRWL = kRE + 8;   // padded rows (2-way bank spread)
+constexpr int kRXL = kRT + 8, kRWL = kRE + 8;   // padded rows: conflict-free fragment reads
 
 __device__ __forceinline__ void dmma_8x8x4(double &d0, double &d1, double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
@@ -44,8 +46,8 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
     const __nv_bfloat16 *__restrict__ x, const float *__restrict__ W,
     const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits) {
   grid_dependency_wait();
-  __shared__ double xs[kRK][kRXL];
-  __shared__ double ws[kRK][kRWL];
+  __shared__ float xs[2][kRK][kRXL];
+  __shared__ float ws[2][kRK][kRWL];
   const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wt = (warp & 3) * 32, we = (warp >> 2) * 32;   // warp tile origin in the block
@@ -59,6 +61,19 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
   float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
   if (x_ok) xv = *reinterpret_cast<const uint4 *>(xp);
   if (w_ok) wv = *reinterpret_cast<const float4 *>(wp);
+  auto stage = [&](int b) {
+    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xv);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(h2[q]);
+      xs[b][xc + 2 * q][xr] = f.x;
+      xs[b][xc + 2 * q + 1][xr] = f.y;
+    }
+    ws[b][wc + 0][wr] = wv.x;
+    ws[b][wc + 1][wr] = wv.y;
+    ws[b][wc + 2][wr] = wv.z;
+    ws[b][wc + 3][wr] = wv.w;
+  };
 
   double acc[4][4][2];
 #pragma unroll
@@ -66,22 +81,12 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
 
+  stage(0);
+  __syncthreads();
+  int buf = 0;
   for (int k0 = 0; k0 < H; k0 += kRK) {
-    {
-      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&xv);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(h2[q]);
-        xs[xc + 2 * q][xr] = (double)f.x;
-        xs[xc + 2 * q + 1][xr] = (double)f.y;
-      }
-      ws[wc + 0][wr] = (double)wv.x;
-      ws[wc + 1][wr] = (double)wv.y;
-      ws[wc + 2][wr] = (double)wv.z;
-      ws[wc + 3][wr] = (double)wv.w;
-    }
-    __syncthreads();
-    if (k0 + kRK < H) {
+    const bool more = k0 + kRK < H;
+    if (more) {
       if (x_ok) xv = *reinterpret_cast<const uint4 *>(xp + k0 + kRK);
       if (w_ok) wv = *reinterpret_cast<const float4 *>(wp + k0 + kRK);
     }
@@ -89,15 +94,18 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
     for (int kk = 0; kk < kRK; kk += 4) {
       double a[4], b[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[kk + (lane & 3)][wt + 8 * i + (lane >> 2)];
+      for (int i = 0; i < 4; ++i) a[i] = (double)xs[buf][kk + (lane & 3)][wt + 8 * i + (lane >> 2)];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = ws[kk + (lane & 3)][we + 8 * j + (lane >> 2)];
+      for (int j = 0; j < 4; ++j) b[j] = (double)ws[buf][kk + (lane & 3)][we + 8 * j + (lane >> 2)];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
     }
+    // the other stage was last read before the previous barrier
+    if (more) stage(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
   // lane holds rows (lane >> 2) and columns 2 (lane & 3) + {0, 1} of each tile
 #pragma unroll
