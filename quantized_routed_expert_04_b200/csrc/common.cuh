@@ -143,6 +143,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *s
   }
 }
 
+// Read-only global loads that bypass L1 allocation (data read once per SM).
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *ptr) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ uint2 ldg_nc_v2(const void *ptr) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(ptr));
+  return v;
+}
+
 // ---------------------------------------------------------------- bulk copy
 // Hint: bring `bytes` (a multiple of 16, 16-byte aligned source) into L2 ahead
 // of the copies that will read them; no completion to wait for.

@@ -15,35 +15,39 @@
 // (one MMA N each); every dequantised weight atom feeds both chunks, so an
 // expert with many pairs pays the dequantisation once per 512 pairs.
 //
-// Warp roles (one CTA per SM, persistent; units interleaved over CTAs):
-//   warp 0      activation producer: per 64 K elements (one swizzle atom)
-//               and chunk, the activation rows (f16, 128-byte swizzle; x_perm
-//               or h16) in one 256-row TMA box, or in up to three 64-row
-//               boxes for shorter chunks;
-//   last warp   weight producer: per two K groups (of 128) one bulk copy per
-//               blob tile of packed weights and one of scales;
-//   warp 1      MMA: allocates all 512 TMEM columns (two 256-column
-//               accumulators), and one thread issues 4 tcgen05.mma (M=128,
-//               N=chunk pairs rounded up to 16, K=16) per atom and chunk,
-//               commits to the operand stages and, at the end of a unit, to
-//               the accumulators it used;
-//   warps 2-9   dequant: int4 -> exact f16 integers -> times the fp16 scale
-//               (one f16 rounding), or NVFP4 E2M1 codes times their E4M3
-//               group scale (exact in f16; the fp32 global scale multiplies
-//               the accumulator in the epilogue) -> the K-major
-//               128-byte-swizzled A layout;
-//   warps 10-17 epilogue: two warps per TMEM lane quarter, each taking
-//               alternate 32-column blocks: tcgen05.ld, SwiGLU (gate/up; the
-//               gate lane and its up partner each compute every other
-//               column) or plain (down), transposed through shared memory,
-//               stored.
+// Warp roles (one CTA per SM, persistent; units interleaved over CTAs; the
+// warp ids of each role are in tc_warp below):
+//   activation producer: per 64 K elements (one swizzle atom) and chunk, the
+//               activation rows (f16, 128-byte swizzle; x_perm or h16) in one
+//               256-row TMA box, or in 64-row and 16-row boxes for shorter
+//               chunks;
+//   MMA: allocates all 512 TMEM columns (two 256-column accumulators), and
+//               one thread issues 4 tcgen05.mma (M=128, N=chunk pairs rounded
+//               up to 16, K=16) per atom and chunk, commits to the operand
+//               stages and, at the end of a unit, to the accumulators it used;
+//   8 dequant warps: load their rows' packed weights and scales straight
+//               from global memory (one K group ahead; dequant warp 0 brings
+//               the weights of the units ahead into L2 by bulk prefetches),
+//               int4 -> exact f16 integers -> times the fp16 scale (one f16
+//               rounding), or NVFP4 E2M1 codes times their E4M3 group scale
+//               (exact in f16; the fp32 global scale multiplies the
+//               accumulator in the epilogue) -> the K-major 128-byte-swizzled
+//               A layout, 16 rows each;
+//   8 epilogue warps: two per TMEM lane quarter, each taking alternate
+//               32-column blocks: tcgen05.ld, SwiGLU (gate/up; the gate lane
+//               and its up partner each compute one column of every pair) or
+//               plain (down), transposed through shared memory, stored;
+//   one more warp has no role (it kept a ring of packed weights in shared
+//               memory, which now goes to the activation ring).  One thread
+//               issues all MMAs: a variant with a second issuing thread (one
+//               per accumulator) faulted once and is not used.
 // The A operand (16 KB per atom) and the B operand (32 KB per atom and
-// chunk) have rings of their own (three and four stages) with one "full" and
-// one "empty" mbarrier per stage.  A unit of two chunks uses both
-// accumulators; a unit of one chunk uses the next one in turn, so the
-// epilogue of a unit overlaps the MMAs of the next.  The copy engine's
-// per-operation cost, not bytes, limits this kernel when copies are small,
-// so both producers move few, large pieces.
+// chunk) have rings of their own (three and five stages) with one "full" and
+// one "empty" mbarrier per stage: the kernel is bound by the hand-offs
+// between its roles, and the depth of the activation ring, in stages, is what
+// counts most.  A unit of two chunks uses both accumulators; a unit of one
+// chunk uses the next one in turn, so the epilogue of a unit overlaps the MMAs
+// of the next.
 // Every wait is bounded; on a timeout the status word is set and the roles
 // wind down (the producers let their issued copies land; the allocating warp
 // still frees the tensor memory).
@@ -59,11 +63,9 @@ namespace {
 constexpr int kTcM = 128;          // weight rows per unit
 constexpr int kTcN = 256;          // pairs per chunk (max MMA N used)
 constexpr int kUnitPairs = 2 * kTcN;
-constexpr int kPkStages = 2;       // packed-weight stages
 constexpr int kPfUnits = 2;        // units whose weights are prefetched into L2 ahead
-constexpr int kPkGroups = 2;       // K groups (of 128) per packed stage
 constexpr int kAStages = 3;        // A ring: one 64-wide dequantised atom each
-constexpr int kBStages = 4;        // B ring: one 64-wide activation atom of one chunk each
+constexpr int kBStages = 5;        // B ring: one 64-wide activation atom of one chunk each
 constexpr int kDqWarps = 8;
 constexpr int kDqRows = kTcM / kDqWarps;    // weight rows per dequant warp
 static_assert(kDqRows % 8 == 0, "dequant warps cover whole 8-row groups");
@@ -75,17 +77,13 @@ constexpr uint32_t kTmemCols = 512;
 
 constexpr int kAStageBytes = kTcM * 128;               // one 64-wide atom
 constexpr int kBStageBytes = kTcN * 128;
-constexpr int kPkQBytes = 8 * kPkGroups * 1024;        // 8 blob tiles
-constexpr int kPkSBytes = 8 * kPkGroups * 128;
-constexpr int kPkStageBytes = kPkQBytes + kPkSBytes;
 constexpr int kEpiBytes = kEpiWarps * 1024;            // per epilogue warp: 1 KB
 
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kAStages * kAStageBytes;
-constexpr int kOffPk = kOffB + kBStages * kBStageBytes;
-constexpr int kOffEpi = kOffPk + kPkStages * kPkStageBytes;
+constexpr int kOffEpi = kOffB + kBStages * kBStageBytes;
 constexpr int kOffBar = kOffEpi + kEpiBytes;
-constexpr int kNumBars = 2 * kPkStages + 2 * kAStages + 2 * kBStages + 4;
+constexpr int kNumBars = 2 * kAStages + 2 * kBStages + 4;
 constexpr int kOffTab = kOffBar + kNumBars * 8 + 16;   // + TMEM address slot
 constexpr int kTabBytes = kMaxIds * 8 + (3 * kMaxIds + 1) * 4;
 constexpr int kTcSmem = kOffTab + kTabBytes + 1024;    // + alignment slack
@@ -98,17 +96,17 @@ __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *statu
 
 // Warp roles.  A warp issues from the scheduler of warp id % 4; the single
 // thread that issues every MMA gets scheduler 1 with only warps that mostly
-// sleep (two epilogue warps, both producers), while the dequant warps, the
+// sleep (two epilogue warps, the producer, the warp with no role), while the dequant warps, the
 // busiest, share schedulers 0, 2 and 3 with the other epilogue warps.  An
 // epilogue warp may only read its own TMEM lane quarter (warp id % 4).
-enum TcRole : int { kRoleAct, kRoleMma, kRoleDq, kRoleEpi, kRoleWgt };
+enum TcRole : int { kRoleAct, kRoleMma, kRoleDq, kRoleEpi, kRoleIdle };
 struct TcWarp {
   int role, idx;  // idx: dequant warp 0..7, or epilogue warp 0..7 (= 2 quarter + half)
 };
 __device__ __forceinline__ TcWarp tc_warp(int warp) {
   switch (warp) {
     case 1: return {kRoleMma, 0};
-    case 13: return {kRoleWgt, 0};
+    case 13: return {kRoleIdle, 0};
     case 17: return {kRoleAct, 0};
     case 0: return {kRoleDq, 0};
     case 4: return {kRoleDq, 1};
@@ -186,10 +184,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  uint64_t *pk_full = bars, *pk_empty = pk_full + kPkStages;
   // fullA[s]: the dequant warps' arrivals; fullB[s]: the activation TMA bytes;
   // emptyA/emptyB[s]: the MMAs that read stage s have completed
-  uint64_t *fullA = pk_empty + kPkStages, *emptyA = fullA + kAStages;
+  uint64_t *fullA = bars, *emptyA = fullA + kAStages;
   uint64_t *fullB = emptyA + kAStages, *emptyB = fullB + kBStages;
   uint64_t *acc_full = emptyB + kBStages, *acc_empty = acc_full + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
@@ -201,10 +198,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const TcWarp role = tc_warp(warp);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPkStages; ++s) {
-      mbar_init(&pk_full[s], 1);
-      mbar_init(&pk_empty[s], kDqWarps);
-    }
     for (int s = 0; s < kAStages; ++s) {
       mbar_init(&fullA[s], kDqWarps);
       mbar_init(&emptyA[s], 1);
@@ -321,47 +314,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (uint32_t m = issued > kBStages ? issued - kBStages : 0; m < issued; ++m)
         (void)wwait(&fullB[m % kBStages], (m / kBStages) & 1u, p.status);
     }
-  } else if (role.role == kRoleWgt) {
-    // -------------------------------------------------------- weight producer
-    uint32_t pk_cnt = 0;
-    bool ok = true;
-    int a = 0, a_pf = 0;
-    // the packed weights of a unit stream in from HBM through this small
-    // ring; L2 prefetches of the units ahead hide their latency
-    auto prefetch_unit = [&](int v) {
-      if (v >= n_units || lane >= 8) return;
-      const Unit nx = decode(v, a_pf);
-      const int tile = nx.rt * 8 + lane;
-      bulk_prefetch_l2(nx.blob + p.q_off + (size_t)tile * G * 1024, (uint32_t)G * 1024u);
-      bulk_prefetch_l2(nx.blob + p.s_off + (size_t)tile * G * 128, (uint32_t)G * 128u);
-    };
-    for (int i = 0; i < kPfUnits; ++i) prefetch_unit(blockIdx.x + i * gridDim.x);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit un = decode(u, a);
-      prefetch_unit(u + kPfUnits * gridDim.x);
-      for (int g = 0; g < G && ok; g += kPkGroups) {
-        const int s = (int)(pk_cnt % kPkStages);
-        if (!wwait(&pk_empty[s], ((pk_cnt / kPkStages) & 1u) ^ 1u, p.status)) { ok = false; break; }
-        ++pk_cnt;
-        const int ng = min(kPkGroups, G - g);
-        uint8_t *dst = smem + kOffPk + s * kPkStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(&pk_full[s], 8u * ng * (1024u + 128u));
-        __syncwarp();
-        if (lane < 8) {
-          const int tile = un.rt * 8 + lane;
-          const size_t g0 = (size_t)tile * G + g;
-          bulk_g2s(dst + lane * (kPkGroups * 1024), un.blob + p.q_off + g0 * 1024, ng * 1024u,
-                   &pk_full[s]);
-          bulk_g2s(dst + kPkQBytes + lane * (kPkGroups * 128), un.blob + p.s_off + g0 * 128,
-                   ng * 128u, &pk_full[s]);
-        }
-        __syncwarp();
-      }
-    }
-    if (!ok) {
-      for (uint32_t m = pk_cnt > kPkStages ? pk_cnt - kPkStages : 0; m < pk_cnt; ++m)
-        (void)wwait(&pk_full[m % kPkStages], (m / kPkStages) & 1u, p.status);
-    }
+  } else if (role.role == kRoleIdle) {
+    // -------------------------------------------------------- (no role)
   } else if (role.role == kRoleMma) {
     // -------------------------------------------------------- MMA issue
     // One thread does it all: per atom one wait for A, per chunk one wait for
@@ -423,30 +377,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int w = lane & 3;
     const int q = lane >> 2;
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
-    uint32_t pk_cnt = 0;
     RingPos ra;
     bool ok = true, big_scale = false;
+    int a = 0, a_pf = 0;
+    // warp 0 of the dequant role brings the weights of the units ahead into
+    // L2 (one bulk prefetch per blob tile and section)
+    auto prefetch_unit = [&](int v) {
+      if (dw != 0 || v >= n_units || lane >= 8) return;
+      const Unit nx = decode(v, a_pf);
+      const int tile = nx.rt * 8 + lane;
+      bulk_prefetch_l2(nx.blob + p.q_off + (size_t)tile * G * 1024, (uint32_t)G * 1024u);
+      bulk_prefetch_l2(nx.blob + p.s_off + (size_t)tile * G * 128, (uint32_t)G * 128u);
+    };
+    for (int i = 0; i < kPfUnits; ++i) prefetch_unit(blockIdx.x + i * gridDim.x);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit un = decode(u, a);
+      prefetch_unit(u + kPfUnits * gridDim.x);
+      // this warp's 16 rows are blob tile 8 rt + dw; per K group, row tr holds
+      // 64 bytes of packed weights (word w of each 32-element block: bytes
+      // 16 w .. 16 w + 15 for the group's four blocks) and 8 bytes of scales
+      const uint8_t *gq = un.blob + p.q_off + (size_t)(un.rt * 8 + dw) * G * 1024;
+      const uint8_t *gs = un.blob + p.s_off + (size_t)(un.rt * 8 + dw) * G * 128;
+      uint4 qn[kDqRows / 8];
+      uint2 sn[kDqRows / 8];
+#pragma unroll
+      for (int m = 0; m < kDqRows / 8; ++m) {
+        const int tr = 8 * m + row_in_8;
+        qn[m] = ldg_nc_v4(gq + tr * 64 + w * 16);
+        sn[m] = ldg_nc_v2(gs + tr * 8);
+      }
       for (int g = 0; g < G && ok; ++g) {
-        const int ps = (int)(pk_cnt % kPkStages);
-        if (g % kPkGroups == 0)
-          if (!wwait(&pk_full[ps], (pk_cnt / kPkStages) & 1u, p.status)) { ok = false; break; }
-        const uint8_t *pq = smem + kOffPk + ps * kPkStageBytes;
-        const uint8_t *psc = pq + kPkQBytes;
-        const int gi = g % kPkGroups;
+        uint4 qc[kDqRows / 8];
+        uint2 scur[kDqRows / 8];
+#pragma unroll
+        for (int m = 0; m < kDqRows / 8; ++m) {
+          qc[m] = qn[m];
+          scur[m] = sn[m];
+        }
+        if (g + 1 < G) {
+#pragma unroll
+          for (int m = 0; m < kDqRows / 8; ++m) {
+            const int tr = 8 * m + row_in_8;
+            qn[m] = ldg_nc_v4(gq + (size_t)(g + 1) * 1024 + tr * 64 + w * 16);
+            sn[m] = ldg_nc_v2(gs + (size_t)(g + 1) * 128 + tr * 8);
+          }
+        }
         for (int atom = 0; atom < 2 && ok; ++atom) {
           if (!wwait(&emptyA[ra.st], ra.ph ^ 1u, p.status)) { ok = false; break; }
           uint8_t *ad = smem + kOffA + ra.st * kAStageBytes;
 #pragma unroll
           for (int m = 0; m < kDqRows / 8; ++m) {
             const int r = kDqRows * dw + 8 * m + row_in_8;
-            const int j = r >> 4, tr = r & 15;
             // blocks 2 atom and 2 atom + 1 of this row: word w of each
-            const uint2 qv = *reinterpret_cast<const uint2 *>(
-                pq + j * (kPkGroups * 1024) + gi * 1024 + tr * 64 + w * 16 + atom * 8);
-            const uint32_t sv = *reinterpret_cast<const uint32_t *>(
-                psc + j * (kPkGroups * 128) + gi * 128 + tr * 8 + atom * 4);
-            const uint32_t words[2] = {qv.x, qv.y};
+            const uint32_t words[2] = {atom ? qc[m].z : qc[m].x, atom ? qc[m].w : qc[m].y};
+            const uint32_t sv = atom ? scur[m].y : scur[m].x;
             if (FMT == kFmtInt4) {
               // |scale| >= 8192 (or not finite): q * scale can overflow f16
               big_scale |= __vcmpgeu2(sv & 0x7FFF7FFFu, 0x70007000u) != 0u;
@@ -489,10 +473,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ra.next(kAStages);
         }
         if (!ok) break;
-        if (gi == kPkGroups - 1 || g == G - 1) {
-          if (lane == 0) mbar_arrive(&pk_empty[ps]);
-          ++pk_cnt;
-        }
       }
     }
     if (__any_sync(0xffffffffu, big_scale) && lane == 0) set_status(p.status, STATUS_RANGE);
