@@ -15,6 +15,25 @@
 // (one MMA N each); every dequantised weight atom feeds both chunks, so an
 // expert with many pairs pays the dequantisation once per 512 pairs.
 //
+// Swapped unit = (expert whose last block has <= 128 pairs, 256 weight rows),
+// for int4 blobs whose 128-row tiles pair up: the operands trade places.  The
+// block's activations are the MMA's A (M = 128 rows; rows past the pairs are
+// ignored) and 256 dequantised weight rows its B (N = 256): one MMA covers
+// 256 weight rows where the other form needs two M = 128 MMAs whose cost
+// hardly depends on N (M = 64 when the block has <= 64 pairs).  The
+// accumulator then holds one pair per TMEM lane and one weight row per
+// column.  Each output element is the same K-ordered sum of the same products
+// in every form, and comes out bit for bit the same.
+// Every CTA runs its plain units first, then its swapped ones (phase 2), in
+// which the two rings' shared memory trades roles: activations in the
+// three 16 KB stages, weights in the five 32 KB ones (a swapped atom's 256
+// rows need a stage that size, and the weight ring's depth is what limits
+// these units).  Each ring has one producer role in each phase (a ring
+// filled by two roles that skip each other's positions would let one run
+// two laps ahead, which a phase-parity wait cannot tell apart); phase 2 has
+// barriers of its own, and its producers start once every MMA of phase 1
+// has completed.
+//
 // Warp roles (one CTA per SM, persistent; units interleaved over CTAs; the
 // warp ids of each role are in tc_warp below):
 //   activation producer: per 64 K elements (one swizzle atom) and chunk, the
@@ -63,6 +82,8 @@ namespace {
 constexpr int kTcM = 128;          // weight rows per unit
 constexpr int kTcN = 256;          // pairs per chunk (max MMA N used)
 constexpr int kUnitPairs = 2 * kTcN;
+constexpr int kSwapPairs = kTcM;   // swapped unit: at most this many pairs (MMA M) ...
+constexpr int kSwapRows = kTcN;    // ... and this many weight rows (MMA N)
 constexpr int kPfUnits = 2;        // units whose weights are prefetched into L2 ahead
 constexpr int kAStages = 3;        // A ring: one 64-wide dequantised atom each
 constexpr int kBStages = 5;        // B ring: one 64-wide activation atom of one chunk each
@@ -83,9 +104,9 @@ constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kAStages * kAStageBytes;
 constexpr int kOffEpi = kOffB + kBStages * kBStageBytes;
 constexpr int kOffBar = kOffEpi + kEpiBytes;
-constexpr int kNumBars = 2 * kAStages + 2 * kBStages + 4;
+constexpr int kNumBars = 2 * (2 * kAStages + 2 * kBStages) + 5;
 constexpr int kOffTab = kOffBar + kNumBars * 8 + 16;   // + TMEM address slot
-constexpr int kTabBytes = kMaxIds * 8 + (3 * kMaxIds + 1) * 4;
+constexpr int kTabBytes = kMaxIds * 8 + (4 * kMaxIds + 2) * 4;
 constexpr int kTcSmem = kOffTab + kTabBytes + 1024;    // + alignment slack
 
 __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *status) {
@@ -128,9 +149,15 @@ __device__ __forceinline__ TcWarp tc_warp(int warp) {
 }
 static_assert(kTcWarps == 19 && kDqWarps == 8 && kEpiWarps == 8, "role table");
 
+template <int N>
+struct IntTag {
+  static constexpr int value = N;
+};
+
 struct Unit {
   const uint8_t *blob;
-  int pi0, n, rt;
+  int pi0, n, rt;  // rt: 128-row tile, or 256-row tile of a swapped unit
+  bool sw;
   __device__ __forceinline__ int chunks() const { return n > kTcN ? 2 : 1; }
   __device__ __forceinline__ int chunk_n(int c) const { return c == 0 ? min(n, kTcN) : n - kTcN; }
 };
@@ -184,16 +211,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  // fullA[s]: the dequant warps' arrivals; fullB[s]: the activation TMA bytes;
-  // emptyA/emptyB[s]: the MMAs that read stage s have completed
+  // phase 1 (plain units): fullA[s]: the dequant warps' arrivals; fullB[s]:
+  // the activation TMA bytes; emptyA/emptyB[s]: the MMAs that read stage s
+  // have completed.  Phase 2 (swapped units), on the same shared memory:
+  // fullX/emptyX for the activations in the A stages, fullW/emptyW for the
+  // weights in the B stages.  p1_done: every MMA of phase 1 has completed.
   uint64_t *fullA = bars, *emptyA = fullA + kAStages;
   uint64_t *fullB = emptyA + kAStages, *emptyB = fullB + kBStages;
-  uint64_t *acc_full = emptyB + kBStages, *acc_empty = acc_full + 2;
+  uint64_t *fullX = emptyB + kBStages, *emptyX = fullX + kAStages;
+  uint64_t *fullW = emptyX + kAStages, *emptyW = fullW + kBStages;
+  uint64_t *acc_full = emptyW + kBStages, *acc_empty = acc_full + 2;
+  uint64_t *p1_done = acc_empty + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + kNumBars);
   const uint8_t **t_blob = reinterpret_cast<const uint8_t **>(smem + kOffTab);
   int *t_off = reinterpret_cast<int *>(t_blob + kMaxIds);
   int *t_cnt = t_off + kMaxIds;
-  int *unit_base = t_cnt + kMaxIds;
+  int *unit_base = t_cnt + kMaxIds;        // plain units, prefix over experts
+  int *swap_base = unit_base + kMaxIds + 1;  // swapped units, prefix
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const TcWarp role = tc_warp(warp);
@@ -206,10 +240,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&fullB[s], 1);
       mbar_init(&emptyB[s], 1);
     }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&fullX[s], 1);
+      mbar_init(&emptyX[s], 1);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&fullW[s], kDqWarps);
+      mbar_init(&emptyW[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], kEpiWarps);
     }
+    mbar_init(p1_done, 1);
     fence_mbar_init();
     prefetch_tmap(&tmap_b16);
     prefetch_tmap(&tmap_b64);
@@ -236,34 +279,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  if (warp == 0) {
+  // swapped units need the 128-row tiles to pair up; they are used for int4
+  // blobs (the NVFP4 dequant of two tiles per warp would not fit in the
+  // registers this block size leaves)
+  constexpr bool kSwapFmt = FMT == kFmtInt4;
+  const bool can_swap = kSwapFmt && (p.row_tiles & 1) == 0;
+  // an expert's last block of pairs goes to swapped units if it is that short
+  auto last_swapped = [&](int cnt) {
+    return can_swap && cnt - ((cnt - 1) / kUnitPairs) * kUnitPairs <= kSwapPairs;
+  };
+  if (warp < 2) {
+    // warp 0: plain units per expert (row_tiles per block of 512 pairs but a
+    // swapped last block); warp 1: swapped units (row_tiles / 2 or none)
+    int *base = warp == 0 ? unit_base : swap_base;
     int carry = 0;
     for (int a0 = 0; a0 < n_active; a0 += 32) {
       const int a = a0 + lane;
-      const int v = a < n_active && t_blob[a]
-                        ? ((t_cnt[a] + kUnitPairs - 1) / kUnitPairs) * p.row_tiles : 0;
+      int v = 0;
+      if (a < n_active && t_blob[a] && t_cnt[a] > 0) {
+        const int nb = (t_cnt[a] + kUnitPairs - 1) / kUnitPairs;
+        const bool sl = last_swapped(t_cnt[a]);
+        v = warp == 0 ? (nb - (sl ? 1 : 0)) * p.row_tiles : (sl ? p.row_tiles / 2 : 0);
+      }
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int nb = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += nb;
       }
-      if (a < n_active) unit_base[a] = carry + incl - v;
+      if (a < n_active) base[a] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) unit_base[n_active] = carry;
+    if (lane == 0) base[n_active] = carry;
   }
   __syncthreads();
   grid_dependency_launch();
 
-  const int n_units = unit_base[n_active];
+  // units 0 .. n_plain - 1 are plain, the rest swapped
+  const int n_plain = unit_base[n_active];
+  const int n_units = n_plain + swap_base[n_active];
   const int G = p.K / 128;  // K groups
-  auto decode = [&](int u, int &a) -> Unit {
-    while (unit_base[a + 1] <= u) ++a;
-    const int rem = u - unit_base[a];
-    const int ub = rem / p.row_tiles;
+  // one cursor per phase over the active experts (units are walked in order)
+  struct Cursor {
+    int a = 0, b = 0;
+  };
+  auto decode = [&](int u, Cursor &cur) -> Unit {
     Unit un;
-    un.rt = rem - ub * p.row_tiles;
+    int a, ub;
+    if (!kSwapFmt || u < n_plain) {
+      while (unit_base[cur.a + 1] <= u) ++cur.a;
+      a = cur.a;
+      const int rem = u - unit_base[a];
+      ub = rem / p.row_tiles;
+      un.rt = rem - ub * p.row_tiles;
+      un.sw = false;
+    } else {
+      const int v = u - n_plain;
+      while (swap_base[cur.b + 1] <= v) ++cur.b;
+      a = cur.b;
+      ub = (t_cnt[a] - 1) / kUnitPairs;  // the last block
+      un.rt = v - swap_base[a];
+      un.sw = true;
+    }
     un.pi0 = t_off[a] + ub * kUnitPairs;
     un.n = min(kUnitPairs, t_cnt[a] - ub * kUnitPairs);
     un.blob = t_blob[a];
@@ -272,47 +349,64 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (role.role == kRoleAct) {
     // -------------------------------------------------------- activation producer
-    uint32_t issued = 0;
-    RingPos rb;
-    bool ok = true;
-    int a = 0;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit un = decode(u, a);
+    uint32_t issued_b = 0, issued_x = 0;  // copies into the B stages, the A stages
+    RingPos rb, rx;
+    bool ok = true, phase2 = false;
+    Cursor cur;
+    // a unit's activation rows, per 64 K elements (one swizzle atom) and
+    // chunk: one 256-row box, else 64-row boxes and 16-row boxes for the rest
+    // (rows land at 128 bytes each whatever the box, so the swizzled layout
+    // is the same)
+    auto produce = [&](const Unit &un, uint64_t *full, uint64_t *empty, RingPos &r, uint32_t stages,
+                       uint8_t *ring, int stage_bytes, uint32_t &issued) {
       const int nc = un.chunks();
       for (int at = 0; at < 2 * G && ok; ++at) {
         for (int c = 0; c < nc; ++c) {
-          if (!wwait(&emptyB[rb.st], rb.ph ^ 1u, p.status)) { ok = false; break; }
+          if (!wwait(&empty[r.st], r.ph ^ 1u, p.status)) { ok = false; break; }
           const int cn = un.chunk_n(c), row0 = un.pi0 + c * kTcN;
-          // one 256-row box, else 64-row boxes and 16-row boxes for the rest
-          // (rows land at 128 bytes each whatever the box, so the swizzled
-          // layout is the same)
           const bool wide = cn > 192;
           const int n64 = wide ? 0 : cn / 64;
           const int n16 = wide ? 0 : (cn - 64 * n64 + 15) / 16;
           const uint32_t tx = wide ? 32768u : n64 * 8192u + n16 * 2048u;
-          uint8_t *dst = smem + kOffB + rb.st * kBStageBytes;
+          uint8_t *dst = ring + r.st * stage_bytes;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&fullB[rb.st], tx);
+            mbar_arrive_expect_tx(&full[r.st], tx);
             if (wide) {
-              tma_load_2d(dst, &tmap_b256, at * 64, row0, &fullB[rb.st]);
+              tma_load_2d(dst, &tmap_b256, at * 64, row0, &full[r.st]);
             } else {
               for (int q = 0; q < n64; ++q)
-                tma_load_2d(dst + q * 8192, &tmap_b64, at * 64, row0 + q * 64, &fullB[rb.st]);
+                tma_load_2d(dst + q * 8192, &tmap_b64, at * 64, row0 + q * 64, &full[r.st]);
               for (int q = 0; q < n16; ++q)
                 tma_load_2d(dst + n64 * 8192 + q * 2048, &tmap_b16, at * 64, row0 + 64 * n64 + 16 * q,
-                            &fullB[rb.st]);
+                            &full[r.st]);
             }
           }
           __syncwarp();
           ++issued;
-          rb.next(kBStages);
+          r.next(stages);
         }
       }
+    };
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit un = decode(u, cur);
+      if (!un.sw) {
+        produce(un, fullB, emptyB, rb, kBStages, smem + kOffB, kBStageBytes, issued_b);
+        continue;
+      }
+      // swapped (<= 128 rows, one chunk) into the A stages, once the weights
+      // that phase 1 kept there have been read
+      if (!phase2) {
+        phase2 = true;
+        if (!wwait(p1_done, 0u, p.status)) { ok = false; break; }
+      }
+      produce(un, fullX, emptyX, rx, kAStages, smem + kOffA, kAStageBytes, issued_x);
     }
     if (!ok) {
       // let issued copies land before the CTA exits (bounded waits)
-      for (uint32_t m = issued > kBStages ? issued - kBStages : 0; m < issued; ++m)
+      for (uint32_t m = issued_b > kBStages ? issued_b - kBStages : 0; m < issued_b; ++m)
         (void)wwait(&fullB[m % kBStages], (m / kBStages) & 1u, p.status);
+      for (uint32_t m = issued_x > kAStages ? issued_x - kAStages : 0; m < issued_x; ++m)
+        (void)wwait(&fullX[m % kAStages], (m / kAStages) & 1u, p.status);
     }
   } else if (role.role == kRoleIdle) {
     // -------------------------------------------------------- (no role)
@@ -322,16 +416,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // B, four MMAs and one commit, so the tensor pipe's queue never runs dry
     // behind warp-level overheads.
     if (lane == 0) {
-      RingPos ra, rb;
+      RingPos ra, rb, rx, rw;
       AccTrack acc;
-      bool ok = true;
-      int a = 0;
+      bool ok = true, phase2 = false;
+      Cursor cur;
       // stage 0's descriptors; a stage adds its offset / 16 to the address
       // field, a 16-element K step (32 bytes) adds 2
       const uint64_t a_desc0 = umma_desc_sw128(smem_u32(smem + kOffA));
       const uint64_t b_desc0 = umma_desc_sw128(smem_u32(smem + kOffB));
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const Unit un = decode(u, a);
+        const Unit un = decode(u, cur);
+        if (un.sw) {
+          if (!phase2) {
+            // the producers of phase 2 reuse the stages once these complete
+            phase2 = true;
+            umma_commit(p1_done);
+          }
+          // A: the block's activations (A stages), B: 256 weight rows (B stages)
+          const int buf = acc.buf_of(1, 0);
+          const uint32_t id = umma_idesc_f16(un.n <= 64 ? 64 : kSwapPairs, kSwapRows);
+          const uint32_t dt = tmem_base + buf * kAccCols;
+          if (!mbar_wait(&acc_empty[buf], (acc.uses[buf] & 1u) ^ 1u, p.status)) { ok = false; break; }
+          tc_fence_after();
+          for (int at = 0; at < 2 * G; ++at) {
+            if (!mbar_wait(&fullW[rw.st], rw.ph, p.status) ||
+                !mbar_wait(&fullX[rx.st], rx.ph, p.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = a_desc0 + (uint64_t)((rx.st * kAStageBytes) >> 4);
+            const uint64_t bd = b_desc0 + (uint64_t)((rw.st * kBStageBytes) >> 4);
+            umma_f16(dt, ad, bd, id, at > 0 ? 1u : 0u);
+            umma_f16(dt, ad + 2, bd + 2, id, 1u);
+            umma_f16(dt, ad + 4, bd + 4, id, 1u);
+            umma_f16(dt, ad + 6, bd + 6, id, 1u);
+            umma_commit(&emptyX[rx.st]);
+            umma_commit(&emptyW[rw.st]);
+            rx.next(kAStages);
+            rw.next(kBStages);
+          }
+          if (!ok) break;
+          umma_commit(&acc_full[buf]);
+          acc.done_unit(1);
+          continue;
+        }
         const int nc = un.chunks();
         uint32_t idesc[2], d_tmem[2];
         int bufs[2];
@@ -377,57 +503,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int w = lane & 3;
     const int q = lane >> 2;
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
-    RingPos ra;
-    bool ok = true, big_scale = false;
-    int a = 0, a_pf = 0;
+    RingPos ra, rw;
+    bool ok = true, big_scale = false, phase2 = false;
+    Cursor cur, cur_pf;
     // warp 0 of the dequant role brings the weights of the units ahead into
     // L2 (one bulk prefetch per blob tile and section)
     auto prefetch_unit = [&](int v) {
-      if (dw != 0 || v >= n_units || lane >= 8) return;
-      const Unit nx = decode(v, a_pf);
-      const int tile = nx.rt * 8 + lane;
+      if (dw != 0 || v >= n_units) return;
+      const Unit nx = decode(v, cur_pf);
+      const int ntiles = nx.sw ? kSwapRows / 16 : kTcM / 16;
+      if (lane >= ntiles) return;
+      const int tile = nx.rt * ntiles + lane;
       bulk_prefetch_l2(nx.blob + p.q_off + (size_t)tile * G * 1024, (uint32_t)G * 1024u);
       bulk_prefetch_l2(nx.blob + p.s_off + (size_t)tile * G * 128, (uint32_t)G * 128u);
     };
-    for (int i = 0; i < kPfUnits; ++i) prefetch_unit(blockIdx.x + i * gridDim.x);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit un = decode(u, a);
-      prefetch_unit(u + kPfUnits * gridDim.x);
-      // this warp's 16 rows are blob tile 8 rt + dw; per K group, row tr holds
-      // 64 bytes of packed weights (word w of each 32-element block: bytes
-      // 16 w .. 16 w + 15 for the group's four blocks) and 8 bytes of scales
-      const uint8_t *gq = un.blob + p.q_off + (size_t)(un.rt * 8 + dw) * G * 1024;
-      const uint8_t *gs = un.blob + p.s_off + (size_t)(un.rt * 8 + dw) * G * 128;
-      uint4 qn[kDqRows / 8];
-      uint2 sn[kDqRows / 8];
+    // One unit into one ring: per 64 K, an atom of 128 rows (NA = 1) or of
+    // 256 (NA = 2, a swapped unit: row tiles 2 rt and 2 rt + 1, one below the
+    // other).  This warp's 16 rows of half j are blob tile tile0 + 8 j; per K
+    // group, tile row tr holds 64 bytes of packed weights (word w of each
+    // 32-element block: bytes 16 w .. 16 w + 15 for the group's four blocks)
+    // and 8 bytes of scales.
+    auto dq_unit = [&](const Unit &un, auto na_tag, uint64_t *full, uint64_t *empty, RingPos &r,
+                       uint32_t stages, uint8_t *ring, int stage_bytes) {
+      constexpr int NA = decltype(na_tag)::value;
+      constexpr int NM = NA * (kDqRows / 8);  // groups of 8 rows; half m / 2
+      const int tile0 = un.rt * 8 * NA + dw;
+      const uint8_t *gq = un.blob + p.q_off + (size_t)tile0 * G * 1024;
+      const uint8_t *gs = un.blob + p.s_off + (size_t)tile0 * G * 128;
+      auto q_at = [&](int m, int g) {
+        return gq + ((size_t)(m >> 1) * 8 * G + g) * 1024 + (8 * (m & 1) + row_in_8) * 64 + w * 16;
+      };
+      auto s_at = [&](int m, int g) {
+        return gs + ((size_t)(m >> 1) * 8 * G + g) * 128 + (8 * (m & 1) + row_in_8) * 8;
+      };
+      uint4 qn[NM];
+      uint2 sn[NM];
 #pragma unroll
-      for (int m = 0; m < kDqRows / 8; ++m) {
-        const int tr = 8 * m + row_in_8;
-        qn[m] = ldg_nc_v4(gq + tr * 64 + w * 16);
-        sn[m] = ldg_nc_v2(gs + tr * 8);
+      for (int m = 0; m < NM; ++m) {
+        qn[m] = ldg_nc_v4(q_at(m, 0));
+        sn[m] = ldg_nc_v2(s_at(m, 0));
       }
       for (int g = 0; g < G && ok; ++g) {
-        uint4 qc[kDqRows / 8];
-        uint2 scur[kDqRows / 8];
+        uint4 qc[NM];
+        uint2 scur[NM];
 #pragma unroll
-        for (int m = 0; m < kDqRows / 8; ++m) {
+        for (int m = 0; m < NM; ++m) {
           qc[m] = qn[m];
           scur[m] = sn[m];
         }
         if (g + 1 < G) {
 #pragma unroll
-          for (int m = 0; m < kDqRows / 8; ++m) {
-            const int tr = 8 * m + row_in_8;
-            qn[m] = ldg_nc_v4(gq + (size_t)(g + 1) * 1024 + tr * 64 + w * 16);
-            sn[m] = ldg_nc_v2(gs + (size_t)(g + 1) * 128 + tr * 8);
+          for (int m = 0; m < NM; ++m) {
+            qn[m] = ldg_nc_v4(q_at(m, g + 1));
+            sn[m] = ldg_nc_v2(s_at(m, g + 1));
           }
         }
         for (int atom = 0; atom < 2 && ok; ++atom) {
-          if (!wwait(&emptyA[ra.st], ra.ph ^ 1u, p.status)) { ok = false; break; }
-          uint8_t *ad = smem + kOffA + ra.st * kAStageBytes;
+          if (!wwait(&empty[r.st], r.ph ^ 1u, p.status)) { ok = false; break; }
+          uint8_t *ad = ring + r.st * stage_bytes;
 #pragma unroll
-          for (int m = 0; m < kDqRows / 8; ++m) {
-            const int r = kDqRows * dw + 8 * m + row_in_8;
+          for (int m = 0; m < NM; ++m) {
+            // row of the operand: half m / 2, this warp's 16 rows of it
+            const int rr = kTcM * (m >> 1) + kDqRows * dw + 8 * (m & 1) + row_in_8;
             // blocks 2 atom and 2 atom + 1 of this row: word w of each
             const uint32_t words[2] = {atom ? qc[m].z : qc[m].x, atom ? qc[m].w : qc[m].y};
             const uint32_t sv = atom ? scur[m].y : scur[m].x;
@@ -445,8 +582,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 o.y = h2_bits(__hmul2(bits_h2(f[1]), sc[b]));
                 o.z = h2_bits(__hmul2(bits_h2(f[2]), sc[b]));
                 o.w = h2_bits(__hmul2(bits_h2(f[3]), sc[b]));
-                const int chunk = (b * 4 + w) ^ (r & 7);
-                *reinterpret_cast<uint4 *>(ad + r * 128 + chunk * 16) = o;
+                const int chunk = (b * 4 + w) ^ (rr & 7);
+                *reinterpret_cast<uint4 *>(ad + rr * 128 + chunk * 16) = o;
               }
             } else {
               // NVFP4: word w of block 2 atom + b is scale group 4 atom + 2 b
@@ -462,18 +599,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 o.y = h2_bits(__hmul2(bits_h2(f[1]), z));
                 o.z = h2_bits(__hmul2(bits_h2(f[2]), z));
                 o.w = h2_bits(__hmul2(bits_h2(f[3]), z));
-                const int chunk = (b * 4 + w) ^ (r & 7);
-                *reinterpret_cast<uint4 *>(ad + r * 128 + chunk * 16) = o;
+                const int chunk = (b * 4 + w) ^ (rr & 7);
+                *reinterpret_cast<uint4 *>(ad + rr * 128 + chunk * 16) = o;
               }
             }
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&fullA[ra.st]);
-          ra.next(kAStages);
+          if (lane == 0) mbar_arrive(&full[r.st]);
+          r.next(stages);
         }
-        if (!ok) break;
       }
+    };
+    for (int i = 0; i < kPfUnits; ++i) prefetch_unit(blockIdx.x + i * gridDim.x);
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit un = decode(u, cur);
+      prefetch_unit(u + kPfUnits * gridDim.x);
+      if (!un.sw) {
+        dq_unit(un, IntTag<1>{}, fullA, emptyA, ra, kAStages, smem + kOffA, kAStageBytes);
+        continue;
+      }
+      // swapped: 256 rows into the B stages, once phase 1's activations
+      // there have been read
+      if (!phase2) {
+        phase2 = true;
+        if (!wwait(p1_done, 0u, p.status)) { ok = false; break; }
+      }
+      dq_unit(un, IntTag<2>{}, fullW, emptyW, rw, kBStages, smem + kOffB, kBStageBytes);
     }
     if (__any_sync(0xffffffffu, big_scale) && lane == 0) set_status(p.status, STATUS_RANGE);
   } else {
@@ -484,9 +636,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float *stage = reinterpret_cast<float *>(smem + kOffEpi + ew * 1024);
     AccTrack acc;
     bool ok = true, big_h = false;
-    int a = 0;
+    Cursor cur;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit un = decode(u, a);
+      const Unit un = decode(u, cur);
+      if (un.sw) {
+        // lane L of quarter qd: pair 32 qd + L of the block (M = 128); column c: weight
+        // row c of the unit's 256, i.e. blob tile 16 rt + c / 16, tile row
+        // c % 16 (for gate/up: gate if < 8, its up partner at c + 8)
+        const int buf = acc.buf_of(1, 0);
+        if (!wwait(&acc_full[buf], acc.uses[buf] & 1u, p.status)) { ok = false; break; }
+        tc_fence_after();
+        // M = 64: rows 16 qd .. 16 qd + 15 in lanes 0..15 of quarter qd
+        const bool m64 = un.n <= 64;
+        const int row = m64 ? 16 * qd + (lane & 15) : 32 * qd + lane;
+        const bool mine = row < un.n && (!m64 || lane < 16);
+        for (int col0 = 32 * cpar; col0 < kSwapRows && (m64 ? 16 : 32) * qd < un.n; col0 += 64) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * qd) << 16) + buf * kAccCols + col0, v);
+          if (kGateUp) {
+            // blob tiles 16 rt + col0 / 16 + b: h columns 8 x that tile + the
+            // packed position of the tile row
+            __half hh[16];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float gv = v[16 * b + i], uv = v[16 * b + 8 + i];
+                const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+                big_h |= mine && fabsf(hv) >= kF16Overflow;
+                hh[8 * b + packed_pos<FMT>(i)] = __float2half_rn(hv);
+              }
+            }
+            if (mine) {
+              uint32_t hw[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) hw[k] = h2_bits(__halves2half2(hh[2 * k], hh[2 * k + 1]));
+              uint4 *dst = reinterpret_cast<uint4 *>(p.h_out + (size_t)(un.pi0 + row) * p.out_ld +
+                                                     kTcM * un.rt + col0 / 2);
+              dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            }
+          } else if (mine) {
+            float4 *dst = reinterpret_cast<float4 *>(p.y_out + (size_t)(un.pi0 + row) * p.out_ld +
+                                                     kSwapRows * un.rt + col0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        acc.done_unit(1);
+        continue;
+      }
       const int nc = un.chunks();
       // NVFP4: this lane's row's global scale (gate, up or down)
       float gsc = 1.0f;

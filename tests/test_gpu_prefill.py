@@ -129,6 +129,47 @@ def test_tc_routed_only_binding_bitwise(T):
     lay.close()
 
 
+def test_tc_swapped_and_plain_units_bitwise():
+    """An expert's last block of <= 128 pairs goes to swapped units (the
+    pairs' activations as the MMA's A, with M = 64 for <= 64 pairs, 256 weight
+    rows as its B), other blocks to plain ones (128 weight rows as A, the pairs
+    as B); a token's output must not depend on which.  Tokens are routed to
+    four experts (and the shared one): an 80-token batch whose halves use
+    different experts runs swapped units of M = 64 (40 pairs each) and of
+    M = 128 (the shared expert), a 100-token batch swapped units of M = 128, a
+    300-token batch plain ones only, and a 600-token batch a plain block of
+    512 pairs and a swapped block of 88: the same tokens give the same bits
+    in each.  (Batches of <= 64 tokens take the other kernel.)"""
+    cfg = synth.custom_config("forms", 512, 256, 16, 4, n_shared=1, tokens=(600,))
+    lay = GpuLayer(cfg)
+    x = synth.make_x(cfg, 600, step=21)
+    idx = np.tile(np.array([[3, 0, 9, 5]], np.int32), (600, 1))
+    w = np.random.default_rng(7).dirichlet(np.ones(4), size=600).astype(np.float32)
+    idx80 = idx[:80].copy()
+    idx80[40:] = [1, 2, 4, 6]
+    st, e80 = lay.forward_routed(x[:80], idx80, w[:80])
+    assert int(st[0]) == 0, st
+    st, a100 = lay.forward_routed(x[:100], idx[:100], w[:100])
+    assert int(st[0]) == 0, st
+    st, b300 = lay.forward_routed(x[:300], idx[:300], w[:300])
+    assert int(st[0]) == 0, st
+    st, c600 = lay.forward_routed(x, idx, w)
+    assert int(st[0]) == 0, st
+    assert np.array_equal(e80[:40], b300[:40])
+    assert np.array_equal(a100, b300[:100])
+    assert np.array_equal(b300, c600[:300])
+    # tokens 512..599: swapped in the 600-token batch, plain in this one
+    mix = np.concatenate([np.arange(512, 600), np.arange(0, 212)])
+    st, d300 = lay.forward_routed(x[mix], idx[mix], w[mix])
+    assert int(st[0]) == 0, st
+    assert np.array_equal(d300[:88], c600[512:600])
+    ref, _, _ = oracle_reference(cfg, lay.blobs, lay.W, lay.b, x, idx, w)
+    assert_within_tolerance(c600, ref, "swapped and plain units")
+    ref, _, _ = oracle_reference(cfg, lay.blobs, lay.W, lay.b, x[:80], idx80, w[:80])
+    assert_within_tolerance(e80, ref, "swapped units of M = 64")
+    lay.close()
+
+
 def test_tc_two_runs_bitwise_equal():
     cfg = mid_config(2048)
     lay = GpuLayer(cfg)
