@@ -45,8 +45,8 @@
 //               up to 16, K=16) per atom and chunk, commits to the operand
 //               stages and, at the end of a unit, to the accumulators it used;
 //   8 dequant warps: load their rows' packed weights and scales straight
-//               from global memory (one K group ahead; dequant warp 0 brings
-//               the weights of the units ahead into L2 by bulk prefetches),
+//               from global memory, one K group ahead (an L2 prefetch of the
+//               units ahead only evicted lines before their loads),
 //               int4 -> exact f16 integers -> times the fp16 scale (one f16
 //               rounding), or NVFP4 E2M1 codes times their E4M3 group scale
 //               (exact in f16; the fp32 global scale multiplies the
@@ -84,7 +84,6 @@ constexpr int kTcN = 256;          // pairs per chunk (max MMA N used)
 constexpr int kUnitPairs = 2 * kTcN;
 constexpr int kSwapPairs = kTcM;   // swapped unit: at most this many pairs (MMA M) ...
 constexpr int kSwapRows = kTcN;    // ... and this many weight rows (MMA N)
-constexpr int kPfUnits = 2;        // units whose weights are prefetched into L2 ahead
 constexpr int kAStages = 3;        // A ring: one 64-wide dequantised atom each
 constexpr int kBStages = 5;        // B ring: one 64-wide activation atom of one chunk each
 constexpr int kDqWarps = 8;
@@ -109,10 +108,24 @@ constexpr int kOffTab = kOffBar + kNumBars * 8 + 16;   // + TMEM address slot
 constexpr int kTabBytes = kMaxIds * 8 + (4 * kMaxIds + 2) * 4;
 constexpr int kTcSmem = kOffTab + kTabBytes + 1024;    // + alignment slack
 
+// A warp's wait for a barrier phase: one test by every lane and a vote (no
+// divergent branch when the phase is already complete, the common case),
+// else lane 0 waits with the time limit and tells the others.
 __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, int *status) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// One arrival for the whole (converged) warp, made by the lane elect.sync
+// picks as a predicated instruction rather than under a divergent branch.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 // Warp roles.  A warp issues from the scheduler of warp id % 4; the single
@@ -505,18 +518,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int row_in_8 = (q & 1) * 4 + (q >> 1);  // lanes 8p..8p+7 -> rows p and p + 4
     RingPos ra, rw;
     bool ok = true, big_scale = false, phase2 = false;
-    Cursor cur, cur_pf;
-    // warp 0 of the dequant role brings the weights of the units ahead into
-    // L2 (one bulk prefetch per blob tile and section)
-    auto prefetch_unit = [&](int v) {
-      if (dw != 0 || v >= n_units) return;
-      const Unit nx = decode(v, cur_pf);
-      const int ntiles = nx.sw ? kSwapRows / 16 : kTcM / 16;
-      if (lane >= ntiles) return;
-      const int tile = nx.rt * ntiles + lane;
-      bulk_prefetch_l2(nx.blob + p.q_off + (size_t)tile * G * 1024, (uint32_t)G * 1024u);
-      bulk_prefetch_l2(nx.blob + p.s_off + (size_t)tile * G * 128, (uint32_t)G * 128u);
-    };
+    Cursor cur;
     // One unit into one ring: per 64 K, an atom of 128 rows (NA = 1) or of
     // 256 (NA = 2, a swapped unit: row tiles 2 rt and 2 rt + 1, one below the
     // other).  This warp's 16 rows of half j are blob tile tile0 + 8 j; per K
@@ -606,15 +608,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&full[r.st]);
+          warp_arrive(&full[r.st]);
           r.next(stages);
         }
       }
     };
-    for (int i = 0; i < kPfUnits; ++i) prefetch_unit(blockIdx.x + i * gridDim.x);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit un = decode(u, cur);
-      prefetch_unit(u + kPfUnits * gridDim.x);
       if (!un.sw) {
         dq_unit(un, IntTag<1>{}, fullA, emptyA, ra, kAStages, smem + kOffA, kAStageBytes);
         continue;
@@ -686,7 +686,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        warp_arrive(&acc_empty[buf]);
         acc.done_unit(1);
         continue;
       }
@@ -766,7 +766,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        warp_arrive(&acc_empty[buf]);
       }
       acc.done_unit(nc);
     }
