@@ -560,6 +560,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             sn[m] = ldg_nc_v2(s_at(m, g + 1));
           }
         }
+        if (FMT == kFmtInt4) {
+          // |scale| >= 8192 (or not finite): q * scale can overflow f16
+#pragma unroll
+          for (int m = 0; m < NM; ++m)
+            big_scale |= (__vcmpgeu2(scur[m].x & 0x7FFF7FFFu, 0x70007000u) |
+                          __vcmpgeu2(scur[m].y & 0x7FFF7FFFu, 0x70007000u)) != 0u;
+        }
+#pragma unroll
         for (int atom = 0; atom < 2 && ok; ++atom) {
           if (!wwait(&empty[r.st], r.ph ^ 1u, p.status)) { ok = false; break; }
           uint8_t *ad = ring + r.st * stage_bytes;
@@ -571,8 +579,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t words[2] = {atom ? qc[m].z : qc[m].x, atom ? qc[m].w : qc[m].y};
             const uint32_t sv = atom ? scur[m].y : scur[m].x;
             if (FMT == kFmtInt4) {
-              // |scale| >= 8192 (or not finite): q * scale can overflow f16
-              big_scale |= __vcmpgeu2(sv & 0x7FFF7FFFu, 0x70007000u) != 0u;
               const __half2 sc[2] = {__half2half2(__low2half(bits_h2(sv))),
                                      __half2half2(__high2half(bits_h2(sv)))};
 #pragma unroll
