@@ -471,42 +471,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           acc.done_unit(1);
           continue;
         }
-        const int nc = un.chunks();
-        uint32_t idesc[2], d_tmem[2];
-        int bufs[2];
-        for (int c = 0; c < nc; ++c) {
-          bufs[c] = acc.buf_of(nc, c);
-          idesc[c] = umma_idesc_f16(kTcM, (un.chunk_n(c) + 15) & ~15);
-          d_tmem[c] = tmem_base + bufs[c] * kAccCols;
-        }
-        for (int at = 0; at < 2 * G && ok; ++at) {
-          if (!mbar_wait(&fullA[ra.st], ra.ph, p.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t ad = a_desc0 + (uint64_t)((ra.st * kAStageBytes) >> 4);
-          for (int c = 0; c < nc; ++c) {
-            if (at == 0) {
-              // the accumulator must have been drained by the epilogue
-              const int b = bufs[c];
-              if (!mbar_wait(&acc_empty[b], (acc.uses[b] & 1u) ^ 1u, p.status)) { ok = false; break; }
-              tc_fence_after();
-            }
-            if (!mbar_wait(&fullB[rb.st], rb.ph, p.status)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t bd = b_desc0 + (uint64_t)((rb.st * kBStageBytes) >> 4);
-            umma_f16(d_tmem[c], ad, bd, idesc[c], at > 0 ? 1u : 0u);
-            umma_f16(d_tmem[c], ad + 2, bd + 2, idesc[c], 1u);
-            umma_f16(d_tmem[c], ad + 4, bd + 4, idesc[c], 1u);
-            umma_f16(d_tmem[c], ad + 6, bd + 6, idesc[c], 1u);
-            umma_commit(&emptyB[rb.st]);
-            rb.next(kBStages);
+        // a plain unit of NC chunks (a compile-time count keeps the chunks'
+        // descriptors in registers)
+        auto plain = [&](auto nc_tag) {
+          constexpr int NC = decltype(nc_tag)::value;
+          uint32_t idesc[NC], d_tmem[NC];
+          int bufs[NC];
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
+            bufs[c] = acc.buf_of(NC, c);
+            idesc[c] = umma_idesc_f16(kTcM, (un.chunk_n(c) + 15) & ~15);
+            d_tmem[c] = tmem_base + bufs[c] * kAccCols;
           }
-          if (!ok) break;
-          umma_commit(&emptyA[ra.st]);
-          ra.next(kAStages);
-        }
-        if (!ok) break;
-        for (int c = 0; c < nc; ++c) umma_commit(&acc_full[bufs[c]]);
-        acc.done_unit(nc);
+          for (int at = 0; at < 2 * G && ok; ++at) {
+            if (!mbar_wait(&fullA[ra.st], ra.ph, p.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = a_desc0 + (uint64_t)((ra.st * kAStageBytes) >> 4);
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+              if (at == 0) {
+                // the accumulator must have been drained by the epilogue
+                const int b = bufs[c];
+                if (!mbar_wait(&acc_empty[b], (acc.uses[b] & 1u) ^ 1u, p.status)) { ok = false; break; }
+                tc_fence_after();
+              }
+              if (!mbar_wait(&fullB[rb.st], rb.ph, p.status)) { ok = false; break; }
+              tc_fence_after();
+              const uint64_t bd = b_desc0 + (uint64_t)((rb.st * kBStageBytes) >> 4);
+              umma_f16(d_tmem[c], ad, bd, idesc[c], at > 0 ? 1u : 0u);
+              umma_f16(d_tmem[c], ad + 2, bd + 2, idesc[c], 1u);
+              umma_f16(d_tmem[c], ad + 4, bd + 4, idesc[c], 1u);
+              umma_f16(d_tmem[c], ad + 6, bd + 6, idesc[c], 1u);
+              umma_commit(&emptyB[rb.st]);
+              rb.next(kBStages);
+            }
+            if (!ok) break;
+            umma_commit(&emptyA[ra.st]);
+            ra.next(kAStages);
+          }
+          if (!ok) return;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) umma_commit(&acc_full[bufs[c]]);
+          acc.done_unit(NC);
+        };
+        if (un.chunks() == 2)
+          plain(IntTag<2>{});
+        else
+          plain(IntTag<1>{});
       }
     }
     __syncwarp();
