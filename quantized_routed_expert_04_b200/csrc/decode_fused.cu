@@ -142,11 +142,13 @@ __device__ __forceinline__ int atom_acq_rel_add(int *ptr, int v) {
   return old;
 }
 
-// Ring-stage wait of one warp (lane 0 polls, with the given limit); once the
-// phase is complete every lane observes it itself (acquiring the stage's
-// bytes).
+// Ring-stage wait of one warp: every lane tests the phase and the warp votes
+// (no divergent branch when the stage is ready, the common case); else lane 0
+// polls with the given limit, and once the phase is complete every lane
+// observes it itself (acquiring the stage's bytes).
 __device__ __forceinline__ bool warp_wait_limit(uint64_t *bar, uint32_t parity, int *status,
                                                 unsigned long long limit_ns) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 1;
   if ((threadIdx.x & 31) == 0) {
     if (!mbar_try_wait(bar, parity)) {

@@ -42,8 +42,9 @@
 //               chunks;
 //   MMA: allocates all 512 TMEM columns (two 256-column accumulators), and
 //               one thread issues 4 tcgen05.mma (M=128, N=chunk pairs rounded
-//               up to 16, K=16) per atom and chunk, commits to the operand
-//               stages and, at the end of a unit, to the accumulators it used;
+//               up to 16, K=16) per atom and chunk (swapped: M=64 or 128
+//               pairs, N=256 weight rows), commits to the operand stages and,
+//               at the end of a unit, to the accumulators it used;
 //   8 dequant warps: load their rows' packed weights and scales straight
 //               from global memory, one K group ahead (an L2 prefetch of the
 //               units ahead only evicted lines before their loads),
@@ -51,20 +52,24 @@
 //               rounding), or NVFP4 E2M1 codes times their E4M3 group scale
 //               (exact in f16; the fp32 global scale multiplies the
 //               accumulator in the epilogue) -> the K-major 128-byte-swizzled
-//               A layout, 16 rows each;
+//               layout, 16 rows each of a 128-row atom (swapped: 32 rows,
+//               two blob tiles, of a 256-row atom);
 //   8 epilogue warps: two per TMEM lane quarter, each taking alternate
 //               32-column blocks: tcgen05.ld, SwiGLU (gate/up; the gate lane
 //               and its up partner each compute one column of every pair) or
-//               plain (down), transposed through shared memory, stored;
+//               plain (down), transposed through shared memory, stored (a
+//               swapped unit: each lane holds one pair's row and stores it);
 //   one more warp has no role (it kept a ring of packed weights in shared
 //               memory, which now goes to the activation ring).  One thread
 //               issues all MMAs: a variant with a second issuing thread (one
 //               per accumulator) faulted once and is not used.
-// The A operand (16 KB per atom) and the B operand (32 KB per atom and
-// chunk) have rings of their own (three and five stages) with one "full" and
-// one "empty" mbarrier per stage: the kernel is bound by the hand-offs
+// In phase 1 the A operand (16 KB per atom) and the B operand (32 KB per atom
+// and chunk) have rings of their own (three and five stages) with one "full"
+// and one "empty" mbarrier per stage: the kernel is bound by the hand-offs
 // between its roles, and the depth of the activation ring, in stages, is what
-// counts most.  A unit of two chunks uses both accumulators; a unit of one
+// counts most.  Warps therefore test a barrier on every lane and vote before
+// the bounded single-lane wait, and arrive through an elect.sync-predicated
+// instruction rather than a divergent branch.  A unit of two chunks uses both accumulators; a unit of one
 // chunk uses the next one in turn, so the epilogue of a unit overlaps the MMAs
 // of the next.
 // Every wait is bounded; on a timeout the status word is set and the roles
@@ -162,6 +167,8 @@ __device__ __forceinline__ TcWarp tc_warp(int warp) {
 }
 static_assert(kTcWarps == 19 && kDqWarps == 8 && kEpiWarps == 8, "role table");
 
+// A compile-time int passed as an argument (selects the instance of a
+// generic lambda).
 template <int N>
 struct IntTag {
   static constexpr int value = N;
