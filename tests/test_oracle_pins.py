@@ -103,7 +103,8 @@ def test_down_projection_columns():
 
 
 def test_swiglu_formula():
-    """h = silu(g) * u with silu(z) = z / (1 + e^-z) (spec: SwiGLU)."""
+    """h = silu(g) * u with silu(z) = z / (1 + e^-z): the SwiGLU expert FFN
+    of the W4A16 layer (ro99/strata README, model table)."""
     H, I = 128, 128
     blob, _ = rand_blob(H, I)
     x = synth.bf16_bits_to_f32(bf16(RNG.standard_normal((5, H)) * 4))
