@@ -52,8 +52,14 @@ def _compile(src):
 
 
 def up_to_date() -> bool:
+    """The library exists, is newer than every source, and the ptxas report
+    of each source (which the tests read) is there."""
     if not os.path.exists(LIB):
         return False
+    for src in _sources():
+        name = os.path.splitext(os.path.basename(src))[0]
+        if not os.path.exists(os.path.join(BUILD, "ptxas_%s.log" % name)):
+            return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
